@@ -1,0 +1,390 @@
+"""Pins of the CPU oracle against what the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: values the
+pages print, exact rational arithmetic, library routines (torch casts, SDPA,
+numpy integer matmul), closed forms and invariants.  They are chosen so that a
+plausible slip in the oracle (a wrong rounding mode, a dropped rescale factor,
+a transposed operand, a wrong block index or mask boundary) fails at least one.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import heads
+from tests.exact import all_finite_fp16, fp32, quantize_exact
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, v = line.split("=", 1)
+            out[k.strip()] = [float(t) for t in v.split()]
+    return out
+
+
+# --- quantiser -------------------------------------------------------------------
+
+def test_worked_outlier_example():
+    """The page's worked example: [0.1, 0.2, 0.15, 1000] -> delta ~ 7.87, codes [0,0,0,127]."""
+    g = _golden("p5_outlier_example.txt")
+    A = np.array(g["A"], dtype=np.float32).reshape(1, -1)
+    codes, delta = oracle.quant_block(A)
+    assert codes.ravel().tolist() == [int(c) for c in g["codes"]]
+    assert round(float(delta), int(g["delta_printed_digits"][0])) == g["delta_printed"][0]
+    assert float(delta) == fp32(Fraction(1000) / 127)
+
+
+def test_quantiser_exhaustive_fp16_against_exact_rationals():
+    """Every finite fp16 value, quantised in a block with a seeded max |.|, equals
+    the exact-rational evaluation of the quantiser's binary32 steps."""
+    rng = np.random.default_rng(1)
+    xs = all_finite_fp16().astype(np.float32)
+    ratio = rng.uniform(1.0, 6.0, size=xs.shape).astype(np.float32)
+    for x, r in zip(xs, ratio):
+        ax = abs(float(x))
+        amax = float(np.float16(min(65504.0, ax * float(r)))) if ax > 0 else 1.0
+        amax = max(amax, ax)
+        block = np.array([[x, amax]], dtype=np.float32)
+        codes, delta = oracle.quant_block(block)
+        c_exact, d_exact = quantize_exact(float(x), amax)
+        assert int(codes[0, 0]) == c_exact, (x, amax)
+        assert float(delta) == d_exact
+
+
+def test_quantiser_error_bound_and_page_formula():
+    """|x - code*delta| <= delta*(1/2 + 2^-15), the max element maps to +-127, and
+    codes differ from the page's literal round(x/delta) by at most 1 (rarely)."""
+    rng = np.random.default_rng(2)
+    total = differ = 0
+    for scale in (1e-3, 1.0, 37.0, 3e3):
+        x = (rng.standard_normal((128, 64)) * scale).astype(np.float16).astype(np.float32)
+        codes, delta = oracle.quant_block(x)
+        d = float(delta)
+        err = np.abs(x.astype(np.float64) - codes.astype(np.float64) * d)
+        assert err.max() <= d * (0.5 + 2.0 ** -15)
+        i = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+        assert abs(int(codes[i])) == 127
+        literal = np.rint(x.astype(np.float64) / d)
+        assert np.abs(literal - codes).max() <= 1
+        total += x.size
+        differ += int((literal != codes).sum())
+    assert differ / total < 1e-3
+
+
+def test_integer_block_is_identity():
+    """Integer values with max |.| = 127 give delta = 1 and codes equal to the values."""
+    rng = np.random.default_rng(3)
+    x = rng.integers(-127, 128, size=(128, 128)).astype(np.float32)
+    x[5, 7] = -127.0
+    codes, delta = oracle.quant_block(x)
+    assert float(delta) == 1.0
+    assert np.array_equal(codes.astype(np.float32), x)
+
+
+def test_all_zero_block():
+    codes, delta = oracle.quant_block(np.zeros((128, 64), np.float32))
+    assert float(delta) == 0.0 and not codes.any()
+
+
+def test_quant_head_padding_and_blocks():
+    """Blocks are 128 consecutive tokens; the ragged last block is quantised on its
+    own rows only and the padding rows are zero."""
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((300, 64)).astype(np.float32)
+    x[270, 3] = 50.0                 # outlier only in the last block (rows 256..299)
+    codes, delta = oracle.quant_head(x)
+    assert codes.shape == (384, 64) and delta.shape == (3,)
+    assert not codes[300:].any()
+    for b in range(3):
+        rows = x[b * 128:min(300, (b + 1) * 128)]
+        c, d = oracle.quant_block(rows)
+        assert float(d) == float(delta[b])
+        assert np.array_equal(c, codes[b * 128:b * 128 + rows.shape[0]])
+    assert float(delta[2]) == fp32(Fraction(50) / 127)
+
+
+# --- K mean (smoothing) -------------------------------------------------------------
+
+def test_k_mean_closed_form():
+    """K = c_d + integer noise with zero per-channel sum  =>  mean is exactly c_d."""
+    rng = np.random.default_rng(5)
+    n, D = 1000, 64
+    c = (rng.integers(-200, 200, size=D) / 8.0).astype(np.float32)
+    half = rng.integers(-50, 51, size=(n // 2, D))
+    noise = np.concatenate([half, -half], axis=0)
+    rng.shuffle(noise, axis=0)
+    k = (c[None, :] + noise).astype(np.float16).astype(np.float32)
+    s, m, st = oracle.k_mean(k)
+    assert st == 0
+    assert np.array_equal(m, c)
+    assert np.array_equal(s, (c.astype(np.float64) * n * 2 ** 24).astype(np.int64))
+
+
+def test_k_mean_is_the_mean():
+    """Against the exact rational mean: within one binary32 ulp (fp16 and bf16 data)."""
+    rng = np.random.default_rng(6)
+    for dt in (torch.float16, torch.bfloat16):
+        k = torch.from_numpy(rng.standard_normal((37, 8)).astype(np.float32) * 3 + 1).to(dt)
+        kf = k.float().numpy()
+        _, m, st = oracle.k_mean(kf)
+        assert st == 0
+        for d in range(8):
+            exact = sum(Fraction(float(v)) for v in kf[:, d]) / 37
+            ulp = float(np.spacing(np.float32(float(exact))))
+            assert abs(Fraction(float(m[d])) - exact) <= Fraction(ulp)
+
+
+def test_k_mean_range_flag():
+    k = np.ones((4, 8), np.float32)
+    k[2, 3] = 70000.0
+    _, _, st = oracle.k_mean(k)
+    assert st == oracle.ORACLE_ERR_RANGE
+
+
+# --- number formats ---------------------------------------------------------------
+
+def test_e4m3_against_torch_cast():
+    """Dense sweep of binary32 values in the finite range vs torch.float8_e4m3fn."""
+    rng = np.random.default_rng(7)
+    x = np.concatenate([
+        np.linspace(-464.0, 464.0, 40001, endpoint=False),
+        rng.uniform(-1, 1, 20000) * 2.0 ** rng.integers(-12, 9, 20000),
+        [0.0, -0.0, 2 ** -10, 2 ** -9, 1.5 * 2 ** -9, 2 ** -6, 448.0, -448.0, 464.0 - 2 ** -5],
+    ]).astype(np.float32)
+    ours = oracle.e4m3_encode(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_roundtrip_and_saturation():
+    codes = [c for c in range(256) if (c & 0x7F) != 0x7F]
+    dec = oracle.e4m3_decode(codes)
+    ref = torch.tensor(codes, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(dec, ref)
+    assert np.array_equal(oracle.e4m3_encode(dec.astype(np.float32)), np.array(codes, np.uint8))
+    assert oracle.e4m3_encode([1e6, -500.0]).tolist() == [0x7E, 0xFE]
+
+
+def test_fp16_bf16_rounding_against_torch():
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.uniform(0, 1, 5000), 2.0 ** rng.uniform(-30, 0, 5000),
+                        [2 ** -24, 2 ** -25, 3 * 2 ** -26, 1.0]]).astype(np.float32)
+    for fn, dt in ((oracle.round_fp16, torch.float16), (oracle.round_bf16, torch.bfloat16)):
+        ours = np.array([fn(float(v)) for v in x])
+        ref = torch.from_numpy(x).to(dt).double().numpy()
+        assert np.array_equal(ours, ref)
+
+
+# --- QK^T ----------------------------------------------------------------------------
+
+def test_qk_int_against_numpy_matmul():
+    rng = np.random.default_rng(9)
+    qc = rng.integers(-127, 128, size=(256, 128)).astype(np.int8)
+    kc = rng.integers(-127, 128, size=(256, 128)).astype(np.int8)
+    S = oracle.qk_int(qc, kc, 128, 128, 0, 256)
+    ref = qc[128:256].astype(np.int64) @ kc[0:256].astype(np.int64).T
+    assert np.array_equal(S.astype(np.int64), ref)
+
+
+# --- R: fp64 reference ---------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_reference_against_sdpa(causal):
+    rng = np.random.default_rng(10)
+    n, D = 19, 8
+    q, k, v = (rng.standard_normal((n, D)).astype(np.float32) for _ in range(3))
+    rows = np.arange(n)
+    out = oracle.attn_ref_rows(q, k, v, 0.3, causal, rows)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).double()[None], torch.from_numpy(k).double()[None],
+        torch.from_numpy(v).double()[None], is_causal=causal, scale=0.3)[0].numpy()
+    assert np.abs(out - ref).max() < 1e-12
+
+
+def test_reference_smoothing_invariance():
+    """softmax is unchanged by subtracting a per-channel constant from K."""
+    rng = np.random.default_rng(11)
+    n, D = 64, 16
+    q, k, v = (rng.standard_normal((n, D)).astype(np.float64) for _ in range(3))
+    k = k + rng.standard_normal(D) * 5
+    kbar = k.mean(axis=0)
+    k32 = k.astype(np.float32)
+    ks = (k32.astype(np.float64) - kbar).astype(np.float32)
+    a = oracle.attn_ref_rows(q, k32, v, 0.25, False, np.arange(n))
+    b = oracle.attn_ref_rows(q, ks, v, 0.25, False, np.arange(n))
+    # the only difference is the fp32 rounding of k - kbar (|k| ~ 5, ulp ~ 5e-7)
+    assert np.abs(a - b).max() < 1e-5
+
+
+# --- E: the quantised method ---------------------------------------------------------
+
+def _emulate(q, k, v, causal, pv_mode, sm_scale=None, rows=None):
+    """Run the oracle's own steps over a single-head [1,1,n,D] input."""
+    n, D = q.shape[-2:]
+    qz = heads.quantize(q, k, v, None, pv_mode)
+    rows = list(range(n)) if rows is None else rows
+    picks = [(0, 0, i) for i in rows]
+    out = heads.emulate_rows(qz, v, None, picks, D, causal, pv_mode, sm_scale)
+    return np.stack([out[p] for p in picks]), qz
+
+
+@pytest.mark.parametrize("pv_mode", ["fp16", "fp8"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulation_constant_keys_gives_mean_of_values(causal, pv_mode):
+    """K constant over tokens: smoothing makes K zero, every logit equal, so each
+    output row is the (prefix) mean of the values actually multiplied."""
+    n, D = 333, 64
+    q, k, v = [t[None, None] for t in (torch.randn(n, D), torch.zeros(n, D), torch.randn(n, D))]
+    k = (k + torch.randn(1, 1, 1, D) * 3).half()
+    q, v = q.half(), v.half()
+    out, qz = _emulate(q, k, v, causal, pv_mode)
+    assert not qz.k_codes.any() and not qz.k_delta.any()
+    if pv_mode == "fp16":
+        vals = v[0, 0].double().numpy()
+    else:
+        vals = oracle.e4m3_decode(qz.v_codes[0, 0]).reshape(n, D) * qz.v_delta[0, 0][None, :]
+    if causal:
+        ref = np.cumsum(vals, axis=0) / np.arange(1, n + 1)[:, None]
+    else:
+        ref = np.broadcast_to(vals.mean(axis=0), (n, D))
+    assert np.abs(out - ref).max() < 2e-6 * max(1.0, np.abs(vals).max())
+
+
+@pytest.mark.parametrize("pv_mode", ["fp16", "fp8"])
+def test_emulation_constant_values(pv_mode):
+    """V equal to c_d on every token: every row's output is c_d, up to the P rounding
+    (relative 2^-11 for fp16 P; 2^-4 for e4m3 P; V codes are exact here)."""
+    torch.manual_seed(12)
+    n, D = 300, 64
+    q = torch.randn(1, 1, n, D).half()
+    k = (torch.randn(1, 1, n, D) + 2).half()
+    c = torch.tensor([(-1) ** d * (1 + d / 16) for d in range(D)])
+    v = c.expand(1, 1, n, D).half().contiguous()
+    out, _ = _emulate(q, k, v, False, pv_mode)
+    cd = v[0, 0, 0].double().numpy()
+    tol = 2.0 ** -10 if pv_mode == "fp16" else 2.0 ** -3
+    assert np.abs(out - cd).max() <= tol * np.abs(cd).max()
+
+
+@pytest.mark.parametrize("pv_mode", ["fp16", "fp8"])
+def test_emulation_causal_first_row_is_first_value(pv_mode):
+    torch.manual_seed(13)
+    n, D = 200, 128
+    q, k, v = (torch.randn(1, 1, n, D).half() for _ in range(3))
+    out, qz = _emulate(q, k, v, True, pv_mode, rows=[0])
+    if pv_mode == "fp16":
+        ref = v[0, 0, 0].double().numpy()
+    else:
+        ref = oracle.e4m3_decode(qz.v_codes[0, 0, 0]) * qz.v_delta[0, 0]
+    assert np.abs(out[0] - ref).max() <= 1e-6 * np.abs(ref).max()
+
+
+def _lossless_inputs(n, D, seed, q_exp=(0,), k_exp=(0,)):
+    """q, k whose 128-token blocks are integer codes times a power of two 2^e_b, each
+    block containing the code 127, and whose K blocks have zero channel sums; so
+    deltaQ_b = 2^eq_b, deltaK_b = 2^ek_b exactly, the K mean is 0 and quantisation
+    reproduces the values exactly."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-127, 128, size=(n, D)).astype(np.int64)
+    k = rng.integers(-126, 127, size=(n, D)).astype(np.int64)
+    for bi, b in enumerate(range(0, n, 128)):
+        rows = slice(b, min(n, b + 128))
+        q[b, 0] = 127
+        k[b, 0] = 127
+        kb = k[rows]
+        for d in range(D):
+            s = int(kb[:, d].sum())
+            for r in range(kb.shape[0]):
+                if s == 0:
+                    break
+                if r == 0 and d == 0:
+                    continue
+                step = max(-126 - kb[r, d], min(126 - kb[r, d], -s))
+                kb[r, d] += step
+                s += step
+            assert s == 0
+    qs = np.ones((n, 1)); ks = np.ones((n, 1))
+    for bi, b in enumerate(range(0, n, 128)):
+        qs[b:b + 128] = 2.0 ** q_exp[bi % len(q_exp)]
+        ks[b:b + 128] = 2.0 ** k_exp[bi % len(k_exp)]
+    v = rng.standard_normal((n, D)).astype(np.float16).astype(np.float32)
+    return (q * qs).astype(np.float32), (k * ks).astype(np.float32), v
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulation_lossless_quantisation_matches_reference(causal):
+    """With exactly representable codes the only approximation left in E (16-bit
+    P.V) is rounding P to fp16: |E - R| <= 2^-10 * max|v| (plus fp32 noise).
+    Per-block power-of-two deltas make a wrong block index visible; a transposed
+    operand, missing rescale or mask slip fails as well."""
+    n, D = 300, 16
+    q, k, v = _lossless_inputs(n, D, 14, q_exp=(0, -1, 1), k_exp=(-1, 0, 1))
+    sm = 1.0 / 12000.0
+    qt, kt, vt = (torch.from_numpy(x)[None, None].half() for x in (q, k, v))
+    assert torch.equal(kt.float()[0, 0], torch.from_numpy(k))
+    assert torch.equal(qt.float()[0, 0], torch.from_numpy(q))
+    out, qz = _emulate(qt, kt, vt, causal, "fp16", sm_scale=sm)
+    assert qz.q_delta[0, 0].tolist() == [1.0, 0.5, 2.0]
+    assert qz.k_delta[0, 0].tolist() == [0.5, 1.0, 2.0]
+    assert not qz.k_mean.any()
+    ref = oracle.attn_ref_rows(q, k, v, float(np.float32(sm)), causal, np.arange(n))
+    assert np.abs(out - ref).max() <= 2.0 ** -10 * np.abs(v).max() + 1e-5
+    # the running maximum moves after the first key block for many rows, so the
+    # rescale factor alpha is exercised
+    logits = q.astype(np.float64) @ k.T.astype(np.float64) * sm
+    if not causal:
+        moved = logits[:, :128].max(axis=1) < logits.max(axis=1) - 0.5
+        assert moved.mean() > 0.2
+
+
+def test_v_fp8_quant_against_torch_cast():
+    """Per-channel V scale: delta_d = max_t|v_td|/448 and codes = e4m3(v * 448/max|v|),
+    checked against numpy's per-channel max and torch's float8_e4m3fn cast."""
+    rng = np.random.default_rng(16)
+    v = (rng.standard_normal((333, 64)) * rng.uniform(0.1, 10, 64)).astype(np.float16)
+    v = v.astype(np.float32)
+    v[:, 5] = 0.0
+    codes, delta = oracle.quant_v_fp8(v)
+    amax = np.abs(v).max(axis=0)
+    assert np.array_equal(delta, (amax / np.float32(448)).astype(np.float32))
+    s = np.where(amax > 0, np.float32(448) / np.where(amax > 0, amax, 1), 0).astype(np.float32)
+    ref = torch.from_numpy((v * s[None, :]).astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(codes, ref.view(torch.uint8).numpy())
+
+
+def test_emulation_close_to_reference_on_gaussian_data():
+    """On the smoothing workload recipe, E agrees with R to cosine > 0.9999 (fp16 P)
+    and > 0.999 (fp8 P), and K smoothing is what makes the first one hold."""
+    torch.manual_seed(15)
+    n, D = 384, 64
+    q = torch.randn(1, 1, n, D).half()
+    k = (torch.randn(1, 1, n, D) + torch.randn(1, 1, 1, D) * 4).half()
+    v = torch.randn(1, 1, n, D).half()
+    rows = list(range(0, n, 7))
+    ref = oracle.attn_ref_rows(q[0, 0].float().numpy(), k[0, 0].float().numpy(),
+                               v[0, 0].float().numpy(), 0.125, False, rows)
+    def cos(a):
+        return (a.ravel() @ ref.ravel()) / np.linalg.norm(a) / np.linalg.norm(ref)
+    for mode, bar in (("fp16", 0.9999), ("fp8", 0.999)):
+        out, _ = _emulate(q, k, v, False, mode, rows=rows)
+        assert cos(out) > bar, (mode, cos(out))
+    # the same steps with the smoothing left out fall below the bar
+    qz = heads.quantize(q, k, v, None, "fp16")
+    qz.k_codes[0, 0], qz.k_delta[0, 0] = oracle.quant_head(k[0, 0].float().numpy(), None)
+    picks = [(0, 0, i) for i in rows]
+    o = heads.emulate_rows(qz, v, None, picks, D, False, "fp16")
+    unsmoothed = np.stack([o[p] for p in picks])
+    assert cos(unsmoothed) < 0.9999
