@@ -1,0 +1,225 @@
+/*
+ * sage.h -- C ABI of libsageb200.so: the SageAttention 8-bit attention forward
+ * pass on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources are the SageAttention web pages, cited by page
+ * title and section):
+ *
+ *   - K smoothing: K's per-channel mean over the tokens of each
+ *     (sequence, head) is subtracted before quantisation
+ *     ("SageAttention v1/v2/v2++/v3 overview" (dtcms.com), SageAttention v1,
+ *      bullet 1; "SageAttention -- brand new attention" (postsniper.ru),
+ *      "SageAttention" bullet 1).
+ *   - Per-block INT8 quantisation of Q and smoothed K, 128 tokens x D channels
+ *     per block: delta = max|x| / 127, code = round(x / delta)
+ *     (postsniper.ru page, quantisation intro steps 1-2; dtcms.com page,
+ *      v1 item (1) "per-block").
+ *   - INT8 QK^T on the tensor cores, dequantised by deltaQ * deltaK
+ *     (postsniper.ru page, step 3), fused with the softmax scale.
+ *   - FlashAttention-style tiled online softmax ("Attention机制优化：从
+ *     FlashAttention到SageAttention的工程实践", section 3.1).
+ *   - P.V in 16 bits (postsniper.ru page, "SageAttention" bullet 3), or P and V
+ *     in FP8 E4M3 with the FP8 partial product of every 128-key block flushed
+ *     into an FP32 accumulator (dtcms.com page, SageAttention 2 bullets 1, 3).
+ *   - The drop-in attention call shape q, k, v -> out over [B, H, N, D]
+ *     ("sageattention in DeepSeek-VL2" (deepseek.csdn.net), step 2), plus a
+ *     variable-length packed variant ("SageAttention complete guide"
+ *     (jsqmd.com), API list: sageattn_varlen).
+ *
+ * Conventions for every function below:
+ *   - Pointers are DEVICE pointers unless stated otherwise; the caller owns
+ *     all memory.  The library allocates nothing.  Buffers must be 16-byte
+ *     aligned and densely packed in the stated layout.
+ *   - Compute calls are asynchronous on the given stream (cudaStream_t passed
+ *     as void*; NULL = legacy default stream).  Argument errors are detected on
+ *     the host before anything is launched and returned at once.  Errors found
+ *     on the device (a wait that timed out, inconsistent cu_seqlens, K values
+ *     outside the exact-mean range) are OR-ed into a status word at the start
+ *     of the workspace and reported by sage_sync_status().
+ *   - Workspace: every compute call takes (ws, ws_bytes).  Its first 256 bytes
+ *     hold the status word; sage_workspace_init() must zero them once before
+ *     first use.  Calls on different streams must use different workspaces.
+ *   - Layouts: dense tensors are [B, H, N, D] row-major; varlen tensors are
+ *     [T, H, D] row-major with T = cu_seqlens[batch].  D is 64 or 128.
+ *   - Causal masking is top-left aligned (query i sees keys j <= i), per
+ *     sequence for varlen.
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,   /* bad size, null/misaligned pointer, bad enum   */
+  SAGE_ERR_UNSUPPORTED = 2,   /* valid request this library does not implement */
+  SAGE_ERR_WORKSPACE = 3,     /* ws_bytes smaller than the size function says  */
+  SAGE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed             */
+  SAGE_ERR_TIMEOUT = 5,       /* a device-side wait gave up (status word)      */
+  SAGE_ERR_BAD_SEQLENS = 6,   /* cu_seqlens not monotone / not matching T      */
+  SAGE_ERR_RANGE = 7          /* a K element is non-finite or |k| >= 65536     */
+} sage_status_t;
+
+typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1, SAGE_F32 = 2 /* outputs only */ } sage_dtype_t;
+
+typedef enum {
+  SAGE_PV_FP16 = 0, /* P.V with P rounded to V's 16-bit type, fp32 accumulate   */
+  SAGE_PV_FP8 = 1   /* P, V in FP8 E4M3, per-block fp32 two-level accumulation */
+} sage_pv_mode_t;
+
+/* Token count of one quantisation block and of one attention key/query tile. */
+#define SAGE_BLOCK 128
+
+/* ---------------------------------------------------------------- sizes -- */
+
+/* Workspace bytes for sage_attn_fwd on a dense [B,H,N,D] problem (holds the
+ * status word, the INT8/FP8 codes and scales, and reduction scratch).
+ * Returns 0 for arguments sage_attn_fwd would reject. */
+size_t sage_workspace_bytes(int B, int H, int N, int D, int pv_mode);
+
+/* Workspace bytes for sage_attn_fwd_varlen with `batch` sequences packed into
+ * total_tokens rows.  Sized for the worst case over all length splits. */
+size_t sage_workspace_bytes_varlen(int total_tokens, int batch, int H, int D, int pv_mode);
+
+/* Workspace bytes for sage_quantize / sage_attn_quantized alone (status word
+ * plus reduction scratch; the codes live in caller buffers). */
+size_t sage_scratch_bytes(int B, int H, int D);
+
+/* Zero the status word of a workspace (stream-ordered).  Call once after
+ * allocating a workspace, before its first use. */
+sage_status_t sage_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Wait for `stream`, then read and clear the workspace's status word.
+ * Returns SAGE_OK or the first device-side error recorded since the last
+ * call, in the precedence TIMEOUT > BAD_SEQLENS > RANGE. */
+sage_status_t sage_sync_status(void* ws, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* sage_status_string(sage_status_t s);
+
+/* Message of the last CUDA failure that made a call on this host thread
+ * return SAGE_ERR_CUDA (thread-local, static storage; "" if none). */
+const char* sage_last_cuda_error(void);
+
+/* ------------------------------------------------------ full forward pass -- */
+
+/*
+ * out = SageAttention(q, k, v) for dense [B, H, N, D] tensors.
+ *   q, k, v : 16-bit inputs of type in_dt (SAGE_F16 or SAGE_BF16).
+ *   out     : [B, H, N, D] of type out_dt (SAGE_F16, SAGE_BF16, or SAGE_F32
+ *             for an unrounded fp32 result).
+ *   causal  : nonzero for top-left causal masking.
+ *   sm_scale: softmax scale; <= 0 selects 1/sqrt(D).
+ *   pv_mode : SAGE_PV_FP16 or SAGE_PV_FP8.
+ *   ws      : workspace of at least sage_workspace_bytes(B, H, N, D, pv_mode).
+ * Runs the quantisation kernels then the fused attention kernel on `stream`.
+ * Limits: 1 <= N <= 2^22, D in {64, 128}, B*H <= 65535.
+ */
+sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                            int in_dt, int out_dt, int B, int H, int N, int D, int causal,
+                            float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/*
+ * Variable-length packed variant: `batch` sequences, sequence s occupying rows
+ * cu_seqlens[s] .. cu_seqlens[s+1]-1 of the [T, H, D] tensors q, k, v, out.
+ *   cu_seqlens  : DEVICE int32 [batch + 1], cu_seqlens[0] = 0, non-decreasing,
+ *                 cu_seqlens[batch] = total_tokens; every length <= max_seqlen.
+ *                 Violations are detected on the device (SAGE_ERR_BAD_SEQLENS
+ *                 via sage_sync_status) and leave `out` unspecified.
+ *   max_seqlen  : an upper bound on the sequence lengths (used for validation).
+ * Every sequence has its own K mean, its own quantisation blocks and (FP8) its
+ * own V channel scales.  Other arguments as sage_attn_fwd.
+ */
+sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out,
+                                   int in_dt, int out_dt, const int32_t* cu_seqlens, int batch,
+                                   int max_seqlen, int total_tokens, int H, int D, int causal,
+                                   float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* ------------------------------------------ the two stages, separately -- */
+
+/*
+ * Stage 1 (smoothing + quantisation) of a dense problem into caller buffers:
+ *   q_codes, k_codes : int8 [B, H, NP, D], NP = ceil(N/128)*128; padding rows 0.
+ *   q_scale, k_scale : fp32 [B, H, NP/128], the per-block deltas (max|x|/127).
+ *   k_mean           : fp32 [B, H, D], the per-channel K mean subtracted.
+ *   v_codes          : FP8 mode: E4M3 bytes [B, H, N, D]; else may be NULL.
+ *   v_scale          : FP8 mode: fp32 [B, H, D], per-channel max|v|/448.
+ *   ws               : at least sage_scratch_bytes(B, H, D).
+ * Quantiser arithmetic (binary32, round-half-to-even): s = 127/max|x| per
+ * block, code = clamp(rint(x*s), -127, 127); a block with max|x| = 0 gets
+ * delta 0 and zero codes.  K mean: each k is put on the 2^-24 grid, summed
+ * exactly in int64 and divided once in fp64, m = fp32(sum / (N * 2^24)).
+ */
+sage_status_t sage_quantize(const void* q, const void* k, const void* v, int in_dt, int B, int H,
+                            int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
+                            int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
+                            float* v_scale, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Stage 2 (fused INT8 QK^T + online softmax + P.V) of a dense problem from the
+ * buffers sage_quantize wrote.  v is the original 16-bit V (FP16 mode; of type
+ * v_dt) -- ignored in FP8 mode, where v_codes / v_scale are used instead.
+ * ws: at least sage_scratch_bytes(B, H, D).  Other arguments as sage_attn_fwd.
+ */
+sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
+                                  const int8_t* k_codes, const float* k_scale, const void* v,
+                                  const uint8_t* v_codes, const float* v_scale, void* out,
+                                  int v_dt, int out_dt, int B, int H, int N, int D, int causal,
+                                  float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/*
+ * Stage 1 for a packed varlen batch.  Layouts (TB = number of 128-token blocks
+ * over all sequences = sum_s ceil(n_s/128); blocks of sequence s start at
+ * block index blk_off[s] = sum_{s'<s} ceil(n_s'/128)):
+ *   q_codes, k_codes : int8 [H, TBmax*128, D] with TBmax = total_tokens/128 +
+ *                      batch (upper bound of TB); block b of sequence s of head
+ *                      h at rows (blk_off[s] + b)*128 ...
+ *   q_scale, k_scale : fp32 [H, TBmax].
+ *   k_mean           : fp32 [batch, H, D].
+ *   v_codes          : FP8 mode: E4M3 [T, H, D]; v_scale fp32 [batch, H, D].
+ *   ws               : at least sage_workspace_bytes_varlen(...) (holds the
+ *                      per-sequence schedule as well as the scratch).
+ */
+sage_status_t sage_quantize_varlen(const void* q, const void* k, const void* v, int in_dt,
+                                   const int32_t* cu_seqlens, int batch, int max_seqlen,
+                                   int total_tokens, int H, int D, int pv_mode, int8_t* q_codes,
+                                   float* q_scale, int8_t* k_codes, float* k_scale,
+                                   float* k_mean, uint8_t* v_codes, float* v_scale, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ diagnostics -- */
+
+/*
+ * INT8 QK^T tiles through the same TMA + tcgen05 (kind::i8) path the attention
+ * kernel uses: for each of n_tiles requests tiles[3*t .. 3*t+2] = (bh, I, J)
+ * (host int32 array), writes S[r][c] = sum_d q_codes[bh][128 I + r][d] *
+ * k_codes[bh][128 J + c][d] as int32 into s_out + t*128*128.  q_codes and
+ * k_codes are the dense [B*H, NP, D] code arrays of sage_quantize.
+ */
+sage_status_t sage_qk_int8_tiles(const int8_t* q_codes, const int8_t* k_codes, int BH, int NP,
+                                 int D, const int32_t* tiles, int n_tiles, int32_t* s_out,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Self-test of device-side failure reporting: launches one CTA that waits on
+ * a barrier nothing signals, gives up after wait_cycles (1 .. 2^31) SM clock
+ * cycles and records SAGE_ERR_TIMEOUT in the workspace's status word, which
+ * the next sage_sync_status() returns.  The GPU stays usable.  This is the
+ * same bounded-wait path every pipeline wait of the attention kernel takes.
+ */
+sage_status_t sage_selftest_wait_timeout(long long wait_cycles, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H */

@@ -1,0 +1,13 @@
+"""SageAttention 8-bit attention forward pass for NVIDIA B200 (sm_100a).
+
+K smoothing, per-block INT8 Q/K quantisation, INT8 QK^T on tcgen05 tensor
+cores with TMEM accumulators, online softmax, and P.V in 16 bits or in FP8
+with two-level FP32 accumulation -- as hand-written CUDA kernels behind the C
+ABI declared in include/sage.h (libsageb200.so).  This package is the Python
+binding of that library.
+"""
+from .api import (  # noqa: F401
+    BLOCK, PV_MODES, Quantized, SageError, Workspace, alloc_quantized, attn_fwd, attn_fwd_varlen,
+    attn_quantized, qk_int8_tiles, quantize, quantize_varlen, sageattn, sync_status,
+    workspace_bytes, workspace_bytes_varlen,
+)

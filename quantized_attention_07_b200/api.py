@@ -1,0 +1,326 @@
+"""Python binding of libsageb200.so -- argument marshalling only.
+
+Every step of the method runs in the library's CUDA kernels; this module only
+checks shapes/dtypes, hands device pointers and the current CUDA stream to
+the C ABI, and turns error codes into exceptions.  PyTorch provides device
+memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+
+F16, BF16, F32 = 0, 1, 2
+PV_MODES = {"fp16": 0, "fp8": 1}
+BLOCK = 128
+
+STATUS = {
+    0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED", 3: "SAGE_ERR_WORKSPACE",
+    4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_TIMEOUT", 6: "SAGE_ERR_BAD_SEQLENS", 7: "SAGE_ERR_RANGE",
+}
+
+
+class SageError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        name = STATUS.get(code, f"status {code}")
+        detail = ""
+        if code == 4:
+            detail = _lib.load().sage_last_cuda_error().decode(errors="replace")
+        super().__init__(f"{what}: {name}" + (f" ({detail})" if detail else ""))
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise SageError(code, what)
+
+
+def _dtype_code(t: torch.dtype, allow_f32: bool = False) -> int:
+    if t == torch.float16:
+        return F16
+    if t == torch.bfloat16:
+        return BF16
+    if allow_f32 and t == torch.float32:
+        return F32
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def _pv(pv_mode: str) -> int:
+    if pv_mode not in PV_MODES:
+        raise ValueError(f"pv_mode must be one of {sorted(PV_MODES)}")
+    return PV_MODES[pv_mode]
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda_contig(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+class Workspace:
+    """A caller-owned device workspace (torch uint8 buffer) with its status word."""
+
+    def __init__(self, nbytes: int, device: torch.device | str | int = "cuda"):
+        self.device = torch.device(device)
+        self.buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=self.device)
+        _check(_lib.load().sage_workspace_init(self.ptr, self.nbytes, _stream(self.device)),
+               "sage_workspace_init")
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+    def ensure(self, nbytes: int) -> "Workspace":
+        if nbytes > self.nbytes:
+            self.__init__(nbytes, self.device)
+        return self
+
+    def sync_status(self) -> None:
+        """Synchronise the current stream and raise on any device-side error."""
+        _check(_lib.load().sage_sync_status(self.ptr, _stream(self.device)), "device status")
+
+
+_default_ws: dict = {}
+
+
+def _workspace(dev: torch.device, nbytes: int, ws: Optional[Workspace]) -> Workspace:
+    if ws is not None:
+        return ws.ensure(nbytes)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device())
+    w = _default_ws.get(key)
+    if w is None:
+        w = _default_ws[key] = Workspace(nbytes, dev)
+    return w.ensure(nbytes)
+
+
+def workspace_bytes(B: int, H: int, N: int, D: int, pv_mode: str = "fp16") -> int:
+    return int(_lib.load().sage_workspace_bytes(B, H, N, D, _pv(pv_mode)))
+
+
+def workspace_bytes_varlen(total_tokens: int, batch: int, H: int, D: int,
+                           pv_mode: str = "fp16") -> int:
+    return int(_lib.load().sage_workspace_bytes_varlen(total_tokens, batch, H, D, _pv(pv_mode)))
+
+
+# ----------------------------------------------------------------- forward --
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             sm_scale: Optional[float] = None, pv_mode: str = "fp16",
+             out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
+             workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """SageAttention forward over dense [B, H, N, D] fp16/bf16 tensors."""
+    _need_cuda_contig(q, k, v)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, H, N, D] shape")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype")
+    B, H, N, D = q.shape
+    od = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty((B, H, N, D), dtype=od, device=q.device)
+    _need_cuda_contig(out)
+    mode = _pv(pv_mode)
+    ws = _workspace(q.device, workspace_bytes(B, H, N, D, pv_mode), workspace)
+    _check(_lib.load().sage_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+        _dtype_code(out.dtype, True), B, H, N, D, int(bool(causal)),
+        float(sm_scale) if sm_scale else 0.0, mode, ws.ptr, ws.nbytes, _stream(q.device)),
+        "sage_attn_fwd")
+    return out
+
+
+def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                    max_seqlen: int, causal: bool = False, sm_scale: Optional[float] = None,
+                    pv_mode: str = "fp16", out_dtype: Optional[torch.dtype] = None,
+                    out: Optional[torch.Tensor] = None,
+                    workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """SageAttention forward over packed [T, H, D] tensors with int32 cu_seqlens."""
+    _need_cuda_contig(q, k, v, cu_seqlens)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [T, H, D] shape")
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    T, H, D = q.shape
+    batch = cu_seqlens.numel() - 1
+    od = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty((T, H, D), dtype=od, device=q.device)
+    _need_cuda_contig(out)
+    mode = _pv(pv_mode)
+    ws = _workspace(q.device, workspace_bytes_varlen(T, batch, H, D, pv_mode), workspace)
+    _check(_lib.load().sage_attn_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype), _dtype_code(out.dtype, True),
+        _ptr(cu_seqlens), batch, int(max_seqlen), T, H, D, int(bool(causal)),
+        float(sm_scale) if sm_scale else 0.0, mode, ws.ptr, ws.nbytes, _stream(q.device)),
+        "sage_attn_fwd_varlen")
+    return out
+
+
+# ---------------------------------------------------------------- stages --
+
+@dataclasses.dataclass
+class Quantized:
+    """Outputs of the smoothing + quantisation stage (all device tensors)."""
+    q_codes: torch.Tensor
+    q_scale: torch.Tensor
+    k_codes: torch.Tensor
+    k_scale: torch.Tensor
+    k_mean: torch.Tensor
+    v_codes: Optional[torch.Tensor]
+    v_scale: Optional[torch.Tensor]
+    pv_mode: str
+
+
+def alloc_quantized(B: int, H: int, N: int, D: int, pv_mode: str, device) -> Quantized:
+    NB = (N + BLOCK - 1) // BLOCK
+    fp8 = pv_mode == "fp8"
+    e = dict(device=device)
+    return Quantized(
+        torch.empty((B, H, NB * BLOCK, D), dtype=torch.int8, **e),
+        torch.empty((B, H, NB), dtype=torch.float32, **e),
+        torch.empty((B, H, NB * BLOCK, D), dtype=torch.int8, **e),
+        torch.empty((B, H, NB), dtype=torch.float32, **e),
+        torch.empty((B, H, D), dtype=torch.float32, **e),
+        torch.empty((B, H, N, D), dtype=torch.uint8, **e) if fp8 else None,
+        torch.empty((B, H, D), dtype=torch.float32, **e) if fp8 else None,
+        pv_mode)
+
+
+def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
+             pv_mode: str = "fp16", qz: Optional[Quantized] = None,
+             workspace: Optional[Workspace] = None) -> Quantized:
+    """Stage 1 (K smoothing, per-block INT8 Q/K, FP8 V) of a dense problem."""
+    _need_cuda_contig(q, k)
+    B, H, N, D = q.shape
+    mode = _pv(pv_mode)
+    if mode == 1:
+        if v is None:
+            raise ValueError("FP8 P.V needs v")
+        _need_cuda_contig(v)
+    qz = qz or alloc_quantized(B, H, N, D, pv_mode, q.device)
+    ws = _workspace(q.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
+    _check(_lib.load().sage_quantize(
+        _ptr(q), _ptr(k), _ptr(v) if mode == 1 else None, _dtype_code(q.dtype), B, H, N, D, mode,
+        _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(qz.k_mean),
+        _ptr(qz.v_codes), _ptr(qz.v_scale), ws.ptr, ws.nbytes, _stream(q.device)),
+        "sage_quantize")
+    return qz
+
+
+def attn_quantized(qz: Quantized, v: torch.Tensor, causal: bool = False,
+                   sm_scale: Optional[float] = None, out_dtype: Optional[torch.dtype] = None,
+                   out: Optional[torch.Tensor] = None,
+                   workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """Stage 2 (fused INT8 QK^T, online softmax, P.V) from stage-1 outputs."""
+    _need_cuda_contig(v)
+    B, H, N, D = v.shape
+    mode = _pv(qz.pv_mode)
+    od = out_dtype or v.dtype
+    if out is None:
+        out = torch.empty((B, H, N, D), dtype=od, device=v.device)
+    ws = _workspace(v.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
+    _check(_lib.load().sage_attn_quantized(
+        _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(v),
+        _ptr(qz.v_codes), _ptr(qz.v_scale), _ptr(out), _dtype_code(v.dtype),
+        _dtype_code(out.dtype, True), B, H, N, D, int(bool(causal)),
+        float(sm_scale) if sm_scale else 0.0, mode, ws.ptr, ws.nbytes, _stream(v.device)),
+        "sage_attn_quantized")
+    return out
+
+
+def quantize_varlen(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
+                    cu_seqlens: torch.Tensor, max_seqlen: int, pv_mode: str = "fp16",
+                    workspace: Optional[Workspace] = None) -> Quantized:
+    """Stage 1 of a packed varlen batch; code layout [H, TBmax*128, D]."""
+    _need_cuda_contig(q, k, cu_seqlens)
+    T, H, D = q.shape
+    batch = cu_seqlens.numel() - 1
+    mode = _pv(pv_mode)
+    TB = (T + (BLOCK - 1) * batch) // BLOCK
+    e = dict(device=q.device)
+    fp8 = mode == 1
+    qz = Quantized(
+        torch.empty((H, TB * BLOCK, D), dtype=torch.int8, **e),
+        torch.empty((H, TB), dtype=torch.float32, **e),
+        torch.empty((H, TB * BLOCK, D), dtype=torch.int8, **e),
+        torch.empty((H, TB), dtype=torch.float32, **e),
+        torch.empty((batch, H, D), dtype=torch.float32, **e),
+        torch.empty((T, H, D), dtype=torch.uint8, **e) if fp8 else None,
+        torch.empty((batch, H, D), dtype=torch.float32, **e) if fp8 else None,
+        pv_mode)
+    ws = _workspace(q.device, workspace_bytes_varlen(T, batch, H, D, pv_mode), workspace)
+    _check(_lib.load().sage_quantize_varlen(
+        _ptr(q), _ptr(k), _ptr(v) if fp8 else None, _dtype_code(q.dtype), _ptr(cu_seqlens), batch,
+        int(max_seqlen), T, H, D, mode, _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes),
+        _ptr(qz.k_scale), _ptr(qz.k_mean), _ptr(qz.v_codes), _ptr(qz.v_scale), ws.ptr, ws.nbytes,
+        _stream(q.device)), "sage_quantize_varlen")
+    return qz
+
+
+def qk_int8_tiles(q_codes: torch.Tensor, k_codes: torch.Tensor,
+                  tiles: Sequence[tuple[int, int, int]],
+                  workspace: Optional[Workspace] = None) -> torch.Tensor:
+    """int32 QK^T tiles (bh, I, J) of dense [B, H, NP, D] code arrays, through the
+    attention kernel's TMA + tcgen05 INT8 path.  Returns [n, 128, 128]."""
+    _need_cuda_contig(q_codes, k_codes)
+    B, H, NP, D = q_codes.shape
+    flat = [int(x) for t in tiles for x in t]
+    arr = (ctypes.c_int32 * len(flat))(*flat)
+    out = torch.empty((len(tiles), BLOCK, BLOCK), dtype=torch.int32, device=q_codes.device)
+    ws = _workspace(q_codes.device, 256 + 256 * (1 + len(flat) * 4 // 256), workspace)
+    _check(_lib.load().sage_qk_int8_tiles(
+        _ptr(q_codes), _ptr(k_codes), B * H, NP, D, ctypes.cast(arr, ctypes.c_void_p),
+        len(tiles), _ptr(out), ws.ptr, ws.nbytes, _stream(q_codes.device)), "sage_qk_int8_tiles")
+    return out
+
+
+def sync_status(workspace: Optional[Workspace] = None, device=None) -> None:
+    """Synchronise and raise if any call on the workspace recorded a device error."""
+    if workspace is None:
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        workspace = _default_ws.get(key)
+        if workspace is None:
+            return
+    workspace.sync_status()
+
+
+# --------------------------------------------------------- SDPA-style shim --
+
+def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, attn_mask=None,
+             dropout_p: float = 0.0, is_causal: bool = False, scale: Optional[float] = None,
+             pv_mode: str = "fp16") -> torch.Tensor:
+    """Drop-in for scaled_dot_product_attention on [B, H, N, D] fp16/bf16 inputs.
+
+    Arbitrary masks and dropout are not part of the method; passing them raises
+    SageError(SAGE_ERR_UNSUPPORTED).  Non-contiguous inputs (e.g. the
+    transpose(1, 2) views of a projection output) are made contiguous first.
+    """
+    if attn_mask is not None or dropout_p:
+        raise SageError(2, "sageattn: attn_mask / dropout_p")
+    q, k, v = (t if t.is_contiguous() else t.contiguous() for t in (q, k, v))
+    return attn_fwd(q, k, v, causal=is_causal, sm_scale=scale, pv_mode=pv_mode)
+
+
+def default_sm_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,426 @@
+// C ABI of libsageb200.so: argument validation, workspace layout, launches,
+// and the device status word.  Nothing here allocates device memory; every
+// buffer is the caller's.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace sage {
+
+cudaError_t launch_varlen_prep(const int32_t* cu, int batch, int max_seqlen, int total_tokens,
+                               int32_t* blk_off, int32_t* pair_off, uint32_t* status,
+                               cudaStream_t st);
+cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool fp8,
+                         const void* q, const void* k, const void* v, int8_t* q_codes,
+                         float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
+                         uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
+                         uint32_t* v_amax, uint32_t* status, cudaStream_t st);
+cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
+                            const int32_t* tiles, int n, int32_t* out, uint32_t* status,
+                            cudaStream_t st);
+}  // namespace sage
+
+#include "attn_launch.cuh"
+
+using namespace sage;
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+sage_status_t cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+  return SAGE_ERR_CUDA;
+}
+
+constexpr size_t kHeader = 256;
+constexpr long long kMaxN = 1LL << 22;
+
+size_t al(size_t x) { return (x + 255) & ~size_t(255); }
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool in_dtype_ok(int dt) { return dt == SAGE_F16 || dt == SAGE_BF16; }
+bool out_dtype_ok(int dt) { return dt == SAGE_F16 || dt == SAGE_BF16 || dt == SAGE_F32; }
+
+float kappa_of(float sm_scale, int D) {
+  const float s = sm_scale > 0.0f ? sm_scale : (float)(1.0 / std::sqrt((double)D));
+  return (float)((double)s * 1.4426950408889634);  // fp32(sm_scale * log2 e)
+}
+
+// Workspace layout.  Offsets in bytes from the workspace base.
+struct Layout {
+  size_t k_sum, v_amax, blk_off, pair_off;             // scratch
+  size_t q_codes, k_codes, q_scale, k_scale, k_mean;   // quantised operands
+  size_t v_codes, v_scale;
+  size_t scratch_end, total;
+};
+
+Layout dense_layout(int B, int H, int N, int D, bool fp8) {
+  const size_t BH = (size_t)B * H, NB = ((size_t)N + BLK - 1) / BLK, NP = NB * BLK;
+  Layout L{};
+  size_t o = kHeader;
+  L.k_sum = o; o += al(BH * D * 8);
+  L.v_amax = o; o += al(BH * D * 4);
+  L.scratch_end = o;
+  L.q_codes = o; o += al(BH * NP * D);
+  L.k_codes = o; o += al(BH * NP * D);
+  L.q_scale = o; o += al(BH * NB * 4);
+  L.k_scale = o; o += al(BH * NB * 4);
+  L.k_mean = o; o += al(BH * D * 4);
+  if (fp8) {
+    L.v_codes = o; o += al(BH * (size_t)N * D);
+    L.v_scale = o; o += al(BH * D * 4);
+  }
+  L.total = o;
+  return L;
+}
+
+long long tb_max(long long T, long long batch) { return (T + (BLK - 1) * batch) / BLK; }
+long long pair_max(long long T, long long batch) { return (T + (2 * BLK - 1) * batch) / (2 * BLK); }
+
+Layout varlen_layout(int T, int batch, int H, int D, bool fp8) {
+  const size_t SH = (size_t)batch * H, TB = (size_t)tb_max(T, batch);
+  Layout L{};
+  size_t o = kHeader;
+  L.k_sum = o; o += al(SH * D * 8);
+  L.v_amax = o; o += al(SH * D * 4);
+  L.blk_off = o; o += al(((size_t)batch + 1) * 4);
+  L.pair_off = o; o += al(((size_t)batch + 1) * 4);
+  L.scratch_end = o;
+  L.q_codes = o; o += al((size_t)H * TB * BLK * D);
+  L.k_codes = o; o += al((size_t)H * TB * BLK * D);
+  L.q_scale = o; o += al((size_t)H * TB * 4);
+  L.k_scale = o; o += al((size_t)H * TB * 4);
+  L.k_mean = o; o += al(SH * D * 4);
+  if (fp8) {
+    L.v_codes = o; o += al((size_t)T * H * D);
+    L.v_scale = o; o += al(SH * D * 4);
+  }
+  L.total = o;
+  return L;
+}
+
+bool dense_args_ok(int B, int H, int N, int D, int pv_mode) {
+  return B >= 1 && H >= 1 && N >= 1 && N <= kMaxN && (D == 64 || D == 128) &&
+         (long long)B * H <= 65535 && (pv_mode == SAGE_PV_FP16 || pv_mode == SAGE_PV_FP8);
+}
+
+bool varlen_args_ok(int T, int batch, int max_seqlen, int H, int D, int pv_mode) {
+  return T >= 0 && batch >= 1 && max_seqlen >= 0 && max_seqlen <= kMaxN && H >= 1 &&
+         H <= 65535 && (D == 64 || D == 128) &&
+         (long long)T + 2 * BLK * (long long)batch < (1LL << 31) &&
+         (pv_mode == SAGE_PV_FP16 || pv_mode == SAGE_PV_FP8);
+}
+
+template <class T> T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+sage_status_t clear_scratch(void* ws, const Layout& L, bool fp8, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, L.k_sum), 0, L.v_amax - L.k_sum, st);
+  if (e == cudaSuccess && fp8)
+    e = cudaMemsetAsync(at<uint8_t>(ws, L.v_amax), 0, L.scratch_end - L.v_amax, st);
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "cudaMemsetAsync");
+}
+
+// Dense stage 1 into explicit buffers.
+sage_status_t quantize_dense(const void* q, const void* k, const void* v, int in_dt, int B,
+                             int H, int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
+                             int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
+                             float* v_scale, void* ws, const Layout& L, cudaStream_t st) {
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  sage_status_t r = clear_scratch(ws, L, fp8, st);
+  if (r != SAGE_OK) return r;
+  SeqLayout S{};
+  S.varlen = 0;
+  S.N = N;
+  S.H = H;
+  const dim3 grid((N + BLK - 1) / BLK, B * H);
+  cudaError_t e = launch_quant(S, grid, D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
+                               k_codes, k_scale, k_mean, v_codes, v_scale,
+                               at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
+                               at<uint32_t>(ws, 0), st);
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
+}
+
+sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
+                         const float* k_scale, const void* v, const uint8_t* v_codes,
+                         const float* v_scale, void* out, int v_dt, int out_dt, int B, int H,
+                         int N, int D, int causal, float sm_scale, int pv_mode, void* ws,
+                         cudaStream_t st) {
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  AttnLaunch A{};
+  A.p.H = H;
+  A.p.N = N;
+  A.p.BH = B * H;
+  A.p.NB = (N + BLK - 1) / BLK;
+  A.p.NPAIR = (N + 2 * BLK - 1) / (2 * BLK);
+  A.p.causal = causal ? 1 : 0;
+  A.p.kappa = kappa_of(sm_scale, D);
+  A.p.q_scale = q_scale;
+  A.p.k_scale = k_scale;
+  A.p.v_scale = v_scale;
+  A.p.out = out;
+  A.p.out_dt = out_dt;
+  A.p.varlen = 0;
+  A.p.status = at<uint32_t>(ws, 0);
+  A.D = D;
+  A.pv8 = fp8;
+  A.bf16v = v_dt == SAGE_BF16;
+  A.q_codes = q_codes;
+  A.k_codes = k_codes;
+  A.v = fp8 ? static_cast<const void*>(v_codes) : v;
+  A.code_rows = A.p.NB * BLK;
+  A.code_z = B * H;
+  A.T = 0;
+  A.grid = dim3((unsigned)((long long)B * H * A.p.NPAIR), 1, 1);
+  cudaError_t e = launch_attn(A, st);
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "attention launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sage_workspace_bytes(int B, int H, int N, int D, int pv_mode) {
+  if (!dense_args_ok(B, H, N, D, pv_mode)) return 0;
+  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8).total;
+}
+
+size_t sage_workspace_bytes_varlen(int total_tokens, int batch, int H, int D, int pv_mode) {
+  if (!varlen_args_ok(total_tokens, batch, 0, H, D, pv_mode)) return 0;
+  return varlen_layout(total_tokens, batch, H, D, pv_mode == SAGE_PV_FP8).total;
+}
+
+size_t sage_scratch_bytes(int B, int H, int D) {
+  if (B < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+  return dense_layout(B, H, 1, D, true).scratch_end;
+}
+
+const char* sage_status_string(sage_status_t s) {
+  switch (s) {
+    case SAGE_OK: return "SAGE_OK";
+    case SAGE_ERR_INVALID_ARG: return "SAGE_ERR_INVALID_ARG";
+    case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
+    case SAGE_ERR_WORKSPACE: return "SAGE_ERR_WORKSPACE";
+    case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
+    case SAGE_ERR_TIMEOUT: return "SAGE_ERR_TIMEOUT";
+    case SAGE_ERR_BAD_SEQLENS: return "SAGE_ERR_BAD_SEQLENS";
+    case SAGE_ERR_RANGE: return "SAGE_ERR_RANGE";
+  }
+  return "SAGE_ERR_UNKNOWN";
+}
+
+const char* sage_last_cuda_error(void) { return g_last_error; }
+
+sage_status_t sage_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!aligned16(ws) || ws_bytes < kHeader) return SAGE_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeader, as_stream(stream));
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "cudaMemsetAsync");
+}
+
+sage_status_t sage_sync_status(void* ws, void* stream) {
+  if (!aligned16(ws)) return SAGE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word != 0) {
+    e = cudaMemsetAsync(ws, 0, sizeof(word), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  }
+  if (word & ST_TIMEOUT) return SAGE_ERR_TIMEOUT;
+  if (word & ST_BAD_SEQLENS) return SAGE_ERR_BAD_SEQLENS;
+  if (word & ST_RANGE) return SAGE_ERR_RANGE;
+  return SAGE_OK;
+}
+
+sage_status_t sage_quantize(const void* q, const void* k, const void* v, int in_dt, int B, int H,
+                            int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
+                            int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
+                            float* v_scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !in_dtype_ok(in_dt)) return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes) ||
+      !q_scale || !k_scale || !k_mean || !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
+  const Layout L = dense_layout(B, H, N, D, fp8);
+  if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
+  return quantize_dense(q, k, v, in_dt, B, H, N, D, pv_mode, q_codes, q_scale, k_codes, k_scale,
+                        k_mean, v_codes, v_scale, ws, L, as_stream(stream));
+}
+
+sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
+                                  const int8_t* k_codes, const float* k_scale, const void* v,
+                                  const uint8_t* v_codes, const float* v_scale, void* out,
+                                  int v_dt, int out_dt, int B, int H, int N, int D, int causal,
+                                  float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !k_scale || !aligned16(out) ||
+      !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+    return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
+  return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
+                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream));
+}
+
+sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int in_dt,
+                            int out_dt, int B, int H, int N, int D, int causal, float sm_scale,
+                            int pv_mode, void* ws, size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
+      !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  const Layout L = dense_layout(B, H, N, D, fp8);
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  sage_status_t r = quantize_dense(
+      q, k, v, in_dt, B, H, N, D, pv_mode, at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
+      at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
+      fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr, fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L,
+      st);
+  if (r != SAGE_OK) return r;
+  return attn_dense(at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale), at<int8_t>(ws, L.k_codes),
+                    at<float>(ws, L.k_scale), v, fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
+                    fp8 ? at<float>(ws, L.v_scale) : nullptr, out, in_dt, out_dt, B, H, N, D,
+                    causal, sm_scale, pv_mode, ws, st);
+}
+
+static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, int in_dt,
+                                   const int32_t* cu, int batch, int max_seqlen, int T, int H,
+                                   int D, int pv_mode, int8_t* q_codes, float* q_scale,
+                                   int8_t* k_codes, float* k_scale, float* k_mean,
+                                   uint8_t* v_codes, float* v_scale, void* ws, const Layout& L,
+                                   cudaStream_t st) {
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  sage_status_t r = clear_scratch(ws, L, fp8, st);
+  if (r != SAGE_OK) return r;
+  cudaError_t e = launch_varlen_prep(cu, batch, max_seqlen, T, at<int32_t>(ws, L.blk_off),
+                                     at<int32_t>(ws, L.pair_off), at<uint32_t>(ws, 0), st);
+  if (e != cudaSuccess) return cuda_fail(e, "varlen preparation launch");
+  const long long TB = tb_max(T, batch);
+  if (TB == 0) return SAGE_OK;
+  SeqLayout S{};
+  S.varlen = 1;
+  S.H = H;
+  S.cu = cu;
+  S.blk_off = at<int32_t>(ws, L.blk_off);
+  S.batch = batch;
+  S.TBmax = (int)TB;
+  e = launch_quant(S, dim3((unsigned)TB, H), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
+                   k_codes, k_scale, k_mean, v_codes, v_scale,
+                   at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
+                   at<uint32_t>(ws, 0), st);
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
+}
+
+sage_status_t sage_quantize_varlen(const void* q, const void* k, const void* v, int in_dt,
+                                   const int32_t* cu_seqlens, int batch, int max_seqlen,
+                                   int total_tokens, int H, int D, int pv_mode, int8_t* q_codes,
+                                   float* q_scale, int8_t* k_codes, float* k_scale,
+                                   float* k_mean, uint8_t* v_codes, float* v_scale, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!varlen_args_ok(total_tokens, batch, max_seqlen, H, D, pv_mode) || !in_dtype_ok(in_dt))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes) ||
+      !q_scale || !k_scale || !k_mean || !aligned16(ws) || !cu_seqlens)
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
+  const Layout L = varlen_layout(total_tokens, batch, H, D, fp8);
+  if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
+  if (total_tokens == 0) return SAGE_OK;
+  return varlen_stage1(q, k, v, in_dt, cu_seqlens, batch, max_seqlen, total_tokens, H, D, pv_mode,
+                       q_codes, q_scale, k_codes, k_scale, k_mean, v_codes, v_scale, ws, L,
+                       as_stream(stream));
+}
+
+sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out,
+                                   int in_dt, int out_dt, const int32_t* cu_seqlens, int batch,
+                                   int max_seqlen, int total_tokens, int H, int D, int causal,
+                                   float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (!varlen_args_ok(total_tokens, batch, max_seqlen, H, D, pv_mode) || !in_dtype_ok(in_dt) ||
+      !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws) ||
+      !cu_seqlens)
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  const Layout L = varlen_layout(total_tokens, batch, H, D, fp8);
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  if (total_tokens == 0) return SAGE_OK;
+  cudaStream_t st = as_stream(stream);
+  sage_status_t r = varlen_stage1(
+      q, k, v, in_dt, cu_seqlens, batch, max_seqlen, total_tokens, H, D, pv_mode,
+      at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale), at<int8_t>(ws, L.k_codes),
+      at<float>(ws, L.k_scale), at<float>(ws, L.k_mean), fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
+      fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L, st);
+  if (r != SAGE_OK) return r;
+  const long long TB = tb_max(total_tokens, batch), PM = pair_max(total_tokens, batch);
+  if (PM == 0) return SAGE_OK;
+  AttnLaunch A{};
+  A.p.H = H;
+  A.p.causal = causal ? 1 : 0;
+  A.p.kappa = kappa_of(sm_scale, D);
+  A.p.q_scale = at<float>(ws, L.q_scale);
+  A.p.k_scale = at<float>(ws, L.k_scale);
+  A.p.v_scale = fp8 ? at<float>(ws, L.v_scale) : nullptr;
+  A.p.out = out;
+  A.p.out_dt = out_dt;
+  A.p.varlen = 1;
+  A.p.cu = cu_seqlens;
+  A.p.blk_off = at<int32_t>(ws, L.blk_off);
+  A.p.pair_off = at<int32_t>(ws, L.pair_off);
+  A.p.batch = batch;
+  A.p.TBmax = (int)TB;
+  A.p.status = at<uint32_t>(ws, 0);
+  A.D = D;
+  A.pv8 = fp8;
+  A.bf16v = in_dt == SAGE_BF16;
+  A.q_codes = at<int8_t>(ws, L.q_codes);
+  A.k_codes = at<int8_t>(ws, L.k_codes);
+  A.v = fp8 ? static_cast<const void*>(at<uint8_t>(ws, L.v_codes)) : v;
+  A.code_rows = (int)(TB * BLK);
+  A.code_z = H;
+  A.T = total_tokens;
+  A.grid = dim3((unsigned)PM, H, 1);
+  cudaError_t e = launch_attn(A, st);
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "attention launch");
+}
+
+sage_status_t sage_qk_int8_tiles(const int8_t* q_codes, const int8_t* k_codes, int BH, int NP,
+                                 int D, const int32_t* tiles, int n_tiles, int32_t* s_out,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (BH < 1 || NP < BLK || NP % BLK != 0 || (D != 64 && D != 128) || n_tiles < 1 || !tiles ||
+      !aligned16(q_codes) || !aligned16(k_codes) || !aligned16(s_out) || !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int bh = tiles[3 * t], I = tiles[3 * t + 1], J = tiles[3 * t + 2];
+    if (bh < 0 || bh >= BH || I < 0 || J < 0 || I >= NP / BLK || J >= NP / BLK)
+      return SAGE_ERR_INVALID_ARG;
+  }
+  const size_t need = kHeader + al((size_t)n_tiles * 3 * 4);
+  if (ws_bytes < need) return SAGE_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  int32_t* dtiles = at<int32_t>(ws, kHeader);
+  cudaError_t e = cudaMemcpyAsync(dtiles, tiles, (size_t)n_tiles * 3 * 4, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tile list copy");
+  e = launch_qk_tiles(q_codes, k_codes, BH, NP, D, dtiles, n_tiles, s_out, at<uint32_t>(ws, 0), st);
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "QK tile launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,734 @@
+// Fused SageAttention forward kernel for sm_100a.
+//
+// One CTA handles two 128-row query tiles of one (sequence, head) and streams
+// that head's key/value tiles through shared memory:
+//
+//   warp 8       TMA producer: Q^ tiles once, then K^_j and V_j into an
+//                NS-stage ring (cp.async.bulk.tensor, mbarrier complete_tx).
+//   warp 9       MMA issuer (one thread) and TMEM owner:
+//                  S_t  = Q^_t K^_j^T        tcgen05.mma kind::i8 -> int32 TMEM
+//                  O_t += P_t V_j            kind::f16 (16-bit P.V), or
+//                  Part_t = P^_t V^_j        kind::f8f6f4 (FP8 P.V), with P read
+//                                            from TMEM and V from shared memory.
+//   warps 0-3    softmax for query tile 0, warps 4-7 for query tile 1, one
+//                thread per query row: read S from TMEM, dequantise with
+//                deltaQ*deltaK*sm_scale*log2(e), mask, online softmax in base 2,
+//                write P (fp16/bf16 or e4m3) back over S, rescale O (16-bit P.V)
+//                or fold the block's FP8 partial into an fp32 register
+//                accumulator (two-level accumulation), and finally normalise
+//                and store the output row.
+//
+// The two query tiles ping-pong: while one tile's softmax runs on the CUDA
+// cores, the tensor core works on the other tile's P.V and next QK^T.
+//
+// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
+// O_1 [256+D, 256+2D).
+//
+// Method steps (SageAttention pages): INT8 QK^T with the per-block deltas
+// ("SageAttention -- brand new attention", quantisation intro step 3 and
+// "SageAttention" bullets 1-2), online softmax ("Attention机制优化：从
+// FlashAttention到SageAttention的工程实践", section 3.1), P.V in 16 bits
+// ("SageAttention" bullet 3) or FP8 with two-level accumulation
+// ("SageAttention v1/v2/v2++/v3 overview", SageAttention 2 bullets 1 and 3).
+//
+// Every mbarrier wait is bounded.  On a timeout the waiting role records
+// ST_TIMEOUT, raises a CTA-wide abort flag that the other roles' waits also
+// watch, and everyone falls through to the teardown, which waits (bounded) for
+// the CTA's own TMA loads and MMAs and always frees TMEM.
+#include "attn_launch.cuh"
+#include "ptx.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr int NUM_THREADS = 320;
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
+
+template <int D, bool PV8>
+struct Cfg {
+  static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
+  static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
+  static constexpr int SMEM_BUDGET = 227 * 1024 - 2048;
+  static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT);
+  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;    // pipeline stages
+  static constexpr int SMEM = 1024 + 2 * QT + NS * (QT + VT) + 512;
+  // swizzle of the int8 code tiles: rows of D bytes
+  static constexpr uint32_t QK_SWZ = (D == 128) ? 2u : 4u;  // 128B : 64B
+  static constexpr uint32_t QK_SBO = 8 * D;                 // 8 rows
+  // V tiles, MN-major (D contiguous): 16-bit -> 64-element (128 B) atoms;
+  // 8-bit -> one atom of D bytes.
+  static constexpr int V_ROW_BYTES = PV8 ? D : 128;
+  static constexpr uint32_t V_SWZ = (V_ROW_BYTES == 128) ? 2u : 4u;
+  static constexpr uint32_t V_SBO = 8 * V_ROW_BYTES;         // 8 keys
+  static constexpr uint32_t V_LBO = BLK * 128;               // next 64-column atom (16-bit)
+  static constexpr int PV_KSTEP = PV8 ? 32 : 16;             // keys per MMA
+  static constexpr uint32_t V_KSTEP_BYTES = (PV_KSTEP / 8) * V_SBO;
+  static constexpr int PV_STEPS = BLK / PV_KSTEP;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(NS >= 2, "need at least two stages");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t done;
+  uint64_t k_full[8], v_full[8], kv_empty[8];
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+// Warp-uniform bounded wait: true when the phase completed, false (and the
+// abort flag raised) on timeout or when another role aborted.
+__device__ __forceinline__ bool wait_bar(Bars* B, uint64_t* bar, uint32_t parity,
+                                         uint32_t* status, bool warp_uniform) {
+  bool ok = ptx::mbar_try_wait(bar, parity);
+  if (!ok) {
+    const long long t0 = clock64();
+    while (true) {
+      if (ptx::mbar_try_wait(bar, parity)) { ok = true; break; }
+      if (B->abort) break;
+      if (clock64() - t0 > SAGE_WAIT_LIMIT_CYCLES) {
+        set_status(status, ST_TIMEOUT);
+        B->abort = 1;
+        break;
+      }
+    }
+  }
+  if (warp_uniform) ok = __all_sync(0xffffffffu, ok);
+  return ok;
+}
+
+// Work item of this CTA.
+struct Work {
+  int valid;
+  int n;                 // sequence length (queries = keys)
+  int pair;              // query tile pair index within the sequence
+  int head;              // h
+  int code_z;            // z coordinate of this head in the Q^/K^ code maps
+  int q_y0;              // y coordinate of query tile 0 in the code map
+  int k_y0;              // y coordinate of key tile 0 in the code map
+  int v_y0, v_z0;        // TMA coordinates of V tile 0 (x = column)
+  int v_tok_on_z;        // tokens advance along z (varlen) instead of y (dense)
+  long long qs_idx0;     // q_scale index of query tile 0
+  long long ks_idx0;     // k_scale index of key tile 0
+  long long out_row0;    // row (in units of D elements) of token 0 of the output
+  long long out_stride;  // rows between consecutive tokens
+  long long vs_idx;      // v_scale row index (FP8)
+  int nkv[2];            // key tiles for query tile 0 / 1 (0 = tile absent)
+};
+
+__device__ __forceinline__ Work decode_work(const AttnParams& p) {
+  Work w{};
+  int pair, n;
+  if (!p.varlen) {
+    const int idx = blockIdx.x;
+    int bh;
+    if (p.causal) {  // heaviest pairs first
+      pair = p.NPAIR - 1 - idx / p.BH;
+      bh = idx % p.BH;
+    } else {         // head-major: a head's K^/V stay hot in L2
+      bh = idx / p.NPAIR;
+      pair = idx % p.NPAIR;
+    }
+    n = p.N;
+    w.head = bh % p.H;
+    w.code_z = bh;
+    w.q_y0 = pair * 2 * BLK;
+    w.k_y0 = 0;
+    w.v_y0 = 0;
+    w.v_z0 = bh;
+    w.v_tok_on_z = 0;
+    w.qs_idx0 = (long long)bh * p.NB + 2 * pair;
+    w.ks_idx0 = (long long)bh * p.NB;
+    w.out_row0 = (long long)bh * p.N;
+    w.out_stride = 1;
+    w.vs_idx = bh;
+  } else {
+    const int item = blockIdx.x;
+    const int h = blockIdx.y;
+    const int total = __ldg(p.pair_off + p.batch);
+    if (item >= total) { w.valid = 0; return w; }
+    const int s = find_segment(p.pair_off, p.batch + 1, item);
+    const int tok0 = __ldg(p.cu + s);
+    n = __ldg(p.cu + s + 1) - tok0;
+    const int npairs = __ldg(p.pair_off + s + 1) - __ldg(p.pair_off + s);
+    pair = npairs - 1 - (item - __ldg(p.pair_off + s));  // diagonal-heavy pairs first
+    const int blk0 = __ldg(p.blk_off + s);
+    w.head = h;
+    w.code_z = h;
+    w.q_y0 = (blk0 + 2 * pair) * BLK;
+    w.k_y0 = blk0 * BLK;
+    w.v_y0 = h;
+    w.v_z0 = tok0;
+    w.v_tok_on_z = 1;
+    w.qs_idx0 = (long long)h * p.TBmax + blk0 + 2 * pair;
+    w.ks_idx0 = (long long)h * p.TBmax + blk0;
+    w.out_row0 = (long long)tok0 * p.H + h;
+    w.out_stride = p.H;
+    w.vs_idx = (long long)s * p.H + h;
+  }
+  w.valid = 1;
+  w.n = n;
+  w.pair = pair;
+  const int nb = (n + BLK - 1) / BLK;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * pair + t;
+    w.nkv[t] = (qt * BLK >= n) ? 0 : (p.causal ? min(nb, qt + 1) : nb);
+  }
+  return w;
+}
+
+// --------------------------------------------------------------- producer --
+
+template <int D, bool PV8>
+__device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                         const Work& w, Bars* B, uint8_t* sQ, uint8_t* sK, uint8_t* sV,
+                         uint32_t* status) {
+  using C = Cfg<D, PV8>;
+  ptx::prefetch_tmap(tm_q);
+  ptx::prefetch_tmap(tm_k);
+  ptx::prefetch_tmap(tm_v);
+  // both Q^ tiles (an absent second tile reads zero-filled or padding rows)
+  ptx::mbar_arrive_expect_tx(&B->q_full, 2 * C::QT);
+  ptx::tma_load_3d(sQ, tm_q, &B->q_full, 0, w.q_y0, w.code_z);
+  ptx::tma_load_3d(sQ + C::QT, tm_q, &B->q_full, 0, w.q_y0 + BLK, w.code_z);
+  const int nkv = max(w.nkv[0], w.nkv[1]);
+  int j = 0;
+  for (; j < nkv; ++j) {
+    const int s = j % C::NS;
+    if (j >= C::NS && !wait_bar(B, &B->kv_empty[s], ((j / C::NS) - 1) & 1, status, false)) break;
+    ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT);
+    ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.code_z);
+    ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
+    uint8_t* dst = sV + s * C::VT;
+    const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
+    const int z = w.v_tok_on_z ? w.v_z0 + j * BLK : w.v_z0;
+    ptx::tma_load_3d(dst, tm_v, &B->v_full[s], 0, y, z);
+    if (!PV8 && D == 128)  // 16-bit V rows are 256 B: second 64-column box
+      ptx::tma_load_3d(dst + BLK * 128, tm_v, &B->v_full[s], 64, y, z);
+  }
+  // Teardown: the most recent load of every stage must have landed before
+  // this CTA may exit (the earlier ones were consumed already).
+  for (int jj = max(0, j - C::NS); jj < j; ++jj) {
+    const int s = jj % C::NS;
+    const uint32_t ph = (jj / C::NS) & 1;
+    ptx::mbar_wait(&B->k_full[s], ph);
+    ptx::mbar_wait(&B->v_full[s], ph);
+  }
+  ptx::mbar_wait(&B->q_full, 0);
+}
+
+// ------------------------------------------------------------ MMA issuer --
+
+template <int D, bool PV8, bool BF16V>
+__device__ void mma_issuer(const Work& w, Bars* B, uint32_t tmem, const uint8_t* sQ,
+                           const uint8_t* sK, const uint8_t* sV, uint32_t* status) {
+  using C = Cfg<D, PV8>;
+  constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, 128);
+  constexpr uint32_t IDESC_PV =
+      PV8 ? ptx::instr_desc(1, 0, 0, 0, 1, 128, D)
+          : ptx::instr_desc(1, BF16V ? 1 : 0, BF16V ? 1 : 0, 0, 1, 128, D);
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+  const int nkv = max(w.nkv[0], w.nkv[1]);
+
+  auto issue_qk = [&](int t, int j) {
+    const int s = j % C::NS;
+    const uint32_t qa = ptx::smem_u32(sQ + t * C::QT);
+    const uint32_t kb = ptx::smem_u32(sK + s * C::QT);
+#pragma unroll
+    for (int kk = 0; kk < D / 32; ++kk) {
+      const uint64_t ad = ptx::smem_desc(qa + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
+      const uint64_t bd = ptx::smem_desc(kb + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
+      ptx::mma_i8_ss(tS[t], ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+    }
+    ptx::mma_commit(&B->s_full[t]);
+  };
+  auto issue_pv = [&](int t, int j) {
+    const int s = j % C::NS;
+    const uint32_t vb = ptx::smem_u32(sV + s * C::VT);
+    const uint32_t acc0 = PV8 ? 0u : (j > 0 ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < C::PV_STEPS; ++kk) {
+      const uint64_t bd = ptx::smem_desc(vb + kk * C::V_KSTEP_BYTES, C::V_LBO, C::V_SBO, C::V_SWZ);
+      const uint32_t acc = kk > 0 ? 1u : acc0;
+      if constexpr (PV8) ptx::mma_f8_ts(tO[t], tS[t] + 8 * kk, bd, IDESC_PV, acc);
+      else ptx::mma_f16_ts(tO[t], tS[t] + 8 * kk, bd, IDESC_PV, acc);
+    }
+    ptx::mma_commit(&B->o_full[t]);
+  };
+
+  bool ok = wait_bar(B, &B->q_full, 0, status, false);
+  int k_ready = -1;  // highest key tile whose K^ is known to be in shared memory
+  if (ok && nkv > 0) {
+    ok = wait_bar(B, &B->k_full[0], 0, status, false);
+    k_ready = 0;
+    if (ok) {
+      ptx::tc_fence_after();
+      for (int t = 0; t < 2; ++t)
+        if (w.nkv[t] > 0) issue_qk(t, 0);
+    }
+  }
+  for (int j = 0; ok && j < nkv; ++j) {
+    const int s = j % C::NS;
+    if (!wait_bar(B, &B->v_full[s], (j / C::NS) & 1, status, false)) break;
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (j >= w.nkv[t]) continue;
+      if (!wait_bar(B, &B->p_full[t], j & 1, status, false)) { ok = false; break; }
+      ptx::tc_fence_after();
+      issue_pv(t, j);
+      if (j + 1 < w.nkv[t]) {
+        if (k_ready < j + 1) {
+          const int s1 = (j + 1) % C::NS;
+          if (!wait_bar(B, &B->k_full[s1], ((j + 1) / C::NS) & 1, status, false)) { ok = false; break; }
+          k_ready = j + 1;
+        }
+        issue_qk(t, j + 1);
+      }
+    }
+    ptx::mma_commit(&B->kv_empty[s]);
+  }
+  // Drain: every MMA issued above completes before TMEM is released.
+  ptx::mma_commit(&B->done);
+  ptx::mbar_wait(&B->done, 0);
+}
+
+// --------------------------------------------------------------- softmax --
+
+template <int D, bool PV8, bool BF16V>
+__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t tmem, int t) {
+  using In = In16<BF16V>;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;              // row within the query tile
+  const int qt = 2 * w.pair + t;
+  const int row = qt * BLK + r;                   // query index in the sequence
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  const uint32_t tS = tmem + 128 * t + lane_off;
+  const uint32_t tO = tmem + 256 + D * t + lane_off;
+  const int nkv = w.nkv[t];
+  if (nkv == 0) return;
+
+  const float qd = __ldg(p.q_scale + w.qs_idx0 + t);
+  float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f;
+  float o32[PV8 ? D : 1];
+  if constexpr (PV8) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) o32[i] = 0.0f;
+  }
+
+  for (int j = 0; j < nkv; ++j) {
+    if (!wait_bar(B, &B->s_full[t], j & 1, p.status, true)) return;
+    ptx::tc_fence_after();
+    const float kd = __ldg(p.k_scale + w.ks_idx0 + j);
+    const float c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
+    const int key0 = j * BLK;
+    // keys >= limit are masked for this row
+    const int limit = p.causal ? min(w.n, row + 1) : w.n;
+    const bool full_tile = (key0 + BLK <= w.n) && (!p.causal || key0 + BLK - 1 <= qt * BLK);
+    float alpha, rowsum = 0.0f, m_new;
+
+    if constexpr (!PV8) {
+      uint32_t sv[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]);
+        ptx::tmem_ld32(tS + 32 * cc, chunk);
+      }
+      ptx::tmem_wait_ld();
+      int smax = INT_MIN;
+      if (full_tile) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) smax = max(smax, (int)sv[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (key0 + i < limit) smax = max(smax, (int)sv[i]);
+      }
+      m_new = fmaxf(m, __fmul_rn((float)smax, c));
+      alpha = ptx::ex2(__fsub_rn(m, m_new));
+      const float neg = -m_new;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = 32 * cc + 2 * i;
+          float p0 = ptx::ex2(__fmaf_rn((float)(int)sv[c0], c, neg));
+          float p1 = ptx::ex2(__fmaf_rn((float)(int)sv[c0 + 1], c, neg));
+          if (!full_tile) {
+            if (key0 + c0 >= limit) p0 = 0.0f;
+            if (key0 + c0 + 1 >= limit) p1 = 0.0f;
+          }
+          rowsum += p0;
+          rowsum += p1;
+          packed[i] = In::pack(p0, p1);
+        }
+        ptx::tmem_st16(tS + 16 * cc, packed);
+      }
+    } else {
+      // pass 1: row maximum
+      int smax = INT_MIN;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sv[32];
+        ptx::tmem_ld32(tS + 32 * cc, sv);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (full_tile || key0 + 32 * cc + i < limit) smax = max(smax, (int)sv[i]);
+      }
+      m_new = fmaxf(m, __fmul_rn((float)smax, c));
+      alpha = ptx::ex2(__fsub_rn(m, m_new));
+      const float neg = -m_new;
+      // pass 2: P^ = e4m3(448 p), four per TMEM column, written over S
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sv[32];
+        ptx::tmem_ld32(tS + 32 * cc, sv);
+        ptx::tmem_wait_ld();
+        uint32_t packed[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float pp[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 32 * cc + 4 * i + e;
+            float pe = ptx::ex2(__fmaf_rn((float)(int)sv[4 * i + e], c, neg));
+            if (!full_tile && key0 + col >= limit) pe = 0.0f;
+            rowsum += pe;
+            pp[e] = __fmul_rn(pe, 448.0f);
+          }
+          packed[i] = pack_e4m3x4(pp[0], pp[1], pp[2], pp[3]);
+        }
+        ptx::tmem_st8(tS + 8 * cc, packed);
+      }
+    }
+    l = __fadd_rn(__fmul_rn(alpha, l), rowsum);
+
+    if (j > 0) {
+      if (!wait_bar(B, &B->o_full[t], (j - 1) & 1, p.status, true)) return;
+      ptx::tc_fence_after();
+      if constexpr (!PV8) {
+        // O <- alpha * O before this block's P.V accumulates into it
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(tO + 32 * cc, ov);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__fmul_rn(alpha, __uint_as_float(ov[i])));
+            ptx::tmem_st32(tO + 32 * cc, ov);
+          }
+        }
+      } else {
+        // two-level accumulation: O32 <- alpha_{j-1} O32 + Part_{j-1}
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t pv[32];
+          ptx::tmem_ld32(tO + 32 * cc, pv);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            o32[32 * cc + i] = __fmaf_rn(alpha_prev, o32[32 * cc + i], __uint_as_float(pv[i]));
+        }
+      }
+    }
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(&B->p_full[t]);
+    m = m_new;
+    alpha_prev = alpha;
+  }
+
+  // ------------------------------------------------------------ epilogue --
+  if (!wait_bar(B, &B->o_full[t], (nkv - 1) & 1, p.status, true)) return;
+  ptx::tc_fence_after();
+  const bool store = row < w.n;
+  const long long orow = (w.out_row0 + (long long)row * w.out_stride) * D;
+  const float inv_l = 1.0f / l;
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t ov[32];
+    ptx::tmem_ld32(tO + 32 * cc, ov);
+    ptx::tmem_wait_ld();
+    float o[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if constexpr (PV8) {
+        const float acc = __fmaf_rn(alpha_prev, o32[32 * cc + i], __uint_as_float(ov[i]));
+        const float vf = __fdiv_rn(__ldg(p.v_scale + w.vs_idx * D + 32 * cc + i), 448.0f);
+        o[i] = __fmul_rn(__fmul_rn(acc, vf), inv_l);
+      } else {
+        o[i] = __fmul_rn(__uint_as_float(ov[i]), inv_l);
+      }
+    }
+    if (!store) continue;
+    if (p.out_dt == SAGE_F32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + 32 * cc);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + 32 * cc);
+      const bool ob = p.out_dt == SAGE_BF16;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t u[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = o[8 * i + 2 * e], b = o[8 * i + 2 * e + 1];
+          u[e] = ob ? In16<true>::pack(a, b) : In16<false>::pack(a, b);
+        }
+        dst[i] = make_uint4(u[0], u[1], u[2], u[3]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- kernel --
+
+template <int D, bool PV8, bool BF16V>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = Cfg<D, PV8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + 2 * C::QT;
+  uint8_t* sV = sK + C::NS * C::QT;
+  Bars* B = reinterpret_cast<Bars*>(sV + C::NS * C::VT);
+
+  const Work w = decode_work(p);
+  if (!w.valid) return;
+  const int warp = threadIdx.x / 32;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&B->q_full, 1);
+    ptx::mbar_init(&B->done, 1);
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(&B->s_full[t], 1);
+      ptx::mbar_init(&B->p_full[t], 128);
+      ptx::mbar_init(&B->o_full[t], 1);
+    }
+    for (int s = 0; s < C::NS; ++s) {
+      ptx::mbar_init(&B->k_full[s], 1);
+      ptx::mbar_init(&B->v_full[s], 1);
+      ptx::mbar_init(&B->kv_empty[s], 1);
+    }
+    B->abort = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == WARP_MMA) {
+    ptx::tmem_alloc(&B->tmem_base, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = B->tmem_base;
+
+  if (warp == WARP_TMA) {
+    if ((threadIdx.x & 31) == 0) producer<D, PV8>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, p.status);
+  } else if (warp == WARP_MMA) {
+    if ((threadIdx.x & 31) == 0) mma_issuer<D, PV8, BF16V>(w, B, tmem, sQ, sK, sV, p.status);
+  } else {
+    softmax_wg<D, PV8, BF16V>(p, w, B, tmem, warp / 4);
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == WARP_MMA) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------ QK^T tile diagnostic --
+
+// One CTA per requested tile (bh, I, J): TMA-load Q^ tile I and K^ tile J,
+// the same kind::i8 MMA sequence the attention kernel issues, then 4 warps
+// copy the int32 tile out of TMEM.
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    qk_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const int32_t* __restrict__ tiles, int32_t* __restrict__ s_out,
+                   uint32_t* status) {
+  constexpr int QT = BLK * D;
+  constexpr uint32_t SWZ = (D == 128) ? 2u : 4u;
+  constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, 128);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + QT;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * QT);
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
+  int* okflag = reinterpret_cast<int*>(tbase + 1);
+  const int bh = __ldg(tiles + 3 * blockIdx.x), I = __ldg(tiles + 3 * blockIdx.x + 1),
+            J = __ldg(tiles + 3 * blockIdx.x + 2);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar[0], 1);
+    ptx::mbar_init(&bar[1], 1);
+    ptx::fence_barrier_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(tbase, 128);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tbase;
+  if (threadIdx.x == 0) {
+    ptx::mbar_arrive_expect_tx(&bar[0], 2 * QT);
+    ptx::tma_load_3d(sA, &tm_q, &bar[0], 0, I * BLK, bh);
+    ptx::tma_load_3d(sB, &tm_k, &bar[0], 0, J * BLK, bh);
+    bool ok = ptx::mbar_wait(&bar[0], 0);
+    if (ok) {
+      ptx::tc_fence_after();
+      const uint32_t a = ptx::smem_u32(sA), b = ptx::smem_u32(sB);
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk)
+        ptx::mma_i8_ss(tmem, ptx::smem_desc(a + 32 * kk, 16, 8 * D, SWZ),
+                       ptx::smem_desc(b + 32 * kk, 16, 8 * D, SWZ), IDESC_QK, kk > 0 ? 1u : 0u);
+    }
+    ptx::mma_commit(&bar[1]);
+    ok = ptx::mbar_wait(&bar[1], 0) && ok;
+    if (!ok) set_status(status, ST_TIMEOUT);
+    *okflag = ok ? 1 : 0;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (*okflag) {
+    const int r = warp * 32 + lane;
+    int32_t* dst = s_out + (long long)blockIdx.x * BLK * BLK + (long long)r * BLK;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * cc, v);
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<int4*>(dst + 32 * cc + i) = make_int4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 128);
+}
+
+}  // namespace
+
+// =================================================================== host ==
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D tiled map over a row-major tensor [dim2][dim1][dim0] with element size
+// esz; box {b0, b1, b2}.  Returns false when the driver rejects it.
+static bool make_map3(CUtensorMap* m, CUtensorMapDataType dt, int esz, const void* base,
+                      uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes, uint64_t s2_bytes,
+                      uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  (void)esz;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static CUtensorMapSwizzle swz_for(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+}
+
+template <int D, bool PV8, bool BF16V>
+static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
+  using C = Cfg<D, PV8>;
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle cs = swz_for(D);
+  if (!make_map3(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.q_codes, D, L.code_rows, L.code_z, D,
+                 (uint64_t)D * L.code_rows, D, BLK, 1, cs) ||
+      !make_map3(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.k_codes, D, L.code_rows, L.code_z, D,
+                 (uint64_t)D * L.code_rows, D, BLK, 1, cs))
+    return cudaErrorInvalidValue;
+  const int esz = PV8 ? 1 : 2;
+  const CUtensorMapDataType vdt = PV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                      : (BF16V ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  const uint32_t vbox0 = PV8 ? D : 64;  // box inner extent in elements (128 B or 64 B)
+  const CUtensorMapSwizzle vs = swz_for(vbox0 * esz);
+  bool okv;
+  if (!L.p.varlen)
+    okv = make_map3(&tv, vdt, esz, L.v, D, L.p.N, L.p.BH, (uint64_t)D * esz,
+                    (uint64_t)D * esz * L.p.N, vbox0, BLK, 1, vs);
+  else
+    okv = make_map3(&tv, vdt, esz, L.v, D, L.p.H, L.T, (uint64_t)D * esz,
+                    (uint64_t)D * esz * L.p.H, vbox0, 1, BLK, vs);
+  if (!okv) return cudaErrorInvalidValue;
+  auto kern = attn_fwd_kernel<D, PV8, BF16V>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<L.grid, NUM_THREADS, C::SMEM, st>>>(tq, tk, tv, L.p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st) {
+  if (L.D == 64) {
+    if (L.pv8) return launch_attn_t<64, true, false>(L, st);
+    return L.bf16v ? launch_attn_t<64, false, true>(L, st) : launch_attn_t<64, false, false>(L, st);
+  }
+  if (L.pv8) return launch_attn_t<128, true, false>(L, st);
+  return L.bf16v ? launch_attn_t<128, false, true>(L, st) : launch_attn_t<128, false, false>(L, st);
+}
+
+template <int D>
+static cudaError_t launch_qk_tiles_t(const int8_t* qc, const int8_t* kc, int BH, int NP,
+                                     const int32_t* tiles, int n, int32_t* out, uint32_t* status,
+                                     cudaStream_t st) {
+  CUtensorMap tq, tk;
+  const CUtensorMapSwizzle cs = swz_for(D);
+  if (!make_map3(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qc, D, NP, BH, D, (uint64_t)D * NP, D,
+                 BLK, 1, cs) ||
+      !make_map3(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kc, D, NP, BH, D, (uint64_t)D * NP, D,
+                 BLK, 1, cs))
+    return cudaErrorInvalidValue;
+  const int smem = 1024 + 2 * BLK * D + 64;
+  auto kern = qk_tile_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<n, 128, smem, st>>>(tq, tk, tiles, out, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
+                            const int32_t* tiles, int n, int32_t* out, uint32_t* status,
+                            cudaStream_t st) {
+  return D == 64 ? launch_qk_tiles_t<64>(qc, kc, BH, NP, tiles, n, out, status, st)
+                 : launch_qk_tiles_t<128>(qc, kc, BH, NP, tiles, n, out, status, st);
+}
+
+}  // namespace sage

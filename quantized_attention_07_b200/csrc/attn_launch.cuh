@@ -1,0 +1,43 @@
+// Host/device interface of the fused attention kernel.
+#pragma once
+
+#include "common.cuh"
+
+namespace sage {
+
+struct AttnParams {
+  int H, N, BH;          // dense: N, BH = B*H
+  int NB;                // dense: key blocks per head = ceil(N/128)
+  int NPAIR;             // dense: query tile pairs per head = ceil(N/256)
+  int causal;
+  float kappa;           // fp32(sm_scale * log2 e)
+  const float* q_scale;  // dense [BH][NB]; varlen [H][TBmax]
+  const float* k_scale;
+  const float* v_scale;  // FP8: dense [BH][D]; varlen [batch][H][D]
+  void* out;
+  int out_dt;
+  // varlen
+  int varlen;
+  const int32_t* cu;
+  const int32_t* blk_off;
+  const int32_t* pair_off;
+  int batch;
+  int TBmax;
+  uint32_t* status;
+};
+
+struct AttnLaunch {
+  AttnParams p;
+  int D, pv8, bf16v;
+  const int8_t* q_codes;
+  const int8_t* k_codes;
+  const void* v;         // 16-bit V (FP16 mode) or E4M3 codes (FP8 mode)
+  int code_rows;         // rows per z-slice of the code arrays (NP or TBmax*128)
+  int code_z;            // BH (dense) or H (varlen)
+  int T;                 // varlen tokens
+  dim3 grid;
+};
+
+cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st);
+
+}  // namespace sage

@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every function include/sage.h declares, and
+its host-side logic (sizes, argument validation) behaves as documented.  No
+call here reaches the GPU: every call either computes sizes or is rejected by
+host-side validation before anything is launched."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_attention_07_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sage.h")
+
+FAKE = 0x10000  # a 16-byte aligned non-null "device pointer" never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions() -> list[str]:
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sage_attn_fwd", "sage_attn_fwd_varlen", "sage_quantize",
+                     "sage_attn_quantized", "sage_quantize_varlen", "sage_sync_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # and the binding attaches a signature to each of them
+    assert set(declared_functions()) == set(_lib.SIGNATURES)
+
+
+def test_workspace_sizes(lib):
+    B, H, N, D = 1, 32, 32768, 128
+    NP = N
+    fp16 = lib.sage_workspace_bytes(B, H, N, D, 0)
+    fp8 = lib.sage_workspace_bytes(B, H, N, D, 1)
+    codes = 2 * B * H * NP * D
+    assert codes < fp16 < codes + (1 << 20)
+    assert fp8 - fp16 >= B * H * N * D            # FP8 V codes
+    assert lib.sage_workspace_bytes(1, 1, 100, 96, 0) == 0   # rejected shapes -> 0
+    assert lib.sage_workspace_bytes(1, 1, 0, 64, 0) == 0
+    assert lib.sage_workspace_bytes(1, 1, 1 << 23, 64, 0) == 0
+    v = lib.sage_workspace_bytes_varlen(34000, 8, 32, 128, 1)
+    assert v > 2 * 32 * 34000 * 128
+    assert lib.sage_scratch_bytes(2, 16, 128) >= 256 + 2 * 16 * 128 * 12
+
+
+def test_status_strings(lib):
+    for code, name in ((0, b"SAGE_OK"), (1, b"SAGE_ERR_INVALID_ARG"), (5, b"SAGE_ERR_TIMEOUT"),
+                       (6, b"SAGE_ERR_BAD_SEQLENS"), (7, b"SAGE_ERR_RANGE")):
+        assert lib.sage_status_string(code) == name
+
+
+def _fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, in_dt=0, out_dt=0, B=1, H=2, N=256, D=64,
+             causal=0, sm_scale=0.0, pv_mode=0, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return lib.sage_attn_fwd(*a.values())
+
+
+@pytest.mark.parametrize("bad", [dict(D=96), dict(D=0), dict(N=0), dict(B=0), dict(H=-1),
+                                 dict(pv_mode=2), dict(in_dt=2), dict(out_dt=7),
+                                 dict(q=None), dict(v=FAKE + 8), dict(out=FAKE + 2),
+                                 dict(ws=None), dict(sm_scale=float("nan")),
+                                 dict(N=(1 << 22) + 1), dict(B=300, H=300)])
+def test_invalid_arguments_rejected_on_host(lib, bad):
+    assert _fwd(lib, **bad) == 1
+
+
+def test_small_workspace_rejected_on_host(lib):
+    need = lib.sage_workspace_bytes(1, 2, 256, 64, 0)
+    assert _fwd(lib, ws_bytes=need - 1) == 3
+
+
+def test_varlen_and_stage_validation(lib):
+    f = lib.sage_attn_fwd_varlen
+    # batch 0, D=96, null cu_seqlens
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 0, 100, 100, 2, 64, 0, 0.0, 0, FAKE, 1 << 40, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 100, 100, 2, 96, 0, 0.0, 0, FAKE, 1 << 40, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 0, None, 1, 100, 100, 2, 64, 0, 0.0, 0, FAKE, 1 << 40, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 100, 100, 2, 64, 0, 0.0, 0, FAKE, 1000, None) == 3
+    q = lib.sage_quantize
+    # FP8 mode without V codes
+    assert q(FAKE, FAKE, FAKE, 0, 1, 2, 256, 64, 1, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+             FAKE, 1 << 30, None) == 1
+    assert q(FAKE, FAKE, None, 0, 1, 2, 256, 64, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+             FAKE, 16, None) == 3
+    t = (ctypes.c_int32 * 3)(0, 5, 0)   # tile row out of range for NP = 256
+    assert lib.sage_qk_int8_tiles(FAKE, FAKE, 1, 256, 64, ctypes.cast(t, ctypes.c_void_p), 1,
+                                  FAKE, FAKE, 1 << 20, None) == 1

@@ -1,0 +1,161 @@
+"""GPU parity: the CUDA library against the CPU oracle on the same seeded inputs.
+
+  * quantisation outputs (codes, deltas, K mean, FP8 V codes/scales): bit-exact,
+  * int32 QK^T tiles from the tcgen05 INT8 path: bit-exact,
+  * attention output: within the stated max-abs tolerance of the oracle's
+    emulation of the method (fp32 output, and 16-bit output with half an ulp
+    of slack), and cosine >= 0.999 against the fp64 reference (or, where the
+    method's own accuracy is lower, no worse than the emulation's cosine).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_07_b200 as sage
+from oracle import heads
+from quantized_attention_07_b200 import workloads as W
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from quantized_attention_07_b200 import build
+    build.build()
+    oracle.build()
+    assert torch.cuda.is_available()
+
+
+# ----------------------------------------------------------- quantisation --
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("N", [1, 127, 300, 1000])
+@pytest.mark.parametrize("pv_mode", ["fp16", "fp8"])
+def test_quantize_bit_exact_small(D, dtype, N, pv_mode):
+    q, k, v = W.make_dense(2, 3, N, D, dtype, bias_sigma=3.0, outlier_p=0.01, outlier_scale=20.0,
+                           seed=1000 + N + D)
+    qz = U.gpu_quantize_dense(q, k, v, pv_mode)
+    U.compare_quant_dense(qz, heads.quantize(q, k, v, None, pv_mode), pv_mode)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_quantize_bit_exact_full_workloads(name):
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl)
+    ref = heads.quantize(inp.q, inp.k, inp.v, inp.cu_seqlens, wl.pv_mode)
+    if wl.varlen:
+        dev = torch.device("cuda")
+        qz = sage.quantize_varlen(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev),
+                                  inp.cu_seqlens.to(dev), max(inp.seqlens), wl.pv_mode)
+        torch.cuda.synchronize()
+        sage.sync_status()
+        U.compare_quant_varlen(qz, ref, inp.cu_seqlens, wl.pv_mode)
+    else:
+        qz = U.gpu_quantize_dense(inp.q, inp.k, inp.v, wl.pv_mode)
+        U.compare_quant_dense(qz, ref, wl.pv_mode)
+
+
+def test_constant_k_channels_give_zero_codes():
+    """K constant over tokens: the smoothed K is exactly zero (mean is exact)."""
+    q, k, v = W.make_dense(1, 2, 333, 128, "fp16", bias_sigma=5.0, seed=7, k_const_over_tokens=True)
+    qz = U.gpu_quantize_dense(q, k, v, "fp16")
+    assert not qz.k_codes.any().item() and not qz.k_scale.any().item()
+    assert torch.equal(qz.k_mean.cpu(), k[:, :, 0, :].float())
+
+
+# ----------------------------------------------------------- INT8 QK^T --
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_qk_int8_tiles_bit_exact(D):
+    rng = np.random.default_rng(D)
+    B, H, NP = 1, 3, 512
+    qc = torch.from_numpy(rng.integers(-127, 128, size=(B, H, NP, D)).astype(np.int8))
+    kc = torch.from_numpy(rng.integers(-127, 128, size=(B, H, NP, D)).astype(np.int8))
+    qc[0, 1, 5, :] = 127
+    kc[0, 1, 9, :] = -127                       # extreme products
+    tiles = [(0, 0, 0), (1, 0, 0), (1, 3, 2), (2, 1, 3), (2, 3, 3)]
+    S = sage.qk_int8_tiles(qc.cuda(), kc.cuda(), tiles).cpu().numpy()
+    sage.sync_status()
+    for t, (bh, I, J) in enumerate(tiles):
+        ref = oracle.qk_int(qc[0, bh].numpy(), kc[0, bh].numpy(), I * 128, 128, J * 128, 128)
+        assert np.array_equal(S[t], ref), (bh, I, J)
+
+
+def test_qk_int8_tiles_of_quantised_workload():
+    wl = W.WORKLOADS["llm_causal_2k"]
+    q, k, v = W.make_dense(1, 2, 2048, 128, "bf16", 3.0, seed=wl.seed)
+    qz = U.gpu_quantize_dense(q, k, v, "fp16")
+    tiles = [(0, 0, 0), (0, 15, 15), (1, 15, 0), (1, 7, 8), (0, 3, 12)]
+    S = sage.qk_int8_tiles(qz.q_codes, qz.k_codes, tiles).cpu().numpy()
+    qc, kc = qz.q_codes.cpu().numpy(), qz.k_codes.cpu().numpy()
+    for t, (bh, I, J) in enumerate(tiles):
+        ref = qc[0, bh, I * 128:(I + 1) * 128].astype(np.int64) @ \
+            kc[0, bh, J * 128:(J + 1) * 128].astype(np.int64).T
+        assert np.array_equal(S[t].astype(np.int64), ref)
+
+
+# ------------------------------------------------------------- attention --
+
+SMALL = [
+    # (B, H, N, D, dtype, causal, pv_mode)
+    (1, 2, 256, 64, "fp16", False, "fp16"),
+    (1, 2, 256, 128, "fp16", False, "fp16"),
+    (2, 1, 300, 128, "bf16", True, "fp16"),
+    (1, 2, 777, 64, "bf16", False, "fp16"),
+    (1, 2, 777, 64, "fp16", True, "fp16"),
+    (1, 1, 1, 128, "fp16", False, "fp16"),
+    (1, 1, 1, 64, "bf16", True, "fp8"),
+    (1, 2, 127, 128, "fp16", True, "fp8"),
+    (1, 2, 640, 64, "fp16", False, "fp8"),
+    (2, 2, 513, 128, "bf16", False, "fp8"),
+    (1, 2, 1000, 128, "bf16", True, "fp8"),
+    (1, 3, 129, 64, "fp16", True, "fp16"),
+]
+
+
+@pytest.mark.parametrize("B,H,N,D,dtype,causal,pv_mode", SMALL)
+def test_attention_small_all_rows(B, H, N, D, dtype, causal, pv_mode):
+    q, k, v = W.make_dense(B, H, N, D, dtype, bias_sigma=3.0, seed=N * 7 + D)
+    picks = [(b * H + h, h, i) for b in range(B) for h in range(H) for i in range(N)]
+    # dense picks index [B, H] as (b, h); emulate/reference take (seq=b, head=h)
+    picks = [(b, h, i) for b in range(B) for h in range(H) for i in range(N)]
+    U.check_against_oracle(q, k, v, None, causal, pv_mode, picks)
+
+
+def test_attention_custom_scale():
+    q, k, v = W.make_dense(1, 2, 384, 64, "fp16", 2.0, seed=5)
+    picks = [(0, h, i) for h in range(2) for i in range(0, 384, 5)]
+    U.check_against_oracle(q, k, v, None, False, "fp16", picks, sm_scale=0.05)
+
+
+def test_attention_varlen_small():
+    lens = [1, 129, 300, 0, 511, 64]
+    for causal, pv_mode, dt in ((True, "fp8", "bf16"), (False, "fp16", "fp16"),
+                                (True, "fp16", "bf16"), (False, "fp8", "fp16")):
+        q, k, v, cu = W.make_varlen(lens, 2, 128 if pv_mode == "fp8" else 64, dt, seed=11)
+        picks = [(s, h, i) for s, n in enumerate(lens) for h in range(2) for i in range(n)]
+        U.check_against_oracle(q, k, v, cu, causal, pv_mode, picks)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_attention_full_workloads_sampled_rows(name):
+    """Each workload at full size, in the launch configuration the benchmark
+    times; the oracle checks 512 seeded rows (all rows for the small one)."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl)
+    lens = inp.seqlens
+    if wl.varlen:
+        picks = W.sample_rows(lens, wl.H, 512, seed=wl.seed)
+    elif wl.B * wl.H * wl.N <= 4096:
+        picks = [(b, h, i) for b in range(wl.B) for h in range(wl.H) for i in range(wl.N)]
+    else:
+        flat = W.sample_rows([wl.N] * wl.B, wl.H, 512, seed=wl.seed)
+        picks = flat
+    stats = U.check_against_oracle(inp.q, inp.k, inp.v, inp.cu_seqlens, wl.causal, wl.pv_mode,
+                                   picks)
+    print(name, stats)
