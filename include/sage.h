@@ -195,6 +195,36 @@ sage_status_t sage_quantize_varlen(const void* q, const void* k, const void* v, 
                                    float* k_mean, uint8_t* v_codes, float* v_scale, void* ws,
                                    size_t ws_bytes, void* stream);
 
+/*
+ * Stage 1 of a dense problem without a workspace: the same smoothing and
+ * quantisation, outputs and layouts as sage_quantize, but its reduction
+ * scratch (exact K channel sums, V channel maxima, status word) lives in a
+ * fixed SAGE_NOALLOC_SCRATCH_BYTES array of device memory inside the library.
+ * The SageAttention pages have no counterpart of this entry point; it exists
+ * for callers that may not allocate device memory and cannot pass a
+ * workspace (for instance an extension whose host application owns every
+ * device allocation, or a path that must not pay cudaMalloc's implicit
+ * synchronisation).  It allocates nothing.
+ *   status_out : optional DEVICE uint32; cleared by the call, then OR-ed with
+ *                4 when a K element is non-finite or |k| >= 65536.  NULL:
+ *                such errors are not reported.
+ * Limits and rules:
+ *   - B*H*D <= SAGE_NOALLOC_MAX_BHD, else SAGE_ERR_WORKSPACE (nothing runs).
+ *   - Every call shares the one array (per device) and it keeps the last
+ *     call's contents; calls whose GPU work overlaps in time (other streams,
+ *     other host threads) race on it.
+ *   - The first call on a device looks the array's address up with that
+ *     device current; make that first call before any stream capture.
+ *   - Each GPU that loads the library holds the array until the process exits.
+ */
+#define SAGE_NOALLOC_SCRATCH_BYTES (1 << 20)
+#define SAGE_NOALLOC_MAX_BHD 65536
+sage_status_t sage_quantize_noalloc(const void* q, const void* k, const void* v, int in_dt, int B,
+                                    int H, int N, int D, int pv_mode, int8_t* q_codes,
+                                    float* q_scale, int8_t* k_codes, float* k_scale,
+                                    float* k_mean, uint8_t* v_codes, float* v_scale,
+                                    uint32_t* status_out, void* stream);
+
 /* ------------------------------------------------------------ diagnostics -- */
 
 /*
