@@ -106,6 +106,24 @@ def recorded_traffic(workload: str):
     return None
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(wl, rank: int):
+    """Each rank's independent, seeded instance of the workload (weak scaling)."""
+    return wl if rank == 0 else dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
+
+
+def job_throughput(ops_per_rank: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job TOPS: the work of all ranks over the slowest rank's time."""
+    return ops_per_rank * world * steps / (max_ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -169,7 +187,7 @@ def run_ours(args, rank, world, local):
     if args.heads:
         wl = dataclasses.replace(wl, H=args.heads)
     # each rank: its own seeded instance of the workload
-    inp = W.make_inputs(wl if rank == 0 else dataclasses.replace(wl, seed=wl.seed + 1000 * rank))
+    inp = W.make_inputs(rank_workload(wl, rank))
     ops = W.attention_ops(wl, inp.seqlens)
     q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
     cu = inp.cu_seqlens.to(dev) if inp.cu_seqlens is not None else None
@@ -230,10 +248,7 @@ def run_ours(args, rank, world, local):
     total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
     attn_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
     quant_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     # end to end through the public call with host buffers: pinned H2D of the
     # step's inputs, the forward pass, D2H of the output, every step.
@@ -265,12 +280,10 @@ def run_ours(args, rank, world, local):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(ems, op=torch.distributed.ReduceOp.MAX)
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
         ws.sync_status()
         h2d = in_bytes + (hcu.numel() * 4 if hcu is not None else 0)
-        e2e = {"value": ops * world * Ke / (float(ems.item()) * 1e-3) / 1e12, "unit": "TOPS",
+        e2e = {"value": round(job_throughput(ops, world, Ke, ems), 2), "unit": "TOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out.numel() * out.element_size(),
                "steps": Ke}
 
@@ -287,7 +300,7 @@ def run_ours(args, rank, world, local):
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = ops / (attn_avg_ms * 1e-3) / 1e12
     peak = tensor_peak(pk, wl.pv_mode)
-    value = ops * world * K / (total_ms * 1e-3) / 1e12
+    value = job_throughput(ops, world, K, total_ms)
     clocks = clk.summary()
     line = {
         "metric": METRIC,

@@ -1,0 +1,57 @@
+"""The multi-GPU path of bench.py, on CPU with two gloo ranks: every rank gets
+its own independent seeded problem (no data-path exchange), the step time is
+the max over ranks, and the job throughput counts the work of all ranks."""
+from __future__ import annotations
+
+import os
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from quantized_attention_07_b200 import workloads as W
+
+
+def _worker(rank: int, world: int, port: int, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = W.WORKLOADS["small_d64"]
+        mine = W.make_inputs(bench.rank_workload(wl, rank))
+        # gather a fingerprint of every rank's inputs: problems must differ
+        fp = torch.tensor([float(mine.q.float().sum()), float(mine.k.float().sum())])
+        allfp = [torch.zeros(2) for _ in range(world)]
+        dist.all_gather(allfp, fp)
+        local_ms = 10.0 + 5.0 * rank           # rank 1 is the slow one
+        mx = bench.max_over_ranks(local_ms, torch.device("cpu"))
+        ops = W.attention_ops(wl)
+        q.put((rank, mx, bench.job_throughput(ops, world, 4, mx),
+               [t.tolist() for t in allfp]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_and_independent_problems():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ops = W.attention_ops(W.WORKLOADS["small_d64"])
+    for rank, mx, tops, fps in res:
+        assert mx == 15.0                                   # max over ranks
+        assert tops == pytest.approx(ops * 2 * 4 / 15e-3 / 1e12)
+        assert fps[0] != fps[1]                             # independent problems
+
+
+def test_single_process_defaults():
+    assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
+    assert bench.rank_workload(W.WORKLOADS["long_32k"], 0) is W.WORKLOADS["long_32k"]
