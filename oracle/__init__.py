@@ -28,6 +28,11 @@ _CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
 ORACLE_OK = 0
 ORACLE_ERR_RANGE = 1
 
+# Key-tile length of the online softmax (and of the FP8 two-level flush).
+# FlashAttention's tiling has no fixed tile size on the pages; 64 keys is the
+# reading taken (the quantisation block stays 128 tokens).
+KV_TILE = 64
+
 
 def build(force: bool = False) -> str:
     """Compile sage_oracle.c into liboracle.so (gcc, no fast-math, no FP contraction)."""
@@ -58,8 +63,8 @@ def lib():
         L.oracle_qk_int.argtypes = [P, P, i32, i64, i32, i64, i32, P]; L.oracle_qk_int.restype = None
         L.oracle_attn_ref_rows.argtypes = [P, P, P, i64, i32, i64, i64, i64, f64, i32, P, i64, P]
         L.oracle_attn_ref_rows.restype = None
-        L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, f32, i32, i32,
-                                            i32, P, i64, P]
+        L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, i32, f32, i32,
+                                            i32, i32, P, i64, P]
         L.oracle_attn_emul_rows.restype = None
         _lib = L
     return _lib
@@ -169,8 +174,11 @@ def attn_ref_rows(q, k, v, sm_scale: float, causal: bool, rows) -> np.ndarray:
 
 def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, causal: bool,
                    pv_mode: str, rows, v=None, p16: str = "fp16", vc=None, vdelta=None,
-                   blk: int = 128) -> np.ndarray:
-    """The quantised method's output rows (fp32) for one head; see sage_oracle.c."""
+                   blk: int = 128, kv: int = KV_TILE) -> np.ndarray:
+    """The quantised method's output rows (fp32) for one head; see sage_oracle.c.
+    blk: quantisation block (tokens); kv: key tile of the online softmax."""
+    if blk % kv:
+        raise ValueError("the key tile must divide the quantisation block")
     qc = np.ascontiguousarray(qc, dtype=np.int8)
     kc = np.ascontiguousarray(kc, dtype=np.int8)
     qdelta, kdelta = _f32(qdelta), _f32(kdelta)
@@ -184,6 +192,6 @@ def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, caus
         vdelta = _f32(vdelta)
         vc_p, vd_p, v_p, ldv, mode = _p(vc), _p(vdelta), None, D, 1
     lib().oracle_attn_emul_rows(_p(qc), _p(qdelta), _p(kc), _p(kdelta), v_p, ldv, vc_p, vd_p, n,
-                                D, blk, float(kappa(sm_scale)), int(causal), mode,
+                                D, blk, kv, float(kappa(sm_scale)), int(causal), mode,
                                 1 if p16 == "bf16" else 0, _p(rows), len(rows), _p(out))
     return out

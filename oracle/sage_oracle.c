@@ -315,12 +315,15 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *
  * Inputs are the outputs of the steps above: q codes/deltas, k codes/deltas
  * (smoothed K), and either the 16-bit V values (pv_mode 0) or V's E4M3 codes
- * and per-channel deltas (pv_mode 1).  `blk` is both the quantisation block
- * and the key-block length of the tiled softmax.  kappa = fp32(sm_scale *
- * log2(e)): the softmax runs in base 2.
+ * and per-channel deltas (pv_mode 1).  `blk` is the quantisation block; `kv`
+ * (a divisor of blk) is the key-tile length of the tiled online softmax and of
+ * the FP8 two-level flush -- the pages give FlashAttention's tiling without a
+ * tile size ("Attention机制优化", section 3.1); the reading taken is 64 keys.
+ * kappa = fp32(sm_scale * log2(e)): the softmax runs in base 2.
  *
- * For each row i (query block I = i / blk) and key block J = 0, 1, ... in
- * ascending order (only J <= I when causal), with m = -inf, l = 0, O = 0:
+ * For each row i (query block I = i / blk) and key tile T = 0, 1, ... in
+ * ascending order (tiles starting at or before i when causal), the tile's keys
+ * lying in quantisation block J = T*kv / blk, with m = -inf, l = 0, O = 0:
  *
  *   S_ij   = sum_d q^_id k^_jd                       exact int32
  *   c_IJ   = fp32( fp32(deltaQ_I * deltaK_J) * kappa )   dequant x softmax scale
@@ -349,30 +352,33 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *           out_d = fp32(fp32(O_d * fp32(deltaV_d / 448)) / l)   (pv_mode 1).
  *
  * Masked keys (j >= n, or j > i when causal) take no part in the maximum and
- * contribute p = 0.
+ * contribute p = 0.  (A tile is entered only if it holds at least one
+ * unmasked key of the row.)
  *
  * p16_format: 0 = fp16, 1 = bf16 (V's own format, used for P in pv_mode 0).
  * out: [nrows][D] fp32.
  */
 void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* kc,
                            const float* kdelta, const float* v, long ldv, const uint8_t* vc,
-                           const float* vdelta, long n, int D, int blk, float kappa, int causal,
-                           int pv_mode, int p16_format, const long* rows, long nrows, float* out)
+                           const float* vdelta, long n, int D, int blk, int kv, float kappa,
+                           int causal, int pv_mode, int p16_format, const long* rows, long nrows,
+                           float* out)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (long r = 0; r < nrows; ++r) {
         long i = rows[r];
         long I = i / blk;
-        long nblk = (n + blk - 1) / blk;
-        long Jend = causal ? I + 1 : nblk;
+        long ntile = (n + kv - 1) / kv;
+        long Tend = causal ? i / kv + 1 : ntile;
         float m = -INFINITY, l = 0.0f;
         float* O = (float*)calloc((size_t)D, sizeof(float));
         double* part = (double*)malloc(sizeof(double) * (size_t)D);
-        int32_t* S = (int32_t*)malloc(sizeof(int32_t) * (size_t)blk);
-        float* p = (float*)malloc(sizeof(float) * (size_t)blk);
-        for (long J = 0; J < Jend; ++J) {
-            long j0 = J * blk;
-            long j1 = j0 + blk < n ? j0 + blk : n;
+        int32_t* S = (int32_t*)malloc(sizeof(int32_t) * (size_t)kv);
+        float* p = (float*)malloc(sizeof(float) * (size_t)kv);
+        for (long T = 0; T < Tend; ++T) {
+            long j0 = T * kv;
+            long J = j0 / blk;
+            long j1 = j0 + kv < n ? j0 + kv : n;
             if (causal && j1 > i + 1) j1 = i + 1;
             int nj = (int)(j1 - j0);
             int32_t smax = INT32_MIN;

@@ -1,28 +1,30 @@
 // Fused SageAttention forward kernel for sm_100a.
 //
 // One CTA handles two 128-row query tiles of one (sequence, head) and streams
-// that head's key/value tiles through shared memory:
+// that head's keys and values through shared memory in 128-key stages; the
+// online softmax works on 64-key sub-tiles.
 //
-//   warp 8       TMA producer: Q^ tiles once, then K^_j and V_j into an
-//                NS-stage ring (cp.async.bulk.tensor, mbarrier complete_tx).
-//   warp 9       MMA issuer (one thread) and TMEM owner:
-//                  S_t  = Q^_t K^_j^T        tcgen05.mma kind::i8 -> int32 TMEM
-//                  O_t += P_t V_j            kind::f16 (16-bit P.V), or
-//                  Part_t = P^_t V^_j        kind::f8f6f4 (FP8 P.V), with P read
-//                                            from TMEM and V from shared memory.
-//   warps 0-3    softmax for query tile 0, warps 4-7 for query tile 1, one
-//                thread per query row: read S from TMEM, dequantise with
-//                deltaQ*deltaK*sm_scale*log2(e), mask, online softmax in base 2,
-//                write P (fp16/bf16 or e4m3) back over S, rescale O (16-bit P.V)
-//                or fold the block's FP8 partial into an fp32 register
-//                accumulator (two-level accumulation), and finally normalise
-//                and store the output row.
+//   control warpgroup (warp 0 of it: TMA producer; warp 1: TMEM owner and
+//                single-thread MMA issuer):
+//                  S_t[b]  = Q^_t K^_i^T     tcgen05.mma kind::i8 -> int32 TMEM
+//                  O_t    += P_t[b] V_i      kind::f16 (16-bit P.V), or
+//                  Part_t  = P^_t[b] V^_i    kind::f8f6f4 (FP8 P.V),
+//                P read from TMEM (written over S), V from shared memory.
+//   softmax warpgroups 0 and 1 (one per query tile, one thread per row):
+//                read S from TMEM, dequantise with deltaQ*deltaK*sm_scale*log2 e,
+//                mask, online softmax in base 2, write P (fp16/bf16 or e4m3)
+//                back over S; FP8: fold the previous sub-tile's partial into an
+//                fp32 register accumulator (two-level accumulation).
+//   correction warpgroup (16-bit P.V only): O_t <- alpha * O_t in TMEM when a
+//                row maximum grew, between two P.V accumulations, off the
+//                softmax warps' path.
 //
-// The two query tiles ping-pong: while one tile's softmax runs on the CUDA
-// cores, the tensor core works on the other tile's P.V and next QK^T.
+// Each query tile owns two 64-column S buffers, so QK^T of sub-tile i+1 runs
+// on the tensor core while the softmax works on sub-tile i, and the two query
+// tiles keep both softmax warpgroups busy.
 //
-// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).
+// TMEM columns (512): S_0[0] [0,64) S_0[1] [64,128) S_1[0] [128,192)
+// S_1[1] [192,256) O_0 [256,256+D) O_1 [256+D,256+2D).
 //
 // Method steps (SageAttention pages): INT8 QK^T with the per-block deltas
 // ("SageAttention -- brand new attention", quantisation intro step 3 and
@@ -42,38 +44,56 @@ namespace sage {
 
 namespace {
 
-constexpr int NUM_THREADS = 320;
-constexpr int WARP_TMA = 8;
-constexpr int WARP_MMA = 9;
+constexpr int SUB = 64;  // keys per softmax sub-tile
 
 template <int D, bool PV8>
 struct Cfg {
+  // warpgroups: 2 softmax, [1 correction (16-bit P.V)], 1 control
+  static constexpr int WGS = PV8 ? 3 : 4;
+  static constexpr int THREADS = WGS * 128;
+  static constexpr int WG_CTRL = WGS - 1;
+  static constexpr int WG_CORR = 2;
+  // register split, summing to the launch allocation (65536 regs for 512
+  // threads at 128 each; 64512 for 384 threads at 168 each)
+  static constexpr int REG_SOFTMAX = PV8 ? 224 : 192;
+  static constexpr int REG_CORR = 80;
+  static constexpr int REG_CTRL = PV8 ? 56 : 48;
+  static_assert(PV8 ? (256 * 224 + 128 * 56 <= 384 * 168)
+                    : (256 * 192 + 128 * 80 + 128 * 48 <= 65536),
+                "register split exceeds the launch allocation");
+
   static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
   static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
-  static constexpr int SMEM_BUDGET = 227 * 1024 - 2048;
+  static constexpr int AUX = 4096;                      // barriers + alpha exchange
+  static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - AUX;
   static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT);
-  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;    // pipeline stages
-  static constexpr int SMEM = 1024 + 2 * QT + NS * (QT + VT) + 512;
-  // swizzle of the int8 code tiles: rows of D bytes
-  static constexpr uint32_t QK_SWZ = (D == 128) ? 2u : 4u;  // 128B : 64B
+  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;    // pipeline stages (128 keys each)
+  static constexpr int SMEM = 1024 + 2 * QT + NS * (QT + VT) + AUX;
+  // int8 code tiles: rows of D bytes
+  static constexpr uint32_t QK_SWZ = (D == 128) ? 2u : 4u;  // 128B : 64B swizzle
   static constexpr uint32_t QK_SBO = 8 * D;                 // 8 rows
+  static constexpr uint32_t K_SUB_BYTES = SUB * D;          // 64 keys of K^
   // V tiles, MN-major (D contiguous): 16-bit -> 64-element (128 B) atoms;
   // 8-bit -> one atom of D bytes.
   static constexpr int V_ROW_BYTES = PV8 ? D : 128;
   static constexpr uint32_t V_SWZ = (V_ROW_BYTES == 128) ? 2u : 4u;
   static constexpr uint32_t V_SBO = 8 * V_ROW_BYTES;         // 8 keys
   static constexpr uint32_t V_LBO = BLK * 128;               // next 64-column atom (16-bit)
+  static constexpr uint32_t V_SUB_BYTES = (SUB / 8) * V_SBO; // 64 keys
   static constexpr int PV_KSTEP = PV8 ? 32 : 16;             // keys per MMA
   static constexpr uint32_t V_KSTEP_BYTES = (PV_KSTEP / 8) * V_SBO;
-  static constexpr int PV_STEPS = BLK / PV_KSTEP;
+  static constexpr int PV_STEPS = SUB / PV_KSTEP;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(NS >= 2, "need at least two stages");
 };
 
 struct Bars {
-  uint64_t q_full;
-  uint64_t s_full[2], p_full[2], o_full[2];
-  uint64_t done;
+  uint64_t q_full, done;
+  uint64_t s_full[2][2];   // [tile][S buffer]: QK^T of a sub-tile landed
+  uint64_t p_full[2][2];   // P of a sub-tile written (128 softmax threads)
+  uint64_t o_ready[2][2];  // 16-bit P.V: O rescaled for the sub-tile (128 correction threads)
+  uint64_t o_full[2];      // P.V of a sub-tile completed
+  uint64_t o_done[2];      // the last P.V of a query tile completed (one phase)
   uint64_t k_full[8], v_full[8], kv_empty[8];
   uint32_t tmem_base;
   volatile int abort;
@@ -105,18 +125,18 @@ struct Work {
   int valid;
   int n;                 // sequence length (queries = keys)
   int pair;              // query tile pair index within the sequence
-  int head;              // h
   int code_z;            // z coordinate of this head in the Q^/K^ code maps
   int q_y0;              // y coordinate of query tile 0 in the code map
   int k_y0;              // y coordinate of key tile 0 in the code map
   int v_y0, v_z0;        // TMA coordinates of V tile 0 (x = column)
   int v_tok_on_z;        // tokens advance along z (varlen) instead of y (dense)
   long long qs_idx0;     // q_scale index of query tile 0
-  long long ks_idx0;     // k_scale index of key tile 0
+  long long ks_idx0;     // k_scale index of key block 0
   long long out_row0;    // row (in units of D elements) of token 0 of the output
   long long out_stride;  // rows between consecutive tokens
   long long vs_idx;      // v_scale row index (FP8)
-  int nkv[2];            // key tiles for query tile 0 / 1 (0 = tile absent)
+  int nsub0, nsub1;      // 64-key sub-tiles for query tile 0 / 1 (0 = tile absent)
+  int nkv;               // 128-key stages to stream
 };
 
 __device__ __forceinline__ Work decode_work(const AttnParams& p) {
@@ -133,7 +153,6 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
       pair = idx % p.NPAIR;
     }
     n = p.N;
-    w.head = bh % p.H;
     w.code_z = bh;
     w.q_y0 = pair * 2 * BLK;
     w.k_y0 = 0;
@@ -156,7 +175,6 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
     const int npairs = __ldg(p.pair_off + s + 1) - __ldg(p.pair_off + s);
     pair = npairs - 1 - (item - __ldg(p.pair_off + s));  // diagonal-heavy pairs first
     const int blk0 = __ldg(p.blk_off + s);
-    w.head = h;
     w.code_z = h;
     w.q_y0 = (blk0 + 2 * pair) * BLK;
     w.k_y0 = blk0 * BLK;
@@ -172,12 +190,11 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
   w.valid = 1;
   w.n = n;
   w.pair = pair;
-  const int nb = (n + BLK - 1) / BLK;
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qt = 2 * pair + t;
-    w.nkv[t] = (qt * BLK >= n) ? 0 : (p.causal ? min(nb, qt + 1) : nb);
-  }
+  const int ns = (n + SUB - 1) / SUB;
+  int q0 = 2 * pair, q1 = 2 * pair + 1;
+  w.nsub0 = (q0 * BLK >= n) ? 0 : (p.causal ? min(ns, 2 * q0 + 2) : ns);
+  w.nsub1 = (q1 * BLK >= n) ? 0 : (p.causal ? min(ns, 2 * q1 + 2) : ns);
+  w.nkv = (max(w.nsub0, w.nsub1) + 1) / 2;
   return w;
 }
 
@@ -188,27 +205,34 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
                          const Work& w, Bars* B, uint8_t* sQ, uint8_t* sK, uint8_t* sV,
                          uint32_t* status) {
   using C = Cfg<D, PV8>;
-  ptx::prefetch_tmap(tm_q);
-  ptx::prefetch_tmap(tm_k);
-  ptx::prefetch_tmap(tm_v);
-  // both Q^ tiles (an absent second tile reads zero-filled or padding rows)
-  ptx::mbar_arrive_expect_tx(&B->q_full, 2 * C::QT);
-  ptx::tma_load_3d(sQ, tm_q, &B->q_full, 0, w.q_y0, w.code_z);
-  ptx::tma_load_3d(sQ + C::QT, tm_q, &B->q_full, 0, w.q_y0 + BLK, w.code_z);
-  const int nkv = max(w.nkv[0], w.nkv[1]);
+  // The whole warp runs this loop (uniform control flow); one elected lane
+  // issues each TMA instruction.
+  if (ptx::elect_one()) {
+    ptx::prefetch_tmap(tm_q);
+    ptx::prefetch_tmap(tm_k);
+    ptx::prefetch_tmap(tm_v);
+    // both Q^ tiles (an absent second tile reads zero-filled or padding rows)
+    ptx::mbar_arrive_expect_tx(&B->q_full, 2 * C::QT);
+    ptx::tma_load_3d(sQ, tm_q, &B->q_full, 0, w.q_y0, w.code_z);
+    ptx::tma_load_3d(sQ + C::QT, tm_q, &B->q_full, 0, w.q_y0 + BLK, w.code_z);
+  }
+  __syncwarp();
   int j = 0;
-  for (; j < nkv; ++j) {
+  for (; j < w.nkv; ++j) {
     const int s = j % C::NS;
-    if (j >= C::NS && !wait_bar(B, &B->kv_empty[s], ((j / C::NS) - 1) & 1, status, false)) break;
-    ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT);
-    ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.code_z);
-    ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
-    uint8_t* dst = sV + s * C::VT;
-    const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
-    const int z = w.v_tok_on_z ? w.v_z0 + j * BLK : w.v_z0;
-    ptx::tma_load_3d(dst, tm_v, &B->v_full[s], 0, y, z);
-    if (!PV8 && D == 128)  // 16-bit V rows are 256 B: second 64-column box
-      ptx::tma_load_3d(dst + BLK * 128, tm_v, &B->v_full[s], 64, y, z);
+    if (j >= C::NS && !wait_bar(B, &B->kv_empty[s], ((j / C::NS) - 1) & 1, status, true)) break;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT);
+      ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.code_z);
+      ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
+      uint8_t* dst = sV + s * C::VT;
+      const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
+      const int z = w.v_tok_on_z ? w.v_z0 + j * BLK : w.v_z0;
+      ptx::tma_load_3d(dst, tm_v, &B->v_full[s], 0, y, z);
+      if (!PV8 && D == 128)  // 16-bit V rows are 256 B: second 64-column box
+        ptx::tma_load_3d(dst + BLK * 128, tm_v, &B->v_full[s], 64, y, z);
+    }
+    __syncwarp();
   }
   // Teardown: the most recent load of every stage must have landed before
   // this CTA may exit (the earlier ones were consumed already).
@@ -227,79 +251,171 @@ template <int D, bool PV8, bool BF16V>
 __device__ void mma_issuer(const Work& w, Bars* B, uint32_t tmem, const uint8_t* sQ,
                            const uint8_t* sK, const uint8_t* sV, uint32_t* status) {
   using C = Cfg<D, PV8>;
-  constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, 128);
+  constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, SUB);
   constexpr uint32_t IDESC_PV =
       PV8 ? ptx::instr_desc(1, 0, 0, 0, 1, 128, D)
           : ptx::instr_desc(1, BF16V ? 1 : 0, BF16V ? 1 : 0, 0, 1, 128, D);
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
-  const int nkv = max(w.nkv[0], w.nkv[1]);
+  const int n0 = w.nsub0, n1 = w.nsub1;
+  const int nsub = max(n0, n1);
+  int k_ready = -1, v_ready = -1;  // highest 128-key stage known to be loaded
+  bool ok = true;
 
-  auto issue_qk = [&](int t, int j) {
-    const int s = j % C::NS;
+  auto need_k = [&](int j) -> bool {
+    if (k_ready >= j) return true;
+    if (!wait_bar(B, &B->k_full[j % C::NS], (j / C::NS) & 1, status, true)) return false;
+    k_ready = j;
+    ptx::tc_fence_after();
+    return true;
+  };
+  auto need_v = [&](int j) -> bool {
+    if (v_ready >= j) return true;
+    if (!wait_bar(B, &B->v_full[j % C::NS], (j / C::NS) & 1, status, true)) return false;
+    v_ready = j;
+    ptx::tc_fence_after();
+    return true;
+  };
+  auto issue_qk = [&](int t, int i) {
+    const int s = (i / 2) % C::NS;
     const uint32_t qa = ptx::smem_u32(sQ + t * C::QT);
-    const uint32_t kb = ptx::smem_u32(sK + s * C::QT);
+    const uint32_t kb = ptx::smem_u32(sK + s * C::QT + (i & 1) * C::K_SUB_BYTES);
+    const uint32_t dst = tmem + 128 * t + SUB * (i & 1);
+    if (ptx::elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < D / 32; ++kk) {
-      const uint64_t ad = ptx::smem_desc(qa + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
-      const uint64_t bd = ptx::smem_desc(kb + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
-      ptx::mma_i8_ss(tS[t], ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < D / 32; ++kk) {
+        const uint64_t ad = ptx::smem_desc(qa + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
+        const uint64_t bd = ptx::smem_desc(kb + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
+        ptx::mma_i8_ss(dst, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+      }
+      ptx::mma_commit(&B->s_full[t][i & 1]);
     }
-    ptx::mma_commit(&B->s_full[t]);
+    __syncwarp();
   };
-  auto issue_pv = [&](int t, int j) {
-    const int s = j % C::NS;
-    const uint32_t vb = ptx::smem_u32(sV + s * C::VT);
-    const uint32_t acc0 = PV8 ? 0u : (j > 0 ? 1u : 0u);
+  auto issue_pv = [&](int t, int i, bool last) {
+    const int s = (i / 2) % C::NS;
+    const uint32_t vb = ptx::smem_u32(sV + s * C::VT + (i & 1) * C::V_SUB_BYTES);
+    const uint32_t tO = tmem + 256 + D * t;
+    const uint32_t tP = tmem + 128 * t + SUB * (i & 1);
+    const uint32_t acc0 = PV8 ? 0u : (i > 0 ? 1u : 0u);
+    if (ptx::elect_one()) {
 #pragma unroll
-    for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-      const uint64_t bd = ptx::smem_desc(vb + kk * C::V_KSTEP_BYTES, C::V_LBO, C::V_SBO, C::V_SWZ);
-      const uint32_t acc = kk > 0 ? 1u : acc0;
-      if constexpr (PV8) ptx::mma_f8_ts(tO[t], tS[t] + 8 * kk, bd, IDESC_PV, acc);
-      else ptx::mma_f16_ts(tO[t], tS[t] + 8 * kk, bd, IDESC_PV, acc);
+      for (int kk = 0; kk < C::PV_STEPS; ++kk) {
+        const uint64_t bd = ptx::smem_desc(vb + kk * C::V_KSTEP_BYTES, C::V_LBO, C::V_SBO, C::V_SWZ);
+        const uint32_t acc = kk > 0 ? 1u : acc0;
+        if constexpr (PV8) ptx::mma_f8_ts(tO, tP + 8 * kk, bd, IDESC_PV, acc);
+        else ptx::mma_f16_ts(tO, tP + 8 * kk, bd, IDESC_PV, acc);
+      }
+      ptx::mma_commit(&B->o_full[t]);
+      if (last) ptx::mma_commit(&B->o_done[t]);
     }
-    ptx::mma_commit(&B->o_full[t]);
+    __syncwarp();
   };
 
-  bool ok = wait_bar(B, &B->q_full, 0, status, false);
-  int k_ready = -1;  // highest key tile whose K^ is known to be in shared memory
-  if (ok && nkv > 0) {
-    ok = wait_bar(B, &B->k_full[0], 0, status, false);
-    k_ready = 0;
-    if (ok) {
-      ptx::tc_fence_after();
-      for (int t = 0; t < 2; ++t)
-        if (w.nkv[t] > 0) issue_qk(t, 0);
-    }
+  ok = wait_bar(B, &B->q_full, 0, status, true);
+  if (ok) ptx::tc_fence_after();
+  // prologue: the first two sub-tiles of each query tile
+  for (int i = 0; ok && i < 2; ++i) {
+    if (i >= nsub) break;
+    if (!need_k(i / 2)) { ok = false; break; }
+    if (i < n0) issue_qk(0, i);
+    if (i < n1) issue_qk(1, i);
   }
-  for (int j = 0; ok && j < nkv; ++j) {
-    const int s = j % C::NS;
-    if (!wait_bar(B, &B->v_full[s], (j / C::NS) & 1, status, false)) break;
-    for (int t = 0; t < 2 && ok; ++t) {
-      if (j >= w.nkv[t]) continue;
-      if (!wait_bar(B, &B->p_full[t], j & 1, status, false)) { ok = false; break; }
+  for (int i = 0; ok && i < nsub; ++i) {
+    if (!need_v(i / 2)) break;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int nt = t == 0 ? n0 : n1;
+      if (i >= nt) continue;
+      // P (and, for 16-bit P.V, the rescaled O) of sub-tile i is ready
+      uint64_t* ready = PV8 ? &B->p_full[t][i & 1] : &B->o_ready[t][i & 1];
+      if (!wait_bar(B, ready, (i / 2) & 1, status, true)) { ok = false; break; }
       ptx::tc_fence_after();
-      issue_pv(t, j);
-      if (j + 1 < w.nkv[t]) {
-        if (k_ready < j + 1) {
-          const int s1 = (j + 1) % C::NS;
-          if (!wait_bar(B, &B->k_full[s1], ((j + 1) / C::NS) & 1, status, false)) { ok = false; break; }
-          k_ready = j + 1;
-        }
-        issue_qk(t, j + 1);
+      issue_pv(t, i, i == nt - 1);
+      if (i + 2 < nt) {
+        if (!need_k((i + 2) / 2)) { ok = false; break; }
+        issue_qk(t, i + 2);
       }
     }
-    ptx::mma_commit(&B->kv_empty[s]);
+    // stage i/2 is done once both of its sub-tiles went through P.V
+    if ((i & 1) || i == nsub - 1) {
+      if (ptx::elect_one()) ptx::mma_commit(&B->kv_empty[(i / 2) % C::NS]);
+      __syncwarp();
+    }
   }
   // Drain: every MMA issued above completes before TMEM is released.
-  ptx::mma_commit(&B->done);
+  if (ptx::elect_one()) ptx::mma_commit(&B->done);
+  __syncwarp();
   ptx::mbar_wait(&B->done, 0);
 }
 
 // --------------------------------------------------------------- softmax --
 
+// Exact int32 -> fp32 for |s| < 2^22: the integer added to the bit pattern of
+// 1.5 * 2^23 gives the float 1.5 * 2^23 + s, and subtracting 1.5 * 2^23 is
+// exact.  One integer add plus (half of) one packed float add, instead of a
+// conversion instruction; |S| <= 127^2 * 128 < 2^21 always holds here.
+__device__ __forceinline__ float2 s32x2_to_f32x2(uint32_t a, uint32_t b) {
+  const float2 f = make_float2(__uint_as_float(a + 0x4B400000u), __uint_as_float(b + 0x4B400000u));
+  return __fadd2_rn(f, make_float2(-12582912.0f, -12582912.0f));
+}
+
+__device__ __forceinline__ int imax3(int a, int b, int c) { return __vimax3_s32(a, b, c); }
+
+// Row maximum of NC columns of S (all valid).
+template <int NC>
+__device__ __forceinline__ int row_max(const uint32_t* v, int acc) {
+  int m0 = acc, m1 = INT_MIN, m2 = INT_MIN, m3 = INT_MIN;
+#pragma unroll
+  for (int i = 0; i < NC; i += 8) {
+    m0 = imax3(m0, (int)v[i], (int)v[i + 1]);
+    m1 = imax3(m1, (int)v[i + 2], (int)v[i + 3]);
+    m2 = imax3(m2, (int)v[i + 4], (int)v[i + 5]);
+    m3 = imax3(m3, (int)v[i + 6], (int)v[i + 7]);
+  }
+  return imax3(m0, imax3(m1, m2, m3), INT_MIN);
+}
+
+// Row maximum over the columns whose key index first_key + col is below `limit`.
+template <int NC>
+__device__ __forceinline__ int row_max_masked(const uint32_t* v, int acc, int first_key,
+                                              int limit) {
+#pragma unroll
+  for (int i = 0; i < NC; ++i)
+    if (first_key + i < limit) acc = max(acc, (int)v[i]);
+  return acc;
+}
+
+// p for NC columns: p = 2^fma(S, c, -m) (masked columns give 0); returns the
+// sum of p.  Results are written to p[].
+template <bool MASKED, int NC>
+__device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m, int first_key,
+                                         int limit, float* p) {
+  const float2 c2 = make_float2(c, c), n2 = make_float2(neg_m, neg_m);
+  float2 s2a = make_float2(0.0f, 0.0f), s2b = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int i = 0; i < NC; i += 2) {
+    const float2 a = __ffma2_rn(s32x2_to_f32x2(v[i], v[i + 1]), c2, n2);
+    float p0 = ptx::ex2(a.x), p1 = ptx::ex2(a.y);
+    if (MASKED) {
+      if (first_key + i >= limit) p0 = 0.0f;
+      if (first_key + i + 1 >= limit) p1 = 0.0f;
+    }
+    p[i] = p0;
+    p[i + 1] = p1;
+    if ((i & 2) == 0) s2a = __fadd2_rn(s2a, make_float2(p0, p1));
+    else s2b = __fadd2_rn(s2b, make_float2(p0, p1));
+  }
+  const float2 s = __fadd2_rn(s2a, s2b);
+  return s.x + s.y;
+}
+
+// Shared-memory exchange of alpha from the softmax to the correction warps.
+struct AlphaBuf {
+  float a[2][2][128];  // [tile][S buffer][row]
+};
+
 template <int D, bool PV8, bool BF16V>
-__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t tmem, int t) {
+__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, AlphaBuf* AB,
+                           uint32_t tmem, int t) {
   using In = In16<BF16V>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
@@ -307,146 +423,118 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
   const int qt = 2 * w.pair + t;
   const int row = qt * BLK + r;                   // query index in the sequence
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-  const uint32_t tS = tmem + 128 * t + lane_off;
+  const uint32_t tS0 = tmem + 128 * t + lane_off;
   const uint32_t tO = tmem + 256 + D * t + lane_off;
-  const int nkv = w.nkv[t];
-  if (nkv == 0) return;
+  const int nsub = t == 0 ? w.nsub0 : w.nsub1;
+  if (nsub == 0) return;
 
   const float qd = __ldg(p.q_scale + w.qs_idx0 + t);
-  float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f;
+  float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f, c = 0.0f;
   float o32[PV8 ? D : 1];
   if constexpr (PV8) {
 #pragma unroll
     for (int i = 0; i < D; ++i) o32[i] = 0.0f;
   }
+  const int limit = p.causal ? min(w.n, row + 1) : w.n;  // keys >= limit are masked
 
-  for (int j = 0; j < nkv; ++j) {
-    if (!wait_bar(B, &B->s_full[t], j & 1, p.status, true)) return;
+  for (int i = 0; i < nsub; ++i) {
+    const int b = i & 1;
+    const uint32_t tS = tS0 + SUB * b;
+    if ((i & 1) == 0) {  // a new 128-key quantisation block: its delta
+      const float kd = __ldg(p.k_scale + w.ks_idx0 + i / 2);
+      c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
+    }
+    if (!wait_bar(B, &B->s_full[t][b], (i / 2) & 1, p.status, true)) return;
     ptx::tc_fence_after();
-    const float kd = __ldg(p.k_scale + w.ks_idx0 + j);
-    const float c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
-    const int key0 = j * BLK;
-    // keys >= limit are masked for this row
-    const int limit = p.causal ? min(w.n, row + 1) : w.n;
-    const bool full_tile = (key0 + BLK <= w.n) && (!p.causal || key0 + BLK - 1 <= qt * BLK);
+    const int key0 = i * SUB;
+    const bool full_tile = (key0 + SUB <= w.n) && (!p.causal || key0 + SUB - 1 <= qt * BLK);
     float alpha, rowsum = 0.0f, m_new;
 
     if constexpr (!PV8) {
-      uint32_t sv[128];
+      uint32_t sv[SUB];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]);
-        ptx::tmem_ld32(tS + 32 * cc, chunk);
-      }
+      for (int cc = 0; cc < SUB / 32; ++cc)
+        ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
       ptx::tmem_wait_ld();
-      int smax = INT_MIN;
-      if (full_tile) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) smax = max(smax, (int)sv[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (key0 + i < limit) smax = max(smax, (int)sv[i]);
-      }
-      m_new = fmaxf(m, __fmul_rn((float)smax, c));
+      const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
+                                 : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
+      // a sub-tile with no unmasked key for this row leaves the maximum unchanged
+      const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+      m_new = fmaxf(m, m_blk);
       alpha = ptx::ex2(__fsub_rn(m, m_new));
-      const float neg = -m_new;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < SUB / 32; ++cc) {
+        float pv[32];
+        rowsum += full_tile ? row_exp<false, 32>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv)
+                            : row_exp<true, 32>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv);
         uint32_t packed[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = 32 * cc + 2 * i;
-          float p0 = ptx::ex2(__fmaf_rn((float)(int)sv[c0], c, neg));
-          float p1 = ptx::ex2(__fmaf_rn((float)(int)sv[c0 + 1], c, neg));
-          if (!full_tile) {
-            if (key0 + c0 >= limit) p0 = 0.0f;
-            if (key0 + c0 + 1 >= limit) p1 = 0.0f;
-          }
-          rowsum += p0;
-          rowsum += p1;
-          packed[i] = In::pack(p0, p1);
-        }
+        for (int k = 0; k < 16; ++k) packed[k] = In::pack(pv[2 * k], pv[2 * k + 1]);
         ptx::tmem_st16(tS + 16 * cc, packed);
       }
+      AB->a[t][b][r] = alpha;  // for the correction warps
     } else {
-      // pass 1: row maximum
+      // pass 1: row maximum (S re-read per chunk keeps registers for O32)
       int smax = INT_MIN;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32];
-        ptx::tmem_ld32(tS + 32 * cc, sv);
+      for (int cc = 0; cc < SUB / 16; ++cc) {
+        uint32_t sv[16];
+        ptx::tmem_ld16(tS + 16 * cc, sv);
         ptx::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (full_tile || key0 + 32 * cc + i < limit) smax = max(smax, (int)sv[i]);
+        smax = full_tile ? row_max<16>(sv, smax) : row_max_masked<16>(sv, smax, key0 + 16 * cc, limit);
       }
-      m_new = fmaxf(m, __fmul_rn((float)smax, c));
+      const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+      m_new = fmaxf(m, m_blk);
       alpha = ptx::ex2(__fsub_rn(m, m_new));
-      const float neg = -m_new;
       // pass 2: P^ = e4m3(448 p), four per TMEM column, written over S
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32];
-        ptx::tmem_ld32(tS + 32 * cc, sv);
+      for (int cc = 0; cc < SUB / 16; ++cc) {
+        uint32_t sv[16];
+        ptx::tmem_ld16(tS + 16 * cc, sv);
         ptx::tmem_wait_ld();
-        uint32_t packed[8];
+        float pv[16];
+        rowsum += full_tile ? row_exp<false, 16>(sv, c, -m_new, key0 + 16 * cc, limit, pv)
+                            : row_exp<true, 16>(sv, c, -m_new, key0 + 16 * cc, limit, pv);
+        uint32_t packed[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float pp[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 32 * cc + 4 * i + e;
-            float pe = ptx::ex2(__fmaf_rn((float)(int)sv[4 * i + e], c, neg));
-            if (!full_tile && key0 + col >= limit) pe = 0.0f;
-            rowsum += pe;
-            pp[e] = __fmul_rn(pe, 448.0f);
-          }
-          packed[i] = pack_e4m3x4(pp[0], pp[1], pp[2], pp[3]);
+        for (int k = 0; k < 4; ++k) {
+          const float2 a = __fmul2_rn(make_float2(pv[4 * k], pv[4 * k + 1]), make_float2(448.0f, 448.0f));
+          const float2 bb = __fmul2_rn(make_float2(pv[4 * k + 2], pv[4 * k + 3]), make_float2(448.0f, 448.0f));
+          packed[k] = pack_e4m3x4(a.x, a.y, bb.x, bb.y);
         }
-        ptx::tmem_st8(tS + 8 * cc, packed);
+        ptx::tmem_st4(tS + 4 * cc, packed);
+      }
+      if (i > 0) {
+        // two-level accumulation: O32 <- alpha_{i-1} O32 + Part_{i-1}
+        if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
+        ptx::tc_fence_after();
+        const float2 a2 = make_float2(alpha_prev, alpha_prev);
+#pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t pv[16];
+          ptx::tmem_ld16(tO + 16 * cc, pv);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 16; k += 2) {
+            const float2 x = __ffma2_rn(a2, make_float2(o32[16 * cc + k], o32[16 * cc + k + 1]),
+                                        make_float2(__uint_as_float(pv[k]), __uint_as_float(pv[k + 1])));
+            o32[16 * cc + k] = x.x;
+            o32[16 * cc + k + 1] = x.y;
+          }
+        }
       }
     }
     l = __fadd_rn(__fmul_rn(alpha, l), rowsum);
-
-    if (j > 0) {
-      if (!wait_bar(B, &B->o_full[t], (j - 1) & 1, p.status, true)) return;
-      ptx::tc_fence_after();
-      if constexpr (!PV8) {
-        // O <- alpha * O before this block's P.V accumulates into it
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ov[32];
-            ptx::tmem_ld32(tO + 32 * cc, ov);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__fmul_rn(alpha, __uint_as_float(ov[i])));
-            ptx::tmem_st32(tO + 32 * cc, ov);
-          }
-        }
-      } else {
-        // two-level accumulation: O32 <- alpha_{j-1} O32 + Part_{j-1}
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t pv[32];
-          ptx::tmem_ld32(tO + 32 * cc, pv);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            o32[32 * cc + i] = __fmaf_rn(alpha_prev, o32[32 * cc + i], __uint_as_float(pv[i]));
-        }
-      }
-    }
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
-    ptx::mbar_arrive(&B->p_full[t]);
+    ptx::mbar_arrive(&B->p_full[t][b]);
     m = m_new;
     alpha_prev = alpha;
   }
 
   // ------------------------------------------------------------ epilogue --
-  if (!wait_bar(B, &B->o_full[t], (nkv - 1) & 1, p.status, true)) return;
+  // (o_full may lag by two phases here in 16-bit mode; o_done is unambiguous)
+  if (!wait_bar(B, &B->o_done[t], 0, p.status, true)) return;
   ptx::tc_fence_after();
   const bool store = row < w.n;
   const long long orow = (w.out_row0 + (long long)row * w.out_stride) * D;
@@ -458,33 +546,81 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
     ptx::tmem_wait_ld();
     float o[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int k = 0; k < 32; ++k) {
       if constexpr (PV8) {
-        const float acc = __fmaf_rn(alpha_prev, o32[32 * cc + i], __uint_as_float(ov[i]));
-        const float vf = __fdiv_rn(__ldg(p.v_scale + w.vs_idx * D + 32 * cc + i), 448.0f);
-        o[i] = __fmul_rn(__fmul_rn(acc, vf), inv_l);
+        const float acc = __fmaf_rn(alpha_prev, o32[32 * cc + k], __uint_as_float(ov[k]));
+        const float vf = __fdiv_rn(__ldg(p.v_scale + w.vs_idx * D + 32 * cc + k), 448.0f);
+        o[k] = __fmul_rn(__fmul_rn(acc, vf), inv_l);
       } else {
-        o[i] = __fmul_rn(__uint_as_float(ov[i]), inv_l);
+        o[k] = __fmul_rn(__uint_as_float(ov[k]), inv_l);
       }
     }
     if (!store) continue;
     if (p.out_dt == SAGE_F32) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + 32 * cc);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      for (int k = 0; k < 8; ++k) dst[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
     } else {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + 32 * cc);
       const bool ob = p.out_dt == SAGE_BF16;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int k = 0; k < 4; ++k) {
         uint32_t u[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = o[8 * i + 2 * e], b = o[8 * i + 2 * e + 1];
-          u[e] = ob ? In16<true>::pack(a, b) : In16<false>::pack(a, b);
+          const float a = o[8 * k + 2 * e], bb = o[8 * k + 2 * e + 1];
+          u[e] = ob ? In16<true>::pack(a, bb) : In16<false>::pack(a, bb);
         }
-        dst[i] = make_uint4(u[0], u[1], u[2], u[3]);
+        dst[k] = make_uint4(u[0], u[1], u[2], u[3]);
       }
+    }
+  }
+}
+
+// ------------------------------------------------------------ correction --
+
+// 16-bit P.V: before P.V of sub-tile i accumulates into O_t, O_t must be
+// scaled by alpha_i (exp2 of the old minus the new row maximum).  The
+// correction warpgroup does this for both query tiles, in sub-tile order,
+// skipping the TMEM round trip when alpha is 1 for all 32 rows of a warp.
+template <int D>
+__device__ void correction_wg(const AttnParams& p, const Work& w, Bars* B, const AlphaBuf* AB,
+                              uint32_t tmem) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  const int n0 = w.nsub0, n1 = w.nsub1;
+  const int nsub = max(n0, n1);
+  for (int i = 0; i < nsub; ++i) {
+    const int b = i & 1;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (i >= (t == 0 ? n0 : n1)) continue;
+      if (!wait_bar(B, &B->p_full[t][b], (i / 2) & 1, p.status, true)) return;
+      const float alpha = AB->a[t][b][r];
+      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
+        ptx::tc_fence_after();
+        const uint32_t tO = tmem + 256 + D * t + lane_off;
+        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tO + 32 * cc, ov);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float2 x = __fmul2_rn(a2, make_float2(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1])));
+            ov[k] = __float_as_uint(x.x);
+            ov[k + 1] = __float_as_uint(x.y);
+          }
+          ptx::tmem_st32(tO + 32 * cc, ov);
+        }
+        ptx::tmem_wait_st();
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&B->o_ready[t][b]);
     }
   }
 }
@@ -492,7 +628,7 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
 // ---------------------------------------------------------------- kernel --
 
 template <int D, bool PV8, bool BF16V>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Cfg<D, PV8>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = Cfg<D, PV8>;
@@ -502,18 +638,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sK = sQ + 2 * C::QT;
   uint8_t* sV = sK + C::NS * C::QT;
   Bars* B = reinterpret_cast<Bars*>(sV + C::NS * C::VT);
+  AlphaBuf* AB = reinterpret_cast<AlphaBuf*>(reinterpret_cast<uint8_t*>(B) + 1024);
+  static_assert(sizeof(Bars) <= 1024 && sizeof(AlphaBuf) + 1024 <= C::AUX, "aux layout");
 
   const Work w = decode_work(p);
   if (!w.valid) return;
   const int warp = threadIdx.x / 32;
+  const int wg = warp / 4;
+  const int warp_tma = 4 * C::WG_CTRL, warp_mma = 4 * C::WG_CTRL + 1;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&B->q_full, 1);
     ptx::mbar_init(&B->done, 1);
     for (int t = 0; t < 2; ++t) {
-      ptx::mbar_init(&B->s_full[t], 1);
-      ptx::mbar_init(&B->p_full[t], 128);
       ptx::mbar_init(&B->o_full[t], 1);
+      ptx::mbar_init(&B->o_done[t], 1);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(&B->s_full[t][b], 1);
+        ptx::mbar_init(&B->p_full[t][b], 128);
+        ptx::mbar_init(&B->o_ready[t][b], 128);
+      }
     }
     for (int s = 0; s < C::NS; ++s) {
       ptx::mbar_init(&B->k_full[s], 1);
@@ -523,7 +667,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     B->abort = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == WARP_MMA) {
+  if (warp == warp_mma) {
     ptx::tmem_alloc(&B->tmem_base, 512);
     ptx::tmem_relinquish();
   }
@@ -532,18 +676,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = B->tmem_base;
 
-  if (warp == WARP_TMA) {
-    if ((threadIdx.x & 31) == 0) producer<D, PV8>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, p.status);
-  } else if (warp == WARP_MMA) {
-    if ((threadIdx.x & 31) == 0) mma_issuer<D, PV8, BF16V>(w, B, tmem, sQ, sK, sV, p.status);
+  if (wg == C::WG_CTRL) {
+    ptx::setmaxnreg_dec<C::REG_CTRL>();
+    if (warp == warp_tma) {
+      producer<D, PV8>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, p.status);
+    } else if (warp == warp_mma) {
+      mma_issuer<D, PV8, BF16V>(w, B, tmem, sQ, sK, sV, p.status);
+    }
+  } else if (!PV8 && wg == C::WG_CORR) {
+    ptx::setmaxnreg_dec<C::REG_CORR>();
+    correction_wg<D>(p, w, B, AB, tmem);
   } else {
-    softmax_wg<D, PV8, BF16V>(p, w, B, tmem, warp / 4);
+    ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
+    softmax_wg<D, PV8, BF16V>(p, w, B, AB, tmem, wg);
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == WARP_MMA) ptx::tmem_dealloc(tmem, 512);
+  if (warp == warp_mma) ptx::tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------ QK^T tile diagnostic --
@@ -692,7 +843,7 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
   auto kern = attn_fwd_kernel<D, PV8, BF16V>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<L.grid, NUM_THREADS, C::SMEM, st>>>(tq, tk, tv, L.p);
+  kern<<<L.grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, L.p);
   return cudaGetLastError();
 }
 
