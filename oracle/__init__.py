@@ -33,6 +33,10 @@ ORACLE_ERR_RANGE = 1
 # reading taken (the quantisation block stays 128 tokens).
 KV_TILE = 64
 
+# How far (base 2) a tile's maximum must exceed the maximum in use before p is
+# re-referenced to it; see sage_oracle.c.  16-bit P.V: 8; FP8 P.V: 0.
+TAU = {"fp16": 8.0, "fp8": 0.0}
+
 
 def build(force: bool = False) -> str:
     """Compile sage_oracle.c into liboracle.so (gcc, no fast-math, no FP contraction)."""
@@ -63,8 +67,8 @@ def lib():
         L.oracle_qk_int.argtypes = [P, P, i32, i64, i32, i64, i32, P]; L.oracle_qk_int.restype = None
         L.oracle_attn_ref_rows.argtypes = [P, P, P, i64, i32, i64, i64, i64, f64, i32, P, i64, P]
         L.oracle_attn_ref_rows.restype = None
-        L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, i32, f32, i32,
-                                            i32, i32, P, i64, P]
+        L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, i32, f32, f32,
+                                            i32, i32, i32, P, i64, P]
         L.oracle_attn_emul_rows.restype = None
         _lib = L
     return _lib
@@ -174,7 +178,7 @@ def attn_ref_rows(q, k, v, sm_scale: float, causal: bool, rows) -> np.ndarray:
 
 def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, causal: bool,
                    pv_mode: str, rows, v=None, p16: str = "fp16", vc=None, vdelta=None,
-                   blk: int = 128, kv: int = KV_TILE) -> np.ndarray:
+                   blk: int = 128, kv: int = KV_TILE, tau=None) -> np.ndarray:
     """The quantised method's output rows (fp32) for one head; see sage_oracle.c.
     blk: quantisation block (tokens); kv: key tile of the online softmax."""
     if blk % kv:
@@ -192,6 +196,7 @@ def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, caus
         vdelta = _f32(vdelta)
         vc_p, vd_p, v_p, ldv, mode = _p(vc), _p(vdelta), None, D, 1
     lib().oracle_attn_emul_rows(_p(qc), _p(qdelta), _p(kc), _p(kdelta), v_p, ldv, vc_p, vd_p, n,
-                                D, blk, kv, float(kappa(sm_scale)), int(causal), mode,
+                                D, blk, kv, float(kappa(sm_scale)),
+                                float(TAU[pv_mode] if tau is None else tau), int(causal), mode,
                                 1 if p16 == "bf16" else 0, _p(rows), len(rows), _p(out))
     return out

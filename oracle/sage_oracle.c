@@ -320,6 +320,12 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  * the FP8 two-level flush -- the pages give FlashAttention's tiling without a
  * tile size ("Attention机制优化", section 3.1); the reading taken is 64 keys.
  * kappa = fp32(sm_scale * log2(e)): the softmax runs in base 2.
+ * tau >= 0: the maximum m used to compute p is moved only when the tile's
+ * maximum exceeds it by more than tau (base-2 units); in real arithmetic the
+ * rescale factors cancel in O / l, so any tau gives the same attention, and
+ * tau = 0 is the plain running maximum.  Reading taken: tau = 8 for 16-bit
+ * P.V (p then stays below 2^8, exactly representable in range of fp16/bf16),
+ * tau = 0 for FP8 P.V (P^ = e4m3(448 p) needs p <= 1).
  *
  * For each row i (query block I = i / blk) and key tile T = 0, 1, ... in
  * ascending order (tiles starting at or before i when causal), the tile's keys
@@ -327,7 +333,8 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *
  *   S_ij   = sum_d q^_id k^_jd                       exact int32
  *   c_IJ   = fp32( fp32(deltaQ_I * deltaK_J) * kappa )   dequant x softmax scale
- *   m_new  = max(m, fp32(max_j S_ij * c_IJ))          the block's scaled max
+ *   mb     = fp32(max_j S_ij * c_IJ)                   the tile's scaled max
+ *   m_new  = mb if mb > m + tau, else m
  *   arg_ij = fmaf(S_ij, c_IJ, -m_new)                 dequant, scale and max
  *                                                     subtraction in one fused
  *                                                     multiply-add (reading of
@@ -361,8 +368,8 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
 void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* kc,
                            const float* kdelta, const float* v, long ldv, const uint8_t* vc,
                            const float* vdelta, long n, int D, int blk, int kv, float kappa,
-                           int causal, int pv_mode, int p16_format, const long* rows, long nrows,
-                           float* out)
+                           float tau, int causal, int pv_mode, int p16_format, const long* rows,
+                           long nrows, float* out)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (long r = 0; r < nrows; ++r) {
@@ -391,7 +398,7 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
             }
             float c = (qdelta[I] * kdelta[J]) * kappa;
             float mblk = (float)smax * c;
-            float m_new = m > mblk ? m : mblk;
+            float m_new = mblk > m + tau ? mblk : m;
             float alpha = (float)exp2((double)(m - m_new));
             double psum = 0.0;
             for (int jj = 0; jj < nj; ++jj) {

@@ -4,8 +4,9 @@
 // that head's keys and values through shared memory in 128-key stages; the
 // online softmax works on 64-key sub-tiles.
 //
-//   control warpgroup (warp 0 of it: TMA producer; warp 1: TMEM owner and
-//                single-thread MMA issuer):
+//   control warpgroup (warp 0 of it: TMA producer; warps 1 and 2: MMA
+//                issue for query tile 0 / 1, one elected lane each; warp 1
+//                also owns TMEM):
 //                  S_t[b]  = Q^_t K^_i^T     tcgen05.mma kind::i8 -> int32 TMEM
 //                  O_t    += P_t[b] V_i      kind::f16 (16-bit P.V), or
 //                  Part_t  = P^_t[b] V^_i    kind::f8f6f4 (FP8 P.V),
@@ -13,15 +14,15 @@
 //   softmax warpgroups 0 and 1 (one per query tile, one thread per row):
 //                read S from TMEM, dequantise with deltaQ*deltaK*sm_scale*log2 e,
 //                mask, online softmax in base 2, write P (fp16/bf16 or e4m3)
-//                back over S; FP8: fold the previous sub-tile's partial into an
-//                fp32 register accumulator (two-level accumulation).
-//   correction warpgroup (16-bit P.V only): O_t <- alpha * O_t in TMEM when a
-//                row maximum grew, between two P.V accumulations, off the
-//                softmax warps' path.
+//                back over S; 16-bit P.V: rescale O in TMEM when the maximum
+//                in use moves; FP8: fold the previous sub-tile's partial into
+//                an fp32 register accumulator (two-level accumulation).
 //
 // Each query tile owns two 64-column S buffers, so QK^T of sub-tile i+1 runs
 // on the tensor core while the softmax works on sub-tile i, and the two query
-// tiles keep both softmax warpgroups busy.
+// tiles keep both softmax warpgroups busy.  The maximum used for P moves only
+// when a row's tile maximum exceeds it by more than TAU (8 for 16-bit P.V,
+// so O rescales are rare; 0 for FP8 P.V, whose rescale is free in the flush).
 //
 // TMEM columns (512): S_0[0] [0,64) S_0[1] [64,128) S_1[0] [128,192)
 // S_1[1] [192,256) O_0 [256,256+D) O_1 [256+D,256+2D).
@@ -48,23 +49,20 @@ constexpr int SUB = 64;  // keys per softmax sub-tile
 
 template <int D, bool PV8>
 struct Cfg {
-  // warpgroups: 2 softmax, [1 correction (16-bit P.V)], 1 control
-  static constexpr int WGS = PV8 ? 3 : 4;
+  // warpgroups: 2 softmax, 1 control
+  static constexpr int WGS = 3;
   static constexpr int THREADS = WGS * 128;
-  static constexpr int WG_CTRL = WGS - 1;
-  static constexpr int WG_CORR = 2;
-  // register split, summing to the launch allocation (65536 regs for 512
-  // threads at 128 each; 64512 for 384 threads at 168 each)
-  static constexpr int REG_SOFTMAX = PV8 ? 224 : 192;
-  static constexpr int REG_CORR = 80;
-  static constexpr int REG_CTRL = PV8 ? 56 : 48;
-  static_assert(PV8 ? (256 * 224 + 128 * 56 <= 384 * 168)
-                    : (256 * 192 + 128 * 80 + 128 * 48 <= 65536),
+  static constexpr int WG_CTRL = 2;
+  // register split, summing to the launch allocation (384 threads at 168)
+  static constexpr int REG_SOFTMAX = 224;
+  static constexpr int REG_CTRL = 56;
+  static_assert(256 * REG_SOFTMAX + 128 * REG_CTRL <= 384 * 168,
                 "register split exceeds the launch allocation");
+  static constexpr float TAU = PV8 ? 0.0f : 8.0f;  // threshold for moving the maximum
 
   static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
   static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
-  static constexpr int AUX = 4096;                      // barriers + alpha exchange
+  static constexpr int AUX = 1024;                      // barriers
   static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - AUX;
   static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;    // pipeline stages (128 keys each)
@@ -88,10 +86,9 @@ struct Cfg {
 };
 
 struct Bars {
-  uint64_t q_full, done;
+  uint64_t q_full, done[2];
   uint64_t s_full[2][2];   // [tile][S buffer]: QK^T of a sub-tile landed
-  uint64_t p_full[2][2];   // P of a sub-tile written (128 softmax threads)
-  uint64_t o_ready[2][2];  // 16-bit P.V: O rescaled for the sub-tile (128 correction threads)
+  uint64_t p_full[2][2];   // P of a sub-tile written, O rescaled (128 softmax threads)
   uint64_t o_full[2];      // P.V of a sub-tile completed
   uint64_t o_done[2];      // the last P.V of a query tile completed (one phase)
   uint64_t k_full[8], v_full[8], kv_empty[8];
@@ -247,104 +244,113 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
 
 // ------------------------------------------------------------ MMA issuer --
 
+// One warp per query tile issues that tile's MMAs (the whole warp runs the
+// loop; one elected lane issues).  Per 64-key sub-tile i:
+//   wait P_t(i) -> O_t (+)= P_t(i) V_i  ->  S_t(i+2) = Q^_t K^_{i+2}^T
+// Issue order per thread is execution order, so S_t(i+2) never overwrites
+// P_t(i) before P.V has read it.  A 128-key stage is released to the producer
+// when both tiles' warps have committed it (kv_empty counts two arrivals).
 template <int D, bool PV8, bool BF16V>
 __device__ void mma_issuer(const Work& w, Bars* B, uint32_t tmem, const uint8_t* sQ,
-                           const uint8_t* sK, const uint8_t* sV, uint32_t* status) {
+                           const uint8_t* sK, const uint8_t* sV, int t, uint32_t* status) {
   using C = Cfg<D, PV8>;
   constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, SUB);
   constexpr uint32_t IDESC_PV =
       PV8 ? ptx::instr_desc(1, 0, 0, 0, 1, 128, D)
           : ptx::instr_desc(1, BF16V ? 1 : 0, BF16V ? 1 : 0, 0, 1, 128, D);
-  const int n0 = w.nsub0, n1 = w.nsub1;
-  const int nsub = max(n0, n1);
-  int k_ready = -1, v_ready = -1;  // highest 128-key stage known to be loaded
-  bool ok = true;
+  const int nt = t == 0 ? w.nsub0 : w.nsub1;
+  const int nst = w.nkv;                      // stages the producer loads
+  const uint32_t qa = ptx::smem_u32(sQ + t * C::QT);
+  const uint32_t tO = tmem + 256 + D * t;
+  int k_ready = -1, v_ready = -1;             // highest stage known to be loaded
+  int released = 0;                           // stages this warp has committed
 
   auto need_k = [&](int j) -> bool {
     if (k_ready >= j) return true;
     if (!wait_bar(B, &B->k_full[j % C::NS], (j / C::NS) & 1, status, true)) return false;
     k_ready = j;
-    ptx::tc_fence_after();
     return true;
   };
   auto need_v = [&](int j) -> bool {
     if (v_ready >= j) return true;
     if (!wait_bar(B, &B->v_full[j % C::NS], (j / C::NS) & 1, status, true)) return false;
     v_ready = j;
-    ptx::tc_fence_after();
     return true;
   };
-  auto issue_qk = [&](int t, int i) {
-    const int s = (i / 2) % C::NS;
-    const uint32_t qa = ptx::smem_u32(sQ + t * C::QT);
-    const uint32_t kb = ptx::smem_u32(sK + s * C::QT + (i & 1) * C::K_SUB_BYTES);
+  auto issue_qk = [&](int i) {
+    const uint32_t kb = ptx::smem_u32(sK + ((i / 2) % C::NS) * C::QT + (i & 1) * C::K_SUB_BYTES);
     const uint32_t dst = tmem + 128 * t + SUB * (i & 1);
     if (ptx::elect_one()) {
+      const uint64_t a0 = ptx::smem_desc(qa, 16, C::QK_SBO, C::QK_SWZ);
+      const uint64_t b0 = ptx::smem_desc(kb, 16, C::QK_SBO, C::QK_SWZ);
 #pragma unroll
-      for (int kk = 0; kk < D / 32; ++kk) {
-        const uint64_t ad = ptx::smem_desc(qa + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
-        const uint64_t bd = ptx::smem_desc(kb + 32 * kk, 16, C::QK_SBO, C::QK_SWZ);
-        ptx::mma_i8_ss(dst, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-      }
+      for (int kk = 0; kk < D / 32; ++kk)  // +32 bytes along K per step: +2 in the address field
+        ptx::mma_i8_ss(dst, a0 + 2 * kk, b0 + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
       ptx::mma_commit(&B->s_full[t][i & 1]);
     }
     __syncwarp();
   };
-  auto issue_pv = [&](int t, int i, bool last) {
-    const int s = (i / 2) % C::NS;
-    const uint32_t vb = ptx::smem_u32(sV + s * C::VT + (i & 1) * C::V_SUB_BYTES);
-    const uint32_t tO = tmem + 256 + D * t;
+  auto issue_pv = [&](int i) {
+    const uint32_t vb = ptx::smem_u32(sV + ((i / 2) % C::NS) * C::VT + (i & 1) * C::V_SUB_BYTES);
     const uint32_t tP = tmem + 128 * t + SUB * (i & 1);
     const uint32_t acc0 = PV8 ? 0u : (i > 0 ? 1u : 0u);
     if (ptx::elect_one()) {
+      const uint64_t b0 = ptx::smem_desc(vb, C::V_LBO, C::V_SBO, C::V_SWZ);
 #pragma unroll
       for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-        const uint64_t bd = ptx::smem_desc(vb + kk * C::V_KSTEP_BYTES, C::V_LBO, C::V_SBO, C::V_SWZ);
+        const uint64_t bd = b0 + (uint64_t)((kk * C::V_KSTEP_BYTES) >> 4);
         const uint32_t acc = kk > 0 ? 1u : acc0;
         if constexpr (PV8) ptx::mma_f8_ts(tO, tP + 8 * kk, bd, IDESC_PV, acc);
         else ptx::mma_f16_ts(tO, tP + 8 * kk, bd, IDESC_PV, acc);
       }
       ptx::mma_commit(&B->o_full[t]);
-      if (last) ptx::mma_commit(&B->o_done[t]);
+      if (i == nt - 1) ptx::mma_commit(&B->o_done[t]);
     }
     __syncwarp();
   };
+  // Commit stage `released` (this warp is done with it).  For a stage this
+  // tile never reads, first wait until the stage's previous use was released,
+  // so the arrival cannot count toward that earlier phase.
+  auto release = [&](bool used) -> bool {
+    const int j = released;
+    if (!used && j >= C::NS &&
+        !wait_bar(B, &B->kv_empty[j % C::NS], ((j / C::NS) - 1) & 1, status, true))
+      return false;
+    if (ptx::elect_one()) ptx::mma_commit(&B->kv_empty[j % C::NS]);
+    __syncwarp();
+    ++released;
+    return true;
+  };
 
-  ok = wait_bar(B, &B->q_full, 0, status, true);
+  bool ok = wait_bar(B, &B->q_full, 0, status, true);
   if (ok) ptx::tc_fence_after();
-  // prologue: the first two sub-tiles of each query tile
-  for (int i = 0; ok && i < 2; ++i) {
-    if (i >= nsub) break;
+  for (int i = 0; ok && i < 2 && i < nt; ++i) {
     if (!need_k(i / 2)) { ok = false; break; }
-    if (i < n0) issue_qk(0, i);
-    if (i < n1) issue_qk(1, i);
+    ptx::tc_fence_after();
+    issue_qk(i);
   }
-  for (int i = 0; ok && i < nsub; ++i) {
+  for (int i = 0; ok && i < nt; ++i) {
     if (!need_v(i / 2)) break;
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int nt = t == 0 ? n0 : n1;
-      if (i >= nt) continue;
-      // P (and, for 16-bit P.V, the rescaled O) of sub-tile i is ready
-      uint64_t* ready = PV8 ? &B->p_full[t][i & 1] : &B->o_ready[t][i & 1];
-      if (!wait_bar(B, ready, (i / 2) & 1, status, true)) { ok = false; break; }
+    if (!wait_bar(B, &B->p_full[t][i & 1], (i / 2) & 1, status, true)) break;
+    ptx::tc_fence_after();
+    issue_pv(i);
+    if (i + 2 < nt) {
+      if (!need_k((i + 2) / 2)) break;
       ptx::tc_fence_after();
-      issue_pv(t, i, i == nt - 1);
-      if (i + 2 < nt) {
-        if (!need_k((i + 2) / 2)) { ok = false; break; }
-        issue_qk(t, i + 2);
-      }
+      issue_qk(i + 2);
     }
-    // stage i/2 is done once both of its sub-tiles went through P.V
-    if ((i & 1) || i == nsub - 1) {
-      if (ptx::elect_one()) ptx::mma_commit(&B->kv_empty[(i / 2) % C::NS]);
-      __syncwarp();
+    if ((i & 1) || i == nt - 1) {
+      if (!release(true)) break;
     }
   }
-  // Drain: every MMA issued above completes before TMEM is released.
-  if (ptx::elect_one()) ptx::mma_commit(&B->done);
+  // stages loaded for the other tile only
+  while (ok && released < nst && released >= (nt + 1) / 2) {
+    if (!release(false)) break;
+  }
+  // Drain: every MMA this warp issued completes before TMEM is released.
+  if (ptx::elect_one()) ptx::mma_commit(&B->done[t]);
   __syncwarp();
-  ptx::mbar_wait(&B->done, 0);
+  ptx::mbar_wait(&B->done[t], 0);
 }
 
 // --------------------------------------------------------------- softmax --
@@ -408,14 +414,9 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
   return s.x + s.y;
 }
 
-// Shared-memory exchange of alpha from the softmax to the correction warps.
-struct AlphaBuf {
-  float a[2][2][128];  // [tile][S buffer][row]
-};
-
 template <int D, bool PV8, bool BF16V>
-__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, AlphaBuf* AB,
-                           uint32_t tmem, int t) {
+__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t tmem, int t) {
+  using C = Cfg<D, PV8>;
   using In = In16<BF16V>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
@@ -460,8 +461,8 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, AlphaBuf
                                  : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
       // a sub-tile with no unmasked key for this row leaves the maximum unchanged
       const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
-      m_new = fmaxf(m, m_blk);
-      alpha = ptx::ex2(__fsub_rn(m, m_new));
+      m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
+      alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
 #pragma unroll
       for (int cc = 0; cc < SUB / 32; ++cc) {
         float pv[32];
@@ -472,7 +473,26 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, AlphaBuf
         for (int k = 0; k < 16; ++k) packed[k] = In::pack(pv[2 * k], pv[2 * k + 1]);
         ptx::tmem_st16(tS + 16 * cc, packed);
       }
-      AB->a[t][b][r] = alpha;  // for the correction warps
+      // O <- alpha * O before this sub-tile's P.V accumulates into it (rare:
+      // only when some row's maximum moved by more than TAU)
+      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
+        ptx::tc_fence_after();
+        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tO + 32 * cc, ov);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float2 x = __fmul2_rn(a2, make_float2(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1])));
+            ov[k] = __float_as_uint(x.x);
+            ov[k + 1] = __float_as_uint(x.y);
+          }
+          ptx::tmem_st32(tO + 32 * cc, ov);
+        }
+      }
     } else {
       // pass 1: row maximum (S re-read per chunk keeps registers for O32)
       int smax = INT_MIN;
@@ -484,8 +504,8 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, AlphaBuf
         smax = full_tile ? row_max<16>(sv, smax) : row_max_masked<16>(sv, smax, key0 + 16 * cc, limit);
       }
       const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
-      m_new = fmaxf(m, m_blk);
-      alpha = ptx::ex2(__fsub_rn(m, m_new));
+      m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
+      alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
       // pass 2: P^ = e4m3(448 p), four per TMEM column, written over S
 #pragma unroll
       for (int cc = 0; cc < SUB / 16; ++cc) {
@@ -577,54 +597,6 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, AlphaBuf
   }
 }
 
-// ------------------------------------------------------------ correction --
-
-// 16-bit P.V: before P.V of sub-tile i accumulates into O_t, O_t must be
-// scaled by alpha_i (exp2 of the old minus the new row maximum).  The
-// correction warpgroup does this for both query tiles, in sub-tile order,
-// skipping the TMEM round trip when alpha is 1 for all 32 rows of a warp.
-template <int D>
-__device__ void correction_wg(const AttnParams& p, const Work& w, Bars* B, const AlphaBuf* AB,
-                              uint32_t tmem) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int quarter = warp & 3;
-  const int r = quarter * 32 + lane;
-  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-  const int n0 = w.nsub0, n1 = w.nsub1;
-  const int nsub = max(n0, n1);
-  for (int i = 0; i < nsub; ++i) {
-    const int b = i & 1;
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (i >= (t == 0 ? n0 : n1)) continue;
-      if (!wait_bar(B, &B->p_full[t][b], (i / 2) & 1, p.status, true)) return;
-      const float alpha = AB->a[t][b][r];
-      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
-        ptx::tc_fence_after();
-        const uint32_t tO = tmem + 256 + D * t + lane_off;
-        const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(tO + 32 * cc, ov);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float2 x = __fmul2_rn(a2, make_float2(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1])));
-            ov[k] = __float_as_uint(x.x);
-            ov[k + 1] = __float_as_uint(x.y);
-          }
-          ptx::tmem_st32(tO + 32 * cc, ov);
-        }
-        ptx::tmem_wait_st();
-      }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&B->o_ready[t][b]);
-    }
-  }
-}
-
 // ---------------------------------------------------------------- kernel --
 
 template <int D, bool PV8, bool BF16V>
@@ -638,31 +610,30 @@ __global__ void __launch_bounds__(Cfg<D, PV8>::THREADS, 1)
   uint8_t* sK = sQ + 2 * C::QT;
   uint8_t* sV = sK + C::NS * C::QT;
   Bars* B = reinterpret_cast<Bars*>(sV + C::NS * C::VT);
-  AlphaBuf* AB = reinterpret_cast<AlphaBuf*>(reinterpret_cast<uint8_t*>(B) + 1024);
-  static_assert(sizeof(Bars) <= 1024 && sizeof(AlphaBuf) + 1024 <= C::AUX, "aux layout");
+  static_assert(sizeof(Bars) <= C::AUX, "aux layout");
 
   const Work w = decode_work(p);
   if (!w.valid) return;
   const int warp = threadIdx.x / 32;
   const int wg = warp / 4;
-  const int warp_tma = 4 * C::WG_CTRL, warp_mma = 4 * C::WG_CTRL + 1;
+  const int warp_tma = 4 * C::WG_CTRL, warp_mma = 4 * C::WG_CTRL + 1;  // MMA warps: +1, +2
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&B->q_full, 1);
-    ptx::mbar_init(&B->done, 1);
+    ptx::mbar_init(&B->done[0], 1);
+    ptx::mbar_init(&B->done[1], 1);
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(&B->o_full[t], 1);
       ptx::mbar_init(&B->o_done[t], 1);
       for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(&B->s_full[t][b], 1);
         ptx::mbar_init(&B->p_full[t][b], 128);
-        ptx::mbar_init(&B->o_ready[t][b], 128);
       }
     }
     for (int s = 0; s < C::NS; ++s) {
       ptx::mbar_init(&B->k_full[s], 1);
       ptx::mbar_init(&B->v_full[s], 1);
-      ptx::mbar_init(&B->kv_empty[s], 1);
+      ptx::mbar_init(&B->kv_empty[s], 2);  // one commit per query tile
     }
     B->abort = 0;
     ptx::fence_barrier_init();
@@ -680,15 +651,12 @@ __global__ void __launch_bounds__(Cfg<D, PV8>::THREADS, 1)
     ptx::setmaxnreg_dec<C::REG_CTRL>();
     if (warp == warp_tma) {
       producer<D, PV8>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, p.status);
-    } else if (warp == warp_mma) {
-      mma_issuer<D, PV8, BF16V>(w, B, tmem, sQ, sK, sV, p.status);
+    } else if (warp == warp_mma || warp == warp_mma + 1) {
+      mma_issuer<D, PV8, BF16V>(w, B, tmem, sQ, sK, sV, warp - warp_mma, p.status);
     }
-  } else if (!PV8 && wg == C::WG_CORR) {
-    ptx::setmaxnreg_dec<C::REG_CORR>();
-    correction_wg<D>(p, w, B, AB, tmem);
   } else {
     ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
-    softmax_wg<D, PV8, BF16V>(p, w, B, AB, tmem, wg);
+    softmax_wg<D, PV8, BF16V>(p, w, B, tmem, wg);
   }
 
   ptx::tc_fence_before();

@@ -388,3 +388,25 @@ def test_emulation_close_to_reference_on_gaussian_data():
     o = heads.emulate_rows(qz, v, None, picks, D, False, "fp16")
     unsmoothed = np.stack([o[p] for p in picks])
     assert cos(unsmoothed) < 0.9999
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulation_rescale_threshold_changes_rounding_only(causal):
+    """The threshold tau of the running maximum cancels in O / l: tau = 8 and
+    tau = 0 differ only through the rounding of P (|diff| <= 2^-10 max|v|), and
+    both stay within that bound of the fp64 reference on lossless inputs."""
+    n, D = 300, 16
+    q, k, v = _lossless_inputs(n, D, 17, q_exp=(0, -1, 1), k_exp=(-1, 0, 1))
+    sm = 1.0 / 12000.0
+    qt, kt, vt = (torch.from_numpy(x)[None, None].half() for x in (q, k, v))
+    qz = heads.quantize(qt, kt, vt, None, "fp16")
+    outs = {}
+    for tau in (0.0, 8.0):
+        outs[tau] = oracle.attn_emul_rows(qz.q_codes[0, 0], qz.q_delta[0, 0], qz.k_codes[0, 0],
+                                          qz.k_delta[0, 0], n, D, sm, causal, "fp16",
+                                          np.arange(n), v=v, tau=tau)
+    bound = 2.0 ** -10 * np.abs(v).max() + 1e-5
+    assert np.abs(outs[0.0] - outs[8.0]).max() <= bound
+    ref = oracle.attn_ref_rows(q, k, v, float(np.float32(sm)), causal, np.arange(n))
+    assert np.abs(outs[8.0] - ref).max() <= bound
+    assert not np.array_equal(outs[0.0], outs[8.0])   # the threshold is in effect
