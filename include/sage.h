@@ -248,6 +248,15 @@ sage_status_t sage_qk_int8_tiles(const int8_t* q_codes, const int8_t* k_codes, i
 sage_status_t sage_selftest_wait_timeout(long long wait_cycles, void* ws, size_t ws_bytes,
                                          void* stream);
 
+/*
+ * Self-test of the software 2^x the attention kernel evaluates on the FMA
+ * pipe for a share of the softmax exponentials (online softmax in base 2,
+ * "Attention机制优化：从FlashAttention到SageAttention的工程实践", section 3.1):
+ * y[i] = 2^x[i] for n DEVICE floats.  Valid for x >= -125 (smaller x are
+ * clamped to -125); relative error below 2.2e-7.
+ */
+sage_status_t sage_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,6 +33,7 @@ SIGNATURES = {
                               _P, _P, _SZ, _P], _I),
     "sage_qk_int8_tiles": ([_P, _P, _I, _I, _I, _P, _I, _P, _P, _SZ, _P], _I),
     "sage_selftest_wait_timeout": ([ctypes.c_longlong, _P, _SZ, _P], _I),
+    "sage_selftest_exp2": ([_P, _P, _I, _P], _I),
     "sage_quantize_noalloc": ([_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
                                _P, _P], _I),
 }

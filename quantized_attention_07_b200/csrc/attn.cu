@@ -39,6 +39,7 @@
 // watch, and everyone falls through to the teardown, which waits (bounded) for
 // the CTA's own TMA loads and MMAs and always frees TMEM.
 #include "attn_launch.cuh"
+#include "exp2.cuh"
 #include "ptx.cuh"
 
 namespace sage {
@@ -390,6 +391,10 @@ __device__ __forceinline__ int row_max_masked(const uint32_t* v, int acc, int fi
   return acc;
 }
 
+// Share of the exponentials computed by the FMA-pipe polynomial: one pair in
+// POLY_EVERY (0 = none; every 2^x on the special-function unit).
+constexpr int POLY_EVERY = 0;
+
 // p for NC columns: p = 2^fma(S, c, -m) (masked columns give 0); returns the
 // sum of p.  Results are written to p[].
 template <bool MASKED, int NC>
@@ -400,7 +405,15 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
 #pragma unroll
   for (int i = 0; i < NC; i += 2) {
     const float2 a = __ffma2_rn(s32x2_to_f32x2(v[i], v[i + 1]), c2, n2);
-    float p0 = ptx::ex2(a.x), p1 = ptx::ex2(a.y);
+    float p0, p1;
+    if (POLY_EVERY > 0 && (i / 2) % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1) {
+      const float2 e = exp2_poly2(a);  // FMA-pipe 2^x for a share of the pairs
+      p0 = e.x;
+      p1 = e.y;
+    } else {
+      p0 = ptx::ex2(a.x);
+      p1 = ptx::ex2(a.y);
+    }
     if (MASKED) {
       if (first_key + i >= limit) p0 = 0.0f;
       if (first_key + i + 1 >= limit) p1 = 0.0f;
