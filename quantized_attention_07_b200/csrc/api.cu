@@ -16,7 +16,8 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
-                         uint32_t* v_amax, uint32_t* status, cudaStream_t st);
+                         uint32_t* v_amax, uint32_t* status, unsigned int* sync,
+                         cudaStream_t st);
 cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
                             const int32_t* tiles, int n, int32_t* out, uint32_t* status,
                             cudaStream_t st);
@@ -50,7 +51,7 @@ float kappa_of(float sm_scale, int D) {
 
 // Workspace layout.  Offsets in bytes from the workspace base.
 struct Layout {
-  size_t k_sum, v_amax, blk_off, pair_off;             // scratch
+  size_t k_sum, v_amax, sync, blk_off, pair_off;       // scratch
   size_t q_codes, k_codes, q_scale, k_scale, k_mean;   // quantised operands
   size_t v_codes, v_scale;
   size_t scratch_end, total;
@@ -62,6 +63,7 @@ Layout dense_layout(int B, int H, int N, int D, bool fp8) {
   size_t o = kHeader;
   L.k_sum = o; o += al(BH * D * 8);
   L.v_amax = o; o += al(BH * D * 4);
+  L.sync = o; o += al((BH + 1) * 4);
   L.scratch_end = o;
   L.q_codes = o; o += al(BH * NP * D);
   L.k_codes = o; o += al(BH * NP * D);
@@ -85,6 +87,7 @@ Layout varlen_layout(int T, int batch, int H, int D, bool fp8) {
   size_t o = kHeader;
   L.k_sum = o; o += al(SH * D * 8);
   L.v_amax = o; o += al(SH * D * 4);
+  L.sync = o; o += al(4);
   L.blk_off = o; o += al(((size_t)batch + 1) * 4);
   L.pair_off = o; o += al(((size_t)batch + 1) * 4);
   L.scratch_end = o;
@@ -120,9 +123,14 @@ template <class T> T* at(void* ws, size_t off) {
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 sage_status_t clear_scratch(void* ws, const Layout& L, bool fp8, cudaStream_t st) {
+  // K sums, (FP8) V maxima and the dense work/completion counters start at 0
   cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, L.k_sum), 0, L.v_amax - L.k_sum, st);
   if (e == cudaSuccess && fp8)
-    e = cudaMemsetAsync(at<uint8_t>(ws, L.v_amax), 0, L.scratch_end - L.v_amax, st);
+    e = cudaMemsetAsync(at<uint8_t>(ws, L.v_amax), 0, L.sync - L.v_amax, st);
+  if (e == cudaSuccess) {
+    const size_t sync_end = L.blk_off ? L.blk_off : L.scratch_end;
+    e = cudaMemsetAsync(at<uint8_t>(ws, L.sync), 0, sync_end - L.sync, st);
+  }
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "cudaMemsetAsync");
 }
 
@@ -142,7 +150,7 @@ sage_status_t quantize_dense(const void* q, const void* k, const void* v, int in
   cudaError_t e = launch_quant(S, grid, D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
                                k_codes, k_scale, k_mean, v_codes, v_scale,
                                at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                               at<uint32_t>(ws, 0), st);
+                               at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync), st);
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
 
@@ -323,7 +331,7 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
   e = launch_quant(S, dim3((unsigned)TB, H), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
                    k_codes, k_scale, k_mean, v_codes, v_scale,
                    at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                   at<uint32_t>(ws, 0), st);
+                   at<uint32_t>(ws, 0), nullptr, st);
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
 

@@ -7,6 +7,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <cstring>
 
 #include "sage.h"
 
@@ -52,25 +53,53 @@ template <bool BF16> struct In16;
 template <> struct In16<false> {
   using T = __half;
   using T2 = __half2;
+  // Lane-wise maximum of two packed pairs (a NaN lane yields the other value).
+  __device__ static uint32_t max2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  }
+  // Lane-wise max(|a|, |b|); the sign bit of each lane is garbage (mask it).
+  __device__ static uint32_t absmax2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  }
+  // Packed pair (element 0 in the low half) -> two exact floats.
   __device__ static float2 to_float2(uint32_t u) {
-    __half2 h = *reinterpret_cast<__half2*>(&u);
+    __half2 h;
+    memcpy(&h, &u, 4);
     return __half22float2(h);
   }
   __device__ static uint32_t pack(float lo, float hi) {
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
+    const __half2 h = __floats2half2_rn(lo, hi);
+    uint32_t u;
+    memcpy(&u, &h, 4);
+    return u;
   }
 };
 template <> struct In16<true> {
   using T = __nv_bfloat16;
   using T2 = __nv_bfloat162;
+  __device__ static uint32_t max2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  }
+  __device__ static uint32_t absmax2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+  }
+  // bf16 is the high half of an fp32 bit pattern.
   __device__ static float2 to_float2(uint32_t u) {
-    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
-    return __bfloat1622float2(h);
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
   }
   __device__ static uint32_t pack(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    uint32_t u;
+    memcpy(&u, &h, 4);
+    return u;
   }
 };
 

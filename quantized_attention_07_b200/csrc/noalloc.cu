@@ -30,7 +30,8 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
-                         uint32_t* v_amax, uint32_t* status, cudaStream_t st);
+                         uint32_t* v_amax, uint32_t* status, unsigned int* sync,
+                         cudaStream_t st);
 }  // namespace sage
 
 namespace {
@@ -38,10 +39,14 @@ namespace {
 constexpr size_t kScratchBytes = SAGE_NOALLOC_SCRATCH_BYTES;
 constexpr long long kMaxBHD = SAGE_NOALLOC_MAX_BHD;
 
-// Layout: [0, 256) status word; then the int64 K sums; then the V maxima.
+// Layout: [0, 256) status word; then the int64 K sums; then the V maxima;
+// then the work / completion counters of the quantisation kernel (one per
+// (batch, head) plus one; B*H <= SAGE_NOALLOC_MAX_BHD / 64).
 constexpr size_t kSumOff = 256;
 constexpr size_t kAmaxOff = kSumOff + (size_t)kMaxBHD * 8;
-static_assert(kAmaxOff + (size_t)kMaxBHD * 4 <= kScratchBytes, "scratch layout");
+constexpr size_t kSyncOff = kAmaxOff + (size_t)kMaxBHD * 4;
+constexpr size_t kMaxUnits = kMaxBHD / 64;
+static_assert(kSyncOff + (kMaxUnits + 1) * 4 <= kScratchBytes, "scratch layout");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -95,6 +100,7 @@ extern "C" sage_status_t sage_quantize_noalloc(
   e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(scratch + kSumOff, 0, bhd * 8, st);
   if (e == cudaSuccess && fp8) e = cudaMemsetAsync(scratch + kAmaxOff, 0, bhd * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(scratch + kSyncOff, 0, ((size_t)B * H + 1) * 4, st);
   if (e != cudaSuccess) return SAGE_ERR_CUDA;
 
   sage::SeqLayout L{};
@@ -104,6 +110,7 @@ extern "C" sage_status_t sage_quantize_noalloc(
   e = sage::launch_quant(L, dim3((N + sage::BLK - 1) / sage::BLK, B * H), D, in_dt == SAGE_BF16,
                          fp8, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes,
                          v_scale, reinterpret_cast<unsigned long long*>(scratch + kSumOff),
-                         reinterpret_cast<uint32_t*>(scratch + kAmaxOff), status, st);
+                         reinterpret_cast<uint32_t*>(scratch + kAmaxOff), status,
+                         reinterpret_cast<unsigned int*>(scratch + kSyncOff), st);
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

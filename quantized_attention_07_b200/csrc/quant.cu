@@ -13,6 +13,14 @@
 //     - V (FP8 P.V only): codes = e4m3(v * 448/max|v_d|), per channel
 //       ("SageAttention v1/v2/v2++/v3 overview", SageAttention 2 bullet 1).
 //
+// Dense inputs run both passes in one persistent kernel (one CTA per SM): a
+// producer warp streams 128-token slabs into shared memory with bulk copies,
+// in the work order  p1(head 0) .. p1(head lag-1), p1(lag), p2(0), p1(lag+1),
+// p2(1), ...  so that a head's K (and V) is re-read by pass 2 from L2 shortly
+// after pass 1 streamed it; eight consumer warps quantise from shared memory.
+// A pass-2 block waits (bounded) until all pass-1 blocks of its head are done.
+// Variable-length batches use two separate launches.
+//
 // Every arithmetic step is one IEEE binary32 (or binary64 for the mean)
 // operation with round-to-nearest-even, written with explicit __f*_rn
 // intrinsics so that no multiply-add contraction changes a code.
@@ -20,7 +28,10 @@
 // Thread layout: 256 threads; a 16-byte vector holds 8 channels; thread t owns
 // channel group c = t % (D/8) of rows t/(D/8) + i*(256/(D/8)).  Consecutive
 // threads read consecutive 16-byte vectors of one row: fully coalesced.
+#include <type_traits>
+
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace sage {
 namespace {
@@ -46,6 +57,18 @@ struct BlockPos {
   long long scale_idx;   // index of this block's delta
   int b;          // block index within the sequence
 };
+
+__device__ __forceinline__ void dense_block_pos(const SeqLayout& L, int bh, int b, BlockPos& P) {
+  const int NB = (L.N + BLK - 1) / BLK;
+  P.b = b;
+  P.seq = bh;
+  P.n = L.N;
+  P.rows = min(BLK, L.N - P.b * BLK);
+  P.row0 = (long long)bh * L.N + (long long)P.b * BLK;
+  P.row_stride = 1;
+  P.code_row0 = ((long long)bh * NB + P.b) * BLK;
+  P.scale_idx = (long long)bh * NB + P.b;
+}
 
 __device__ __forceinline__ bool block_pos(const SeqLayout& L, BlockPos& P) {
   if (!L.varlen) {
@@ -77,26 +100,35 @@ __device__ __forceinline__ bool block_pos(const SeqLayout& L, BlockPos& P) {
   return true;
 }
 
-// Load this thread's rows of a 16-bit [.., D] tensor block as floats (zeros
-// past the valid rows).
-template <int D, bool BF16>
-__device__ __forceinline__ void load_block(const void* base, const BlockPos& P,
-                                           float (&x)[Tile<D>::NIT][8]) {
+// Issue the loads of this thread's rows of a 16-bit [.., D] tensor block
+// (zeros past the valid rows).  Callers issue every tensor's loads before they
+// use any of them, so a CTA keeps all its 16-byte requests in flight at once.
+template <int D>
+__device__ __forceinline__ void load_raw(const void* base, const BlockPos& P,
+                                         uint4 (&u)[Tile<D>::NIT]) {
   using T = Tile<D>;
   const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
   const uint16_t* p16 = static_cast<const uint16_t*>(base);
 #pragma unroll
   for (int i = 0; i < T::NIT; ++i) {
     const int r = r0 + i * T::RS;
-    uint4 u = make_uint4(0, 0, 0, 0);
+    u[i] = make_uint4(0, 0, 0, 0);
     if (r < P.rows) {
       const long long row = P.row0 + (long long)r * P.row_stride;
-      u = __ldg(reinterpret_cast<const uint4*>(p16 + row * D) + c);
+      u[i] = __ldg(reinterpret_cast<const uint4*>(p16 + row * D) + c);
     }
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  }
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ void to_float(const uint4 (&u)[Tile<D>::NIT],
+                                         float (&x)[Tile<D>::NIT][8]) {
+#pragma unroll
+  for (int i = 0; i < Tile<D>::NIT; ++i) {
+    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float2 f = In16<BF16>::to_float2(w[e]);
+      const float2 f = In16<BF16>::to_float2(w[e]);
       x[i][2 * e] = f.x;
       x[i][2 * e + 1] = f.y;
     }
@@ -142,23 +174,26 @@ __device__ __forceinline__ void store_codes(const float (&x)[Tile<D>::NIT][8], f
 // ------------------------------------------------------------------ pass 1 --
 
 template <int D, bool BF16, bool FP8>
-__global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
-    SeqLayout L, const void* __restrict__ q, const void* __restrict__ k,
+__device__ __forceinline__ void pass1_block(
+    const BlockPos& P, const void* __restrict__ q, const void* __restrict__ k,
     const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
     unsigned long long* __restrict__ k_sum, uint32_t* __restrict__ v_amax,
     uint32_t* __restrict__ status) {
   using T = Tile<D>;
   __shared__ float red[THREADS / 32];
   __shared__ long long red64[THREADS / 32][D];
-  BlockPos P;
-  if (!block_pos(L, P)) return;
   const int c = threadIdx.x % T::CPR;
   const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
+
+  uint4 rq[T::NIT], rk[T::NIT], rv[FP8 ? T::NIT : 1];
+  load_raw<D>(q, P, rq);
+  load_raw<D>(k, P, rk);
+  if constexpr (FP8) load_raw<D>(v, P, rv);
 
   // --- Q: per-block quantiser
   {
     float x[T::NIT][8];
-    load_block<D, BF16>(q, P, x);
+    to_float<D, BF16>(rq, x);
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < T::NIT; ++i)
@@ -172,7 +207,7 @@ __global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
   // --- K: exact fixed-point channel sums
   {
     float x[T::NIT][8];
-    load_block<D, BF16>(k, P, x);
+    to_float<D, BF16>(rk, x);
     long long acc[8];
     bool bad = false;
 #pragma unroll
@@ -205,7 +240,7 @@ __global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
   // --- V: per-channel max|v| (FP8 P.V only)
   if constexpr (FP8) {
     float x[T::NIT][8];
-    load_block<D, BF16>(v, P, x);
+    to_float<D, BF16>(rv, x);
     float m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = 0.0f;
@@ -233,6 +268,17 @@ __global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
   }
 }
 
+template <int D, bool BF16, bool FP8>
+__global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
+    SeqLayout L, const void* __restrict__ q, const void* __restrict__ k,
+    const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+    unsigned long long* __restrict__ k_sum, uint32_t* __restrict__ v_amax,
+    uint32_t* __restrict__ status) {
+  BlockPos P;
+  if (!block_pos(L, P)) return;
+  pass1_block<D, BF16, FP8>(P, q, k, v, q_codes, q_scale, k_sum, v_amax, status);
+}
+
 // ------------------------------------------------------------------ pass 2 --
 
 __device__ __forceinline__ float k_mean_value(unsigned long long sum, int n) {
@@ -242,28 +288,40 @@ __device__ __forceinline__ float k_mean_value(unsigned long long sum, int n) {
 }
 
 template <int D, bool BF16, bool FP8>
-__global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
-    SeqLayout L, const void* __restrict__ k, const void* __restrict__ v,
-    const unsigned long long* __restrict__ k_sum, const uint32_t* __restrict__ v_amax,
+__device__ __forceinline__ void pass2_block(
+    const BlockPos& P, const void* __restrict__ k, const void* __restrict__ v,
+    const unsigned long long* k_sum, const uint32_t* v_amax,
     int8_t* __restrict__ k_codes, float* __restrict__ k_scale, float* __restrict__ k_mean,
     uint8_t* __restrict__ v_codes, float* __restrict__ v_scale) {
   using T = Tile<D>;
   __shared__ float red[THREADS / 32];
-  BlockPos P;
-  if (!block_pos(L, P)) return;
+  __shared__ float s_chan[2][D];  // K channel means, V scale factors
   const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
   const long long chan0 = (long long)P.seq * D;
 
-  if (P.b == 0 && threadIdx.x < D)
-    k_mean[chan0 + threadIdx.x] = k_mean_value(__ldg(k_sum + chan0 + threadIdx.x), P.n);
+  uint4 rk[T::NIT], rv[FP8 ? T::NIT : 1];
+  load_raw<D>(k, P, rk);
+  if constexpr (FP8) load_raw<D>(v, P, rv);
+
+  if (threadIdx.x < D) {
+    const float mu = k_mean_value(__ldcg(k_sum + chan0 + threadIdx.x), P.n);
+    s_chan[0][threadIdx.x] = mu;
+    if (P.b == 0) k_mean[chan0 + threadIdx.x] = mu;
+    if constexpr (FP8) {
+      const float am = __uint_as_float(__ldcg(v_amax + chan0 + threadIdx.x));
+      s_chan[1][threadIdx.x] = am > 0.0f ? __fdiv_rn(448.0f, am) : 0.0f;
+      if (P.b == 0) v_scale[chan0 + threadIdx.x] = am > 0.0f ? __fdiv_rn(am, 448.0f) : 0.0f;
+    }
+  }
+  __syncthreads();
 
   // --- K: smoothing + per-block quantiser
   {
     float m[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m[e] = k_mean_value(__ldg(k_sum + chan0 + 8 * c + e), P.n);
+    for (int e = 0; e < 8; ++e) m[e] = s_chan[0][8 * c + e];
     float x[T::NIT][8];
-    load_block<D, BF16>(k, P, x);
+    to_float<D, BF16>(rk, x);
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < T::NIT; ++i) {
@@ -283,16 +341,9 @@ __global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
   if constexpr (FP8) {
     float sv[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float am = __uint_as_float(__ldg(v_amax + chan0 + 8 * c + e));
-      sv[e] = am > 0.0f ? __fdiv_rn(448.0f, am) : 0.0f;
-    }
-    if (P.b == 0 && threadIdx.x < D) {
-      const float am = __uint_as_float(__ldg(v_amax + chan0 + threadIdx.x));
-      v_scale[chan0 + threadIdx.x] = am > 0.0f ? __fdiv_rn(am, 448.0f) : 0.0f;
-    }
+    for (int e = 0; e < 8; ++e) sv[e] = s_chan[1][8 * c + e];
     float x[T::NIT][8];
-    load_block<D, BF16>(v, P, x);
+    to_float<D, BF16>(rv, x);
 #pragma unroll
     for (int i = 0; i < T::NIT; ++i) {
       const int r = r0 + i * T::RS;
@@ -305,6 +356,539 @@ __global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
         *reinterpret_cast<uint2*>(v_codes + row * D + 8 * c) = make_uint2(w0, w1);
       }
     }
+  }
+}
+
+template <int D, bool BF16, bool FP8>
+__global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
+    SeqLayout L, const void* __restrict__ k, const void* __restrict__ v,
+    const unsigned long long* __restrict__ k_sum, const uint32_t* __restrict__ v_amax,
+    int8_t* __restrict__ k_codes, float* __restrict__ k_scale, float* __restrict__ k_mean,
+    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale) {
+  BlockPos P;
+  if (!block_pos(L, P)) return;
+  pass2_block<D, BF16, FP8>(P, k, v, k_sum, v_amax, k_codes, k_scale, k_mean, v_codes, v_scale);
+}
+
+// ---------------------------------------------------------- streamed, dense --
+//
+// Dense inputs: one persistent CTA per SM.  Warp 8 claims work items from a
+// global counter and streams each item's 128-token slabs (in the dense layout
+// a block of one head is one contiguous [rows, D] slab per tensor) into a ring
+// of shared-memory slots with cp.async.bulk; warps 0-7 take the slots in the
+// same order and write codes, scales and sums.
+//
+// Work items are (pass, head, block) in groups of NB blocks ordered
+//   p1(0) .. p1(lag-1), then p1(u), p2(u-lag) for u = lag .. U-1, then the
+//   remaining p2,
+// so that pass 2 re-reads a head's K (and V) from L2 shortly after pass 1
+// streamed it (pass-1 K and V slabs are loaded with an evict-last L2 policy,
+// everything else evict-first).  Before it loads a pass-2 item the producer
+// waits (bounded) until every pass-1 block of that head is counted done; those
+// were claimed earlier by running CTAs, which finish them without waiting on
+// anything claimed later, so the wait ends.
+
+__device__ __forceinline__ void fused_item(int x, int NB, int U, int lag, int& pass, int& u,
+                                           int& b) {
+  const int g = x / NB;
+  b = x - g * NB;
+  if (g < lag) { pass = 1; u = g; return; }
+  const int k = g - lag;
+  if (k < 2 * (U - lag)) {
+    u = lag + k / 2;
+    if (k & 1) { pass = 2; u -= lag; } else { pass = 1; }
+    return;
+  }
+  pass = 2;
+  u = U - lag + (k - 2 * (U - lag));
+}
+
+template <int D>
+struct Stream {
+  static constexpr int CONSUMERS = 256;                   // warps 0-7
+  static constexpr int THREADS = CONSUMERS + 32;          // + producer warp 8
+  static constexpr int SLOT = BLK * D * 2;                // one [128, D] 16-bit slab
+  static constexpr int NS = D == 128 ? 3 : 6;             // ring slots (96 KiB)
+  static constexpr size_t SMEM = (size_t)NS * SLOT;
+  static constexpr int CTAS_PER_SM = 2;
+};
+
+template <int N>
+__device__ __forceinline__ int tensors_of(int pass) {
+  return pass == 1 ? N : N - 1;  // p1: Q, K (, V);  p2: K (, V)
+}
+
+// 1.5 * 2^23: for |y| < 2^22, the fp32 sum y + kMagic is kMagic + rint(y)
+// (round to nearest even), and its low mantissa byte is rint(y) mod 256.
+constexpr float kMagic = 12582912.0f;
+
+// Low bytes of four floats' bit patterns, packed (a in byte 0).
+__device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float d) {
+  const uint32_t ab = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
+  const uint32_t cd = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
+}
+
+// Consumer-side helpers.  Thread t owns the 16-byte chunk c = t % (D/8) of
+// rows r0 + i*RS of a slab (as in the two-launch path); it copies them from
+// shared memory into registers once (zeros past the valid rows), so the slot
+// can be handed back to the producer at once.  FULL: all 128 rows valid.
+
+template <int D, bool FULL>
+__device__ __forceinline__ void slab_to_regs(const uint4* slab, int rows,
+                                             uint4 (&u)[Tile<D>::NIT]) {
+  using T = Tile<D>;
+  const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i) {
+    const int r = r0 + i * T::RS;
+    u[i] = (FULL || r < rows) ? slab[r * T::CPR + c] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// max |x| over the thread's values (zeros do not change it).  The max of
+// 16-bit values is exact; a NaN is ignored as by fmaxf.
+template <int D, bool BF16>
+__device__ __forceinline__ float regs_absmax(const uint4 (&u)[Tile<D>::NIT]) {
+  uint32_t m[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < Tile<D>::NIT; ++i) {
+    m[0] = In16<BF16>::absmax2(m[0], u[i].x);
+    m[1] = In16<BF16>::absmax2(m[1], u[i].y);
+    m[2] = In16<BF16>::absmax2(m[2], u[i].z);
+    m[3] = In16<BF16>::absmax2(m[3], u[i].w);
+  }
+  float a = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = In16<BF16>::to_float2(m[e] & 0x7fff7fffu);
+    a = fmaxf(a, fmaxf(f.x, f.y));
+  }
+  return a;
+}
+
+// codes = rint((x - mean) * s) for the valid rows, 0 for padding rows, with
+// s = 127/amax.  |x - mean| <= amax bounds |(x - mean) * s| by 127(1 + 2^-23),
+// so the codes need no clamp.  Each step is one IEEE fp32 operation
+// (x - mean, the product, the rounding), as in the two-launch path.
+template <int D, bool BF16, bool SUB, bool FULL>
+__device__ __forceinline__ void regs_codes(const uint4 (&u)[Tile<D>::NIT], int rows, float amax,
+                                           const float (&mean)[8], int8_t* codes,
+                                           long long code_row0) {
+  using T = Tile<D>;
+  const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
+  const float s = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  float2 nm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) nm[e] = make_float2(-mean[2 * e], -mean[2 * e + 1]);
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i) {
+    const int r = r0 + i * T::RS;
+    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+    float2 y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float2 f = In16<BF16>::to_float2(w[e]);
+      if constexpr (SUB) f = __fadd2_rn(f, nm[e]);
+      // scalar __fmul_rn / __fadd_rn: documented never to be fused into an
+      // fma (which would round x*s and its rint as one step); the packed
+      // forms were fused here
+      y[e] = make_float2(__fadd_rn(__fmul_rn(f.x, s), kMagic), __fadd_rn(__fmul_rn(f.y, s), kMagic));
+    }
+    uint2 out = make_uint2(low_bytes4(y[0].x, y[0].y, y[1].x, y[1].y),
+                           low_bytes4(y[2].x, y[2].y, y[3].x, y[3].y));
+    if (!FULL && r >= rows) out = make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(codes + (code_row0 + r) * D + 8 * c) = out;
+  }
+}
+
+// max |x - mean| over the thread's valid rows.
+template <int D, bool BF16, bool FULL>
+__device__ __forceinline__ float regs_absmax_sub(const uint4 (&u)[Tile<D>::NIT], int rows,
+                                                 const float (&mean)[8]) {
+  using T = Tile<D>;
+  const int r0 = threadIdx.x / T::CPR;
+  float2 nm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) nm[e] = make_float2(-mean[2 * e], -mean[2 * e + 1]);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i) {
+    if (FULL || r0 + i * T::RS < rows) {
+      const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 y = __fadd2_rn(In16<BF16>::to_float2(w[e]), nm[e]);
+        a = fmaxf(a, fmaxf(fabsf(y.x), fabsf(y.y)));
+      }
+    }
+  }
+  return a;
+}
+
+// Exact sums of rint(x * 2^24) over the thread's rows, per channel, as two
+// fp32 sums: hi = sum of h = rint(16x), fr = sum of d = 16x - h, so that the
+// total is 2^20 (hi + fr).  For |x| < 2^16: |h| <= 2^20 and d is exact with
+// |d| <= 1/2 and a multiple of 2^-20 (x is a multiple of 2^-24 for every
+// fp16, and for every bf16 of magnitude 2^-17 or more; smaller bf16 values
+// take one more rounding of d to that grid, which is rint of x * 2^24).  Over
+// the at most 16 rows that meet in one warp, |sum h| <= 2^24 and |sum d| <= 8
+// on a 2^-20 grid: neither sum ever rounds.
+template <int D, bool BF16>
+__device__ __forceinline__ void regs_fixed_sums(const uint4 (&u)[Tile<D>::NIT], float2 (&hi)[4],
+                                                float2 (&fr)[4], uint32_t& absbits) {
+  const float2 M2 = make_float2(kMagic, kMagic), nM2 = make_float2(-kMagic, -kMagic);
+  const float2 k16 = make_float2(16.0f, 16.0f);
+  const float2 G2 = make_float2(12.0f, 12.0f), nG2 = make_float2(-12.0f, -12.0f);  // 1.5*2^3
+#pragma unroll
+  for (int e = 0; e < 4; ++e) hi[e] = fr[e] = make_float2(0.0f, 0.0f);
+  absbits = 0u;
+#pragma unroll
+  for (int i = 0; i < Tile<D>::NIT; ++i) {
+    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (BF16) absbits = __vmaxu2(absbits, w[e] & 0x7fff7fffu);
+      const float2 f = In16<BF16>::to_float2(w[e]);
+      const float2 h = __fadd2_rn(__ffma2_rn(f, k16, M2), nM2);       // rint(16x)
+      float2 d = __ffma2_rn(f, k16, make_float2(-h.x, -h.y));        // 16x - h, exact
+      if constexpr (BF16) d = __fadd2_rn(__fadd2_rn(d, G2), nG2);     // onto the 2^-20 grid
+      hi[e] = __fadd2_rn(hi[e], h);
+      fr[e] = __fadd2_rn(fr[e], d);
+    }
+  }
+}
+
+// Block max over the 256 consumer threads; red is [2][8], used alternately.
+__device__ __forceinline__ float consumer_block_max(float v, float* red, int& par) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[par * 8 + threadIdx.x / 32] = v;
+  ptx::named_sync<256>();
+  float m = red[par * 8];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = fmaxf(m, red[par * 8 + i]);
+  par ^= 1;
+  return m;
+}
+
+__device__ __forceinline__ void release_slot(uint64_t* empty) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(empty);
+}
+
+// sync[0]: work counter; sync[1 + u]: pass-1 blocks of head u completed.
+template <int D, bool BF16, bool FP8>
+__global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) quant_stream_kernel(
+    SeqLayout L, int U, int lag, const void* __restrict__ q, const void* __restrict__ k,
+    const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+    int8_t* __restrict__ k_codes, float* __restrict__ k_scale, float* __restrict__ k_mean,
+    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale, unsigned long long* k_sum,
+    uint32_t* v_amax, uint32_t* status, unsigned int* sync) {
+  using S = Stream<D>;
+  using T = Tile<D>;
+  constexpr int NS = S::NS;
+  constexpr int NT = FP8 ? 3 : 2;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t full[NS], empty[NS];
+  __shared__ int info[NS];
+  __shared__ float red[16];
+  // per slot, written by the producer with a pass-2 slab: the K channel
+  // means (K slab) or the V scale factors 448/max|v| (V slab)
+  __shared__ float s_side[NS][D];
+  // pass 1: the consumer warps' partial channel sums (or V maxima, as float
+  // bits) of the block, combined after a barrier
+  __shared__ long long red64[8][D];
+  __shared__ int s_abort, s_filled, s_consumed;
+
+  const int NB = (L.N + BLK - 1) / BLK;
+  const int total = 2 * U * NB;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 8);
+    }
+    s_abort = 0;
+    s_filled = 0;
+    s_consumed = 0;
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_first = ptx::l2_evict_first(), pol_last = ptx::l2_evict_last();
+    int fill = 0;
+    while (true) {
+      int x = 0;
+      if (lane == 0) x = (int)atomicAdd(sync, 1u);
+      x = __shfl_sync(0xffffffffu, x, 0);
+      const bool end = x >= total;
+      int pass = 0, u = 0, b = 0;
+      if (!end) fused_item(x, NB, U, lag, pass, u, b);
+      const unsigned target = (unsigned)NB;
+      if (!end && pass == 2 && lane == 0) {
+        const uint32_t* done = sync + 1 + u;
+        if (ptx::ld_acquire_gpu(done) < target) {
+          const long long t0 = clock64();
+          while (ptx::ld_acquire_gpu(done) < target) {
+            if (*reinterpret_cast<volatile uint32_t*>(status) & ST_TIMEOUT) break;
+            if (clock64() - t0 > SAGE_WAIT_LIMIT_CYCLES) {
+              set_status(status, ST_TIMEOUT);
+              break;
+            }
+            __nanosleep(128);
+          }
+        }
+      }
+      __syncwarp();
+      const int nt = end ? 1 : tensors_of<NT>(pass);
+      const long long row0 = (long long)u * L.N + (long long)b * BLK;
+      const int rows = end ? 0 : min(BLK, L.N - b * BLK);
+      bool ok = true;
+      for (int t = 0; t < nt && ok; ++t) {
+        const int slot = fill % NS;
+        if (fill >= NS) {  // lane 0 waits; the verdict is the warp's
+          if (lane == 0) ok = ptx::mbar_wait(&empty[slot], ((fill / NS) & 1) ^ 1);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        if (!ok) break;
+        // tensor t of this item: p1 = (Q, K, V), p2 = (K, V)
+        const int which = pass == 1 ? t : t + 1;
+        if (lane == 0) {
+          info[slot] = end ? -1 : x;
+          if (!end) {
+            const void* base = which == 0 ? q : which == 1 ? k : v;
+            const uint32_t bytes = (uint32_t)rows * D * 2;
+            ptx::mbar_expect_tx(&full[slot], bytes);
+            ptx::bulk_load(smem + (size_t)slot * S::SLOT,
+                           static_cast<const uint16_t*>(base) + row0 * D, bytes, &full[slot],
+                           (pass == 1 && which > 0) ? pol_last : pol_first);
+          }
+        }
+        if (!end && pass == 2) {
+          // per-channel constants of this head, while the copy is in flight
+          // (lane 0's acquire of the completion count, then __syncwarp, orders
+          // these reads after every pass-1 block's sums)
+          const long long chan0 = (long long)u * D;
+#pragma unroll
+          for (int j = 0; j < D / 32; ++j) {
+            const int ch = lane + 32 * j;
+            float val;
+            if (which == 1) {
+              val = k_mean_value(__ldcg(k_sum + chan0 + ch), L.N);
+              if (b == 0) k_mean[chan0 + ch] = val;
+            } else {
+              const float am = __uint_as_float(__ldcg(v_amax + chan0 + ch));
+              val = am > 0.0f ? __fdiv_rn(448.0f, am) : 0.0f;
+              if (b == 0) v_scale[chan0 + ch] = am > 0.0f ? __fdiv_rn(am, 448.0f) : 0.0f;
+            }
+            s_side[slot][ch] = val;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full[slot]);  // release: info, s_side
+        ++fill;
+      }
+      if (!ok) {
+        if (lane == 0) {
+          set_status(status, ST_TIMEOUT);
+          s_abort = 1;
+        }
+        break;
+      }
+      const bool stop = end || *reinterpret_cast<volatile int*>(&s_abort);
+      if (__shfl_sync(0xffffffffu, stop, 0)) break;
+    }
+    if (lane == 0) s_filled = fill;
+  } else {
+    // ----------------------------------------------------------- consumers
+    int cidx = 0, par = 0;
+    bool finished = false;  // left the loop at the end-of-work marker
+    const int c = threadIdx.x % T::CPR;
+    while (true) {
+      const int slot0 = cidx % NS;
+      bool ok = ptx::mbar_wait(&full[slot0], (cidx / NS) & 1);
+      ok = ptx::named_all<256>(ok && !*reinterpret_cast<volatile int*>(&s_abort));
+      if (!ok) break;
+      const int x = info[slot0];
+      if (x < 0) {
+        ++cidx;
+        finished = true;
+        break;
+      }
+      int pass, u, b;
+      fused_item(x, NB, U, lag, pass, u, b);
+      const int nt = tensors_of<NT>(pass);
+      for (int t = 1; t < nt; ++t) ok = ptx::mbar_wait(&full[(cidx + t) % NS], ((cidx + t) / NS) & 1) && ok;
+      ok = ptx::named_all<256>(ok);
+      if (!ok) break;
+      BlockPos P;
+      dense_block_pos(L, u, b, P);
+      const long long chan0 = (long long)P.seq * D;
+      auto slab = [&](int t) {
+        return reinterpret_cast<const uint4*>(smem + (size_t)((cidx + t) % NS) * S::SLOT);
+      };
+      auto empty_of = [&](int t) { return &empty[(cidx + t) % NS]; };
+      const float zero8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+
+      const bool full_blk = P.rows == BLK;
+      uint4 rg[T::NIT];
+      auto take = [&](int t) {  // slab t of this item -> registers; free the slot
+        if (full_blk) slab_to_regs<D, true>(slab(t), P.rows, rg);
+        else slab_to_regs<D, false>(slab(t), P.rows, rg);
+        release_slot(empty_of(t));
+      };
+      auto codes = [&](float amax, const float (&mean)[8], int8_t* out, auto sub) {
+        constexpr bool SUB = decltype(sub)::value;
+        if (full_blk) regs_codes<D, BF16, SUB, true>(rg, P.rows, amax, mean, out, P.code_row0);
+        else regs_codes<D, BF16, SUB, false>(rg, P.rows, amax, mean, out, P.code_row0);
+      };
+
+      if (pass == 1) {
+        // Q: per-block quantiser
+        {
+          take(0);
+          const float amax = consumer_block_max(regs_absmax<D, BF16>(rg), red, par);
+          codes(amax, zero8, q_codes, std::false_type{});
+          if (threadIdx.x == 0)
+            q_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+        }
+        // K: exact fixed-point channel sums
+        {
+          take(1);
+          float2 hi[4], fr[4];
+          uint32_t absbits;
+          regs_fixed_sums<D, BF16>(rg, hi, fr, absbits);
+          bool bad;
+          if constexpr (BF16) {  // |x| >= 2^16 (bf16 0x4780) or not finite
+            bad = (absbits & 0xffffu) >= 0x4780u || (absbits >> 16) >= 0x4780u;
+          } else {  // every finite fp16 is below 2^16: only inf / NaN
+            bad = false;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              bad |= !(fabsf(hi[e].x) <= 16777216.0f) || !(fabsf(hi[e].y) <= 16777216.0f);
+          }
+          if (bad) set_status(status, ST_RANGE);
+#pragma unroll
+          for (int o = T::CPR; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hi[e].x += __shfl_xor_sync(0xffffffffu, hi[e].x, o);
+              hi[e].y += __shfl_xor_sync(0xffffffffu, hi[e].y, o);
+              fr[e].x += __shfl_xor_sync(0xffffffffu, fr[e].x, o);
+              fr[e].y += __shfl_xor_sync(0xffffffffu, fr[e].y, o);
+            }
+          if (lane < T::CPR)  // this warp's share of the channel sums
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              red64[warp][8 * c + 2 * e] = (long long)__float2int_rn(hi[e].x) * 1048576LL +
+                                           __float2int_rn(fr[e].x * 1048576.0f);
+              red64[warp][8 * c + 2 * e + 1] = (long long)__float2int_rn(hi[e].y) * 1048576LL +
+                                               __float2int_rn(fr[e].y * 1048576.0f);
+            }
+          ptx::named_sync<256>();
+          if (threadIdx.x < D) {
+            long long sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += red64[i][threadIdx.x];
+            atomicAdd(k_sum + chan0 + threadIdx.x, (unsigned long long)sum);
+          }
+        }
+        // V: per-channel max|v| (FP8 P.V only)
+        if constexpr (FP8) {
+          take(2);
+          uint32_t m2[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int i = 0; i < T::NIT; ++i) {
+            m2[0] = In16<BF16>::absmax2(m2[0], rg[i].x);
+            m2[1] = In16<BF16>::absmax2(m2[1], rg[i].y);
+            m2[2] = In16<BF16>::absmax2(m2[2], rg[i].z);
+            m2[3] = In16<BF16>::absmax2(m2[3], rg[i].w);
+          }
+          float m[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = In16<BF16>::to_float2(m2[e] & 0x7fff7fffu);
+            m[2 * e] = f.x;
+            m[2 * e + 1] = f.y;
+          }
+#pragma unroll
+          for (int o = T::CPR; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], __shfl_xor_sync(0xffffffffu, m[e], o));
+          ptx::named_sync<256>();  // red64 is free again
+          float* redf = reinterpret_cast<float*>(&red64[0][0]);
+          if (lane < T::CPR)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) redf[warp * D + 8 * c + e] = m[e];
+          ptx::named_sync<256>();
+          if (threadIdx.x < D) {
+            float mx = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx = fmaxf(mx, redf[i * D + threadIdx.x]);
+            // non-negative floats order like their bit patterns
+            atomicMax(v_amax + chan0 + threadIdx.x, __float_as_uint(mx));
+          }
+        }
+        // count this block done once every consumer's atomics are issued
+        ptx::named_sync<256>();
+        if (threadIdx.x == 0) ptx::red_release_add_gpu(sync + 1 + u, 1u);
+      } else {
+        // K: smoothing + per-block quantiser (channel means from the producer)
+        {
+          float m[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m[e] = s_side[slot0][8 * c + e];
+          take(0);
+          const float a = full_blk ? regs_absmax_sub<D, BF16, true>(rg, P.rows, m)
+                                   : regs_absmax_sub<D, BF16, false>(rg, P.rows, m);
+          const float amax = consumer_block_max(a, red, par);
+          codes(amax, m, k_codes, std::true_type{});
+          if (threadIdx.x == 0)
+            k_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+        }
+        // V: FP8 E4M3 codes with a per-channel scale
+        if constexpr (FP8) {
+          const float* side = s_side[(cidx + 1) % NS];  // V scale factors
+          float2 sv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sv[e] = make_float2(side[8 * c + 2 * e], side[8 * c + 2 * e + 1]);
+          take(1);
+          const int r0 = threadIdx.x / T::CPR;
+#pragma unroll
+          for (int i = 0; i < T::NIT; ++i) {
+            const int r = r0 + i * T::RS;
+            if (full_blk || r < P.rows) {
+              const float2 y0 = __fmul2_rn(In16<BF16>::to_float2(rg[i].x), sv[0]);
+              const float2 y1 = __fmul2_rn(In16<BF16>::to_float2(rg[i].y), sv[1]);
+              const float2 y2 = __fmul2_rn(In16<BF16>::to_float2(rg[i].z), sv[2]);
+              const float2 y3 = __fmul2_rn(In16<BF16>::to_float2(rg[i].w), sv[3]);
+              const uint32_t w0 = pack_e4m3x4(y0.x, y0.y, y1.x, y1.y);
+              const uint32_t w1 = pack_e4m3x4(y2.x, y2.y, y3.x, y3.y);
+              const long long row = P.row0 + (long long)r * P.row_stride;
+              *reinterpret_cast<uint2*>(v_codes + row * D + 8 * c) = make_uint2(w0, w1);
+            }
+          }
+        }
+      }
+      cidx += nt;
+    }
+    if (threadIdx.x == 0) {
+      s_consumed = cidx;
+      if (!finished) {  // left the loop on a failed wait
+        set_status(status, ST_TIMEOUT);
+        s_abort = 1;
+      }
+    }
+  }
+  __syncthreads();
+  // Teardown: copies issued but not consumed (only after a failed wait) must
+  // land before the CTA's shared memory goes away.
+  if (warp == 8 && lane == 0) {
+    for (int f = s_consumed; f < s_filled; ++f)
+      if (!ptx::mbar_wait(&full[f % NS], (f / NS) & 1)) break;
   }
 }
 
@@ -353,7 +937,41 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
                                   const void* v, int8_t* q_codes, float* q_scale,
                                   int8_t* k_codes, float* k_scale, float* k_mean,
                                   uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
-                                  uint32_t* v_amax, uint32_t* status, cudaStream_t st) {
+                                  uint32_t* v_amax, uint32_t* status, unsigned int* sync,
+                                  cudaStream_t st) {
+  const int U = grid.y, NB = grid.x;
+  const long long items = 2LL * U * NB;
+  // Dense: one persistent launch in an L2-friendly order (its work counter is
+  // 32-bit).  Variable-length batches, and any larger problem: two launches.
+  if (!L.varlen && items + 4096 < (1LL << 31)) {
+    using S = Stream<D>;
+    static int sms = 0;  // per template instance
+    if (sms == 0) {
+      int dev = 0;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      const cudaError_t e = cudaFuncSetAttribute(quant_stream_kernel<D, BF16, FP8>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)S::SMEM);
+      if (e != cudaSuccess) { sms = 0; return e; }
+    }
+    const long long cap = (long long)sms * S::CTAS_PER_SM;
+    const int blocks = (int)(items < cap ? items : cap);
+    // Items claimed but not yet finished: at most (ring slots + 1) per CTA.
+    // A lag of half that many groups of NB, plus one, keeps pass-2 waits rare
+    // while the re-read window (about lag heads of Q, K and codes) stays
+    // within L2 for long sequences.
+    long long lag = ((long long)blocks * (S::NS + 1) + 2LL * NB - 1) / (2LL * NB) + 1;
+#ifdef SAGE_QUANT_LAG
+    lag = SAGE_QUANT_LAG;
+#endif
+    if (lag > U) lag = U;
+    if (lag < 1) lag = 1;
+    quant_stream_kernel<D, BF16, FP8><<<blocks, S::THREADS, S::SMEM, st>>>(
+        L, U, (int)lag, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
+        k_sum, v_amax, status, sync);
+    return cudaGetLastError();
+  }
   quant_pass1_kernel<D, BF16, FP8>
       <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status);
   cudaError_t e = cudaGetLastError();
@@ -363,16 +981,19 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
   return cudaGetLastError();
 }
 
-// Runs both passes.  k_sum / v_amax must be zero on entry (the caller clears
-// them on the stream).  grid = (blocks per head or TBmax, B*H or H).
+// Runs both passes.  k_sum / v_amax and (dense) sync[0 .. B*H] must be zero on
+// entry (the caller clears them on the stream).  grid = (blocks per head or
+// TBmax, B*H or H).
 cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool fp8,
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
-                         uint32_t* v_amax, uint32_t* status, cudaStream_t st) {
+                         uint32_t* v_amax, uint32_t* status, unsigned int* sync,
+                         cudaStream_t st) {
 #define SAGE_Q(DD, BB, FF)                                                                    \
   return launch_quant_t<DD, BB, FF>(L, grid, q, k, v, q_codes, q_scale, k_codes, k_scale,    \
-                                    k_mean, v_codes, v_scale, k_sum, v_amax, status, st)
+                                    k_mean, v_codes, v_scale, k_sum, v_amax, status, sync,   \
+                                    st)
   if (D == 64) {
     if (bf16) { if (fp8) SAGE_Q(64, true, true); else SAGE_Q(64, true, false); }
     else { if (fp8) SAGE_Q(64, false, true); else SAGE_Q(64, false, false); }

@@ -29,30 +29,41 @@ def gpu_quantize_dense(q, k, v, pv_mode):
     return qz
 
 
+def assert_same(name: str, got: np.ndarray, want: np.ndarray) -> None:
+    """Bit-exact equality; on failure, report where and by how much."""
+    assert got.shape == want.shape, f"{name}: shape {got.shape} != {want.shape}"
+    if np.array_equal(got, want):
+        return
+    bad = np.argwhere(got != want)
+    head = [(tuple(int(i) for i in ix), got[tuple(ix)].item(), want[tuple(ix)].item())
+            for ix in bad[:8]]
+    raise AssertionError(f"{name}: {len(bad)} of {got.size} differ; first (index, got, want): {head}")
+
+
 def compare_quant_dense(qz_gpu, qz_ref, pv_mode):
     c = lambda t: t.cpu().numpy()
-    assert np.array_equal(c(qz_gpu.q_codes), qz_ref.q_codes), "q codes"
-    assert np.array_equal(c(qz_gpu.q_scale), qz_ref.q_delta), "q deltas"
-    assert np.array_equal(c(qz_gpu.k_mean), qz_ref.k_mean), "k mean"
-    assert np.array_equal(c(qz_gpu.k_scale), qz_ref.k_delta), "k deltas"
-    assert np.array_equal(c(qz_gpu.k_codes), qz_ref.k_codes), "k codes"
+    assert_same("q deltas", c(qz_gpu.q_scale), qz_ref.q_delta)
+    assert_same("q codes", c(qz_gpu.q_codes), qz_ref.q_codes)
+    assert_same("k mean", c(qz_gpu.k_mean), qz_ref.k_mean)
+    assert_same("k deltas", c(qz_gpu.k_scale), qz_ref.k_delta)
+    assert_same("k codes", c(qz_gpu.k_codes), qz_ref.k_codes)
     if pv_mode == "fp8":
-        assert np.array_equal(c(qz_gpu.v_scale), qz_ref.v_delta), "v deltas"
-        assert np.array_equal(c(qz_gpu.v_codes), qz_ref.v_codes), "v codes"
+        assert_same("v deltas", c(qz_gpu.v_scale), qz_ref.v_delta)
+        assert_same("v codes", c(qz_gpu.v_codes), qz_ref.v_codes)
 
 
 def compare_quant_varlen(qz_gpu, qz_ref, cu, pv_mode):
     """Varlen code arrays are [H, TBmax*128, D]; only the first TB blocks are written."""
     c = lambda t: t.cpu().numpy()
     TB = qz_ref.q_delta.shape[1]
-    assert np.array_equal(c(qz_gpu.q_codes)[:, :TB * 128], qz_ref.q_codes), "q codes"
-    assert np.array_equal(c(qz_gpu.q_scale)[:, :TB], qz_ref.q_delta), "q deltas"
-    assert np.array_equal(c(qz_gpu.k_mean), qz_ref.k_mean), "k mean"
-    assert np.array_equal(c(qz_gpu.k_scale)[:, :TB], qz_ref.k_delta), "k deltas"
-    assert np.array_equal(c(qz_gpu.k_codes)[:, :TB * 128], qz_ref.k_codes), "k codes"
+    assert_same("q deltas", c(qz_gpu.q_scale)[:, :TB], qz_ref.q_delta)
+    assert_same("q codes", c(qz_gpu.q_codes)[:, :TB * 128], qz_ref.q_codes)
+    assert_same("k mean", c(qz_gpu.k_mean), qz_ref.k_mean)
+    assert_same("k deltas", c(qz_gpu.k_scale)[:, :TB], qz_ref.k_delta)
+    assert_same("k codes", c(qz_gpu.k_codes)[:, :TB * 128], qz_ref.k_codes)
     if pv_mode == "fp8":
-        assert np.array_equal(c(qz_gpu.v_scale), qz_ref.v_delta), "v deltas"
-        assert np.array_equal(c(qz_gpu.v_codes), qz_ref.v_codes), "v codes"
+        assert_same("v deltas", c(qz_gpu.v_scale), qz_ref.v_delta)
+        assert_same("v codes", c(qz_gpu.v_codes), qz_ref.v_codes)
 
 
 def run_dense(q, k, v, causal, pv_mode, out_dtype=torch.float32, sm_scale=None):

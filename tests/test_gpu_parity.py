@@ -60,6 +60,16 @@ def test_quantize_bit_exact_full_workloads(name):
         U.compare_quant_dense(qz, ref, wl.pv_mode)
 
 
+@pytest.mark.parametrize("D,dtype,pv_mode", [(64, "bf16", "fp8"), (128, "fp16", "fp16")])
+def test_quantize_bit_exact_many_heads_ragged(D, dtype, pv_mode):
+    """Many heads of a long ragged sequence: the dense quantiser interleaves the
+    pass-1 blocks of later heads with the pass-2 blocks of earlier ones."""
+    q, k, v = W.make_dense(2, 20, 8000, D, dtype, bias_sigma=3.0, outlier_p=0.01,
+                           outlier_scale=20.0, seed=4242 + D)
+    qz = U.gpu_quantize_dense(q, k, v, pv_mode)
+    U.compare_quant_dense(qz, heads.quantize(q, k, v, None, pv_mode), pv_mode)
+
+
 def test_constant_k_channels_give_zero_codes():
     """K constant over tokens: the smoothed K is exactly zero (mean is exact)."""
     q, k, v = W.make_dense(1, 2, 333, 128, "fp16", bias_sigma=5.0, seed=7, k_const_over_tokens=True)
