@@ -205,7 +205,7 @@ def run_ours(args, rank, world, local):
 
         def stage2():
             api.attn_quantized(qz, v, causal=wl.causal, out=out, workspace=ws)
-        launches_per_step = 3
+        launches_per_step = 2  # quant_stream_kernel, attn_fwd_kernel
     else:
         T, H, D = q.shape
         out = torch.empty_like(q)
@@ -218,7 +218,7 @@ def run_ours(args, rank, world, local):
         def stage2():
             api.attn_fwd_varlen(q, k, v, cu, maxlen, causal=wl.causal, pv_mode=wl.pv_mode, out=out,
                                 workspace=ws)
-        launches_per_step = 4
+        launches_per_step = 4  # varlen_prep, quant_pass1, quant_pass2, attn_fwd
 
     def step():
         stage1()
