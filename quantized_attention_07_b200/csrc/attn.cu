@@ -505,27 +505,23 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
         }
       }
     } else {
-      // pass 1: row maximum (S re-read per chunk keeps registers for O32)
-      int smax = INT_MIN;
+      // S of the sub-tile in one TMEM round trip
+      uint32_t sv[SUB];
 #pragma unroll
-      for (int cc = 0; cc < SUB / 16; ++cc) {
-        uint32_t sv[16];
-        ptx::tmem_ld16(tS + 16 * cc, sv);
-        ptx::tmem_wait_ld();
-        smax = full_tile ? row_max<16>(sv, smax) : row_max_masked<16>(sv, smax, key0 + 16 * cc, limit);
-      }
+      for (int cc = 0; cc < SUB / 32; ++cc)
+        ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
+      ptx::tmem_wait_ld();
+      const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
+                                 : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
       const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
       m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
       alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
-      // pass 2: P^ = e4m3(448 p), four per TMEM column, written over S
+      // P^ = e4m3(448 p), four per TMEM column, written over S
 #pragma unroll
       for (int cc = 0; cc < SUB / 16; ++cc) {
-        uint32_t sv[16];
-        ptx::tmem_ld16(tS + 16 * cc, sv);
-        ptx::tmem_wait_ld();
         float pv[16];
-        rowsum += full_tile ? row_exp<false, 16>(sv, c, -m_new, key0 + 16 * cc, limit, pv)
-                            : row_exp<true, 16>(sv, c, -m_new, key0 + 16 * cc, limit, pv);
+        rowsum += full_tile ? row_exp<false, 16>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv)
+                            : row_exp<true, 16>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv);
         uint32_t packed[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -536,21 +532,23 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
         ptx::tmem_st4(tS + 4 * cc, packed);
       }
       if (i > 0) {
-        // two-level accumulation: O32 <- alpha_{i-1} O32 + Part_{i-1}
+        // two-level accumulation: O32 <- alpha_{i-1} O32 + Part_{i-1}, 64
+        // columns of the partial per TMEM round trip
         if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
         ptx::tc_fence_after();
         const float2 a2 = make_float2(alpha_prev, alpha_prev);
 #pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
-          uint32_t pv[16];
-          ptx::tmem_ld16(tO + 16 * cc, pv);
+        for (int cb = 0; cb < D / 64; ++cb) {
+          uint32_t pv[64];
+          ptx::tmem_ld32(tO + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+          ptx::tmem_ld32(tO + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 16; k += 2) {
-            const float2 x = __ffma2_rn(a2, make_float2(o32[16 * cc + k], o32[16 * cc + k + 1]),
+          for (int k = 0; k < 64; k += 2) {
+            const float2 x = __ffma2_rn(a2, make_float2(o32[64 * cb + k], o32[64 * cb + k + 1]),
                                         make_float2(__uint_as_float(pv[k]), __uint_as_float(pv[k + 1])));
-            o32[16 * cc + k] = x.x;
-            o32[16 * cc + k + 1] = x.y;
+            o32[64 * cb + k] = x.x;
+            o32[64 * cb + k + 1] = x.y;
           }
         }
       }
