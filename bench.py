@@ -194,7 +194,22 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
 
-    if not wl.varlen:
+    grouped = not wl.varlen and wl.kv_heads != wl.H
+    if grouped:
+        # grouped-query attention: the whole public call per step (K, V
+        # quantised over the key/value heads, Q over the query heads, then
+        # the attention kernel)
+        B, H, N, D = q.shape
+        out = torch.empty_like(q)
+        ws = sage.Workspace(sage.workspace_bytes_gqa(B, H, wl.kv_heads, N, D, wl.pv_mode), dev)
+
+        def stage1():
+            pass
+
+        def stage2():
+            api.attn_fwd(q, k, v, causal=wl.causal, pv_mode=wl.pv_mode, out=out, workspace=ws)
+        launches_per_step = 3  # quant_stream_kernel (K, V), quant_stream_kernel (Q), attn_fwd
+    elif not wl.varlen:
         B, H, N, D = q.shape
         qz = api.alloc_quantized(B, H, N, D, wl.pv_mode, dev)
         out = torch.empty_like(q)
@@ -316,6 +331,7 @@ def run_ours(args, rank, world, local):
         "dtype": "int8/fp8" if wl.pv_mode == "fp8" else "int8/fp16",
         "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D,
+                   "Hkv": wl.kv_heads,
                    "in_dtype": wl.dtype, "causal": wl.causal, "pv_mode": wl.pv_mode,
                    "seqlens": inp.seqlens if wl.varlen else None,
                    "l2": f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB of q,k,v > 126 MiB)"
@@ -354,13 +370,12 @@ def cpu_oracle_throughput(wl, inp, budget_rows: int, quant_heads: int, seed: int
     lens = inp.seqlens
     H = wl.H
     hs = min(quant_heads, H)
+    k_in, v_in = inp.k, inp.v
+    if not wl.varlen and wl.kv_heads != H:  # grouped-query: the oracle sees repeated K, V
+        k_in, v_in = heads.repeat_kv(k_in, H // wl.kv_heads), heads.repeat_kv(v_in, H // wl.kv_heads)
     # quantisation of `hs` heads (all sequences), timed
-    if wl.varlen:
-        sl = lambda x: x[:, :hs].contiguous()
-        qh, kh, vh = sl(inp.q), sl(inp.k), sl(inp.v)
-    else:
-        sl = lambda x: x[:, :hs].contiguous()
-        qh, kh, vh = sl(inp.q), sl(inp.k), sl(inp.v)
+    sl = lambda x: x[:, :hs].contiguous()
+    qh, kh, vh = sl(inp.q), sl(k_in), sl(v_in)
     t0 = time.perf_counter()
     qz = heads.quantize(qh, kh, vh, inp.cu_seqlens, wl.pv_mode)
     t_quant = time.perf_counter() - t0

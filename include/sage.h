@@ -126,6 +126,25 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
                             void* stream);
 
 /*
+ * Grouped-query variant: q and out are [B, H, N, D]; k and v are
+ * [B, Hkv, N, D] with H a multiple of Hkv, and query head h reads key/value
+ * head h / (H / Hkv) of its batch -- the grouping of the "sageattention in
+ * DeepSeek-VL2" page's attention code, which repeats each key/value head for
+ * H / Hkv consecutive query heads (repeat_kv) before calling attention.  The
+ * result equals sage_attn_fwd on the repeated k, v (K means, deltas and V
+ * scales are per key/value head, so repeating changes none of them) without
+ * materialising the repeat.
+ *   ws : at least sage_workspace_bytes_gqa(B, H, Hkv, N, D, pv_mode).
+ * Other arguments as sage_attn_fwd; Hkv = H is sage_attn_fwd.  An Hkv that is
+ * not a divisor of H returns SAGE_ERR_INVALID_ARG.
+ */
+size_t sage_workspace_bytes_gqa(int B, int H, int Hkv, int N, int D, int pv_mode);
+sage_status_t sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* out,
+                                int in_dt, int out_dt, int B, int H, int Hkv, int N, int D,
+                                int causal, float sm_scale, int pv_mode, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/*
  * Variable-length packed variant: `batch` sequences, sequence s occupying rows
  * cu_seqlens[s] .. cu_seqlens[s+1]-1 of the [T, H, D] tensors q, k, v, out.
  *   cu_seqlens  : DEVICE int32 [batch + 1], cu_seqlens[0] = 0, non-decreasing,

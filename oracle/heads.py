@@ -53,6 +53,21 @@ def _heads(x: torch.Tensor, cu: Optional[list[int]]):
                 yield s, h, np.ascontiguousarray(xf[cu[s]:cu[s + 1], h])
 
 
+def repeat_kv(x: torch.Tensor, groups: int) -> torch.Tensor:
+    """Grouped-query attention's head mapping, written out: [B, Hkv, N, D] ->
+    [B, Hkv*groups, N, D], query head h reading key/value head h // groups.
+
+    Follows the attention code on the "sageattention in DeepSeek-VL2" page,
+    which repeats every key/value head for `num_key_value_groups` consecutive
+    query heads (repeat_kv) before calling attention.
+    """
+    B, Hkv, N, D = x.shape
+    out = torch.empty((B, Hkv * groups, N, D), dtype=x.dtype)
+    for h in range(Hkv * groups):
+        out[:, h] = x[:, h // groups]
+    return out
+
+
 def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
              cu_seqlens: Optional[torch.Tensor] = None, pv_mode: str = "fp16") -> Quantized:
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]

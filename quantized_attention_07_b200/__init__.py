@@ -9,5 +9,5 @@ binding of that library.
 from .api import (  # noqa: F401
     BLOCK, PV_MODES, Quantized, SageError, Workspace, alloc_quantized, attn_fwd, attn_fwd_varlen,
     attn_quantized, qk_int8_tiles, quantize, quantize_varlen, sageattn, sync_status,
-    workspace_bytes, workspace_bytes_varlen,
+    workspace_bytes, workspace_bytes_gqa, workspace_bytes_varlen,
 )

@@ -117,6 +117,11 @@ def workspace_bytes(B: int, H: int, N: int, D: int, pv_mode: str = "fp16") -> in
     return int(_lib.load().sage_workspace_bytes(B, H, N, D, _pv(pv_mode)))
 
 
+def workspace_bytes_gqa(B: int, H: int, Hkv: int, N: int, D: int, pv_mode: str = "fp16") -> int:
+    """Workspace of attn_fwd with [B, H, N, D] queries over [B, Hkv, N, D] keys/values."""
+    return int(_lib.load().sage_workspace_bytes_gqa(B, H, Hkv, N, D, _pv(pv_mode)))
+
+
 def workspace_bytes_varlen(total_tokens: int, batch: int, H: int, D: int,
                            pv_mode: str = "fp16") -> int:
     return int(_lib.load().sage_workspace_bytes_varlen(total_tokens, batch, H, D, _pv(pv_mode)))
@@ -128,24 +133,39 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
              sm_scale: Optional[float] = None, pv_mode: str = "fp16",
              out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
              workspace: Optional[Workspace] = None) -> torch.Tensor:
-    """SageAttention forward over dense [B, H, N, D] fp16/bf16 tensors."""
+    """SageAttention forward over dense [B, H, N, D] fp16/bf16 tensors.
+
+    k and v may have fewer heads than q ([B, Hkv, N, D], H a multiple of Hkv):
+    grouped-query attention, query head h reading key/value head h // (H // Hkv).
+    """
     _need_cuda_contig(q, k, v)
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must share one [B, H, N, D] shape")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("q must be [B, H, N, D] and k, v one [B, Hkv, N, D] shape")
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    if (k.shape[0], k.shape[2], k.shape[3]) != (B, N, D) or Hkv < 1 or H % Hkv:
+        raise ValueError("k, v must be [B, Hkv, N, D] with Hkv dividing H")
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share one dtype")
-    B, H, N, D = q.shape
     od = out_dtype or q.dtype
     if out is None:
         out = torch.empty((B, H, N, D), dtype=od, device=q.device)
     _need_cuda_contig(out)
     mode = _pv(pv_mode)
-    ws = _workspace(q.device, workspace_bytes(B, H, N, D, pv_mode), workspace)
-    _check(_lib.load().sage_attn_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
-        _dtype_code(out.dtype, True), B, H, N, D, int(bool(causal)),
-        float(sm_scale) if sm_scale else 0.0, mode, ws.ptr, ws.nbytes, _stream(q.device)),
-        "sage_attn_fwd")
+    scale = float(sm_scale) if sm_scale else 0.0
+    lib = _lib.load()
+    if Hkv == H:
+        ws = _workspace(q.device, workspace_bytes(B, H, N, D, pv_mode), workspace)
+        _check(lib.sage_attn_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+            _dtype_code(out.dtype, True), B, H, N, D, int(bool(causal)), scale, mode, ws.ptr,
+            ws.nbytes, _stream(q.device)), "sage_attn_fwd")
+    else:
+        ws = _workspace(q.device, workspace_bytes_gqa(B, H, Hkv, N, D, pv_mode), workspace)
+        _check(lib.sage_attn_fwd_gqa(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+            _dtype_code(out.dtype, True), B, H, Hkv, N, D, int(bool(causal)), scale, mode,
+            ws.ptr, ws.nbytes, _stream(q.device)), "sage_attn_fwd_gqa")
     return out
 
 
@@ -315,6 +335,8 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, attn_mask=None,
     Arbitrary masks and dropout are not part of the method; passing them raises
     SageError(SAGE_ERR_UNSUPPORTED).  Non-contiguous inputs (e.g. the
     transpose(1, 2) views of a projection output) are made contiguous first.
+    k, v with fewer heads than q are grouped-query attention (no repeat_kv
+    needed).
     """
     if attn_mask is not None or dropout_p:
         raise SageError(2, "sageattn: attn_mask / dropout_p")

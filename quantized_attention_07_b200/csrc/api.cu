@@ -16,7 +16,7 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
-                         uint32_t* v_amax, uint32_t* status, unsigned int* sync,
+                         uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
                          cudaStream_t st);
 cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
                             const int32_t* tiles, int n, int32_t* out, uint32_t* status,
@@ -51,32 +51,39 @@ float kappa_of(float sm_scale, int D) {
 
 // Workspace layout.  Offsets in bytes from the workspace base.
 struct Layout {
-  size_t k_sum, v_amax, sync, blk_off, pair_off;       // scratch
+  size_t k_sum, v_amax, sync, sync_q, blk_off, pair_off;  // scratch
   size_t q_codes, k_codes, q_scale, k_scale, k_mean;   // quantised operands
   size_t v_codes, v_scale;
   size_t scratch_end, total;
 };
 
-Layout dense_layout(int B, int H, int N, int D, bool fp8) {
-  const size_t BH = (size_t)B * H, NB = ((size_t)N + BLK - 1) / BLK, NP = NB * BLK;
+// Dense layout for H query heads and Hkv key/value heads per batch (Hkv = H
+// without grouping).  sync: work counter + one completion counter per
+// key/value head for the launch that quantises K (and Q when Hkv = H);
+// sync_q: the work counter of the separate Q launch when Hkv < H.
+Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv) {
+  const size_t BH = (size_t)B * H, BK = (size_t)B * Hkv, NB = ((size_t)N + BLK - 1) / BLK,
+               NP = NB * BLK;
   Layout L{};
   size_t o = kHeader;
-  L.k_sum = o; o += al(BH * D * 8);
-  L.v_amax = o; o += al(BH * D * 4);
-  L.sync = o; o += al((BH + 1) * 4);
+  L.k_sum = o; o += al(BK * D * 8);
+  L.v_amax = o; o += al(BK * D * 4);
+  L.sync = o; o += al((BK + 1) * 4);
+  L.sync_q = o; o += al(4);
   L.scratch_end = o;
   L.q_codes = o; o += al(BH * NP * D);
-  L.k_codes = o; o += al(BH * NP * D);
+  L.k_codes = o; o += al(BK * NP * D);
   L.q_scale = o; o += al(BH * NB * 4);
-  L.k_scale = o; o += al(BH * NB * 4);
-  L.k_mean = o; o += al(BH * D * 4);
+  L.k_scale = o; o += al(BK * NB * 4);
+  L.k_mean = o; o += al(BK * D * 4);
   if (fp8) {
-    L.v_codes = o; o += al(BH * (size_t)N * D);
-    L.v_scale = o; o += al(BH * D * 4);
+    L.v_codes = o; o += al(BK * (size_t)N * D);
+    L.v_scale = o; o += al(BK * D * 4);
   }
   L.total = o;
   return L;
 }
+Layout dense_layout(int B, int H, int N, int D, bool fp8) { return dense_layout(B, H, N, D, fp8, H); }
 
 long long tb_max(long long T, long long batch) { return (T + (BLK - 1) * batch) / BLK; }
 long long pair_max(long long T, long long batch) { return (T + (2 * BLK - 1) * batch) / (2 * BLK); }
@@ -109,6 +116,8 @@ bool dense_args_ok(int B, int H, int N, int D, int pv_mode) {
          (long long)B * H <= 65535 && (pv_mode == SAGE_PV_FP16 || pv_mode == SAGE_PV_FP8);
 }
 
+bool gqa_heads_ok(int H, int Hkv) { return Hkv >= 1 && Hkv <= H && H % Hkv == 0; }
+
 bool varlen_args_ok(int T, int batch, int max_seqlen, int H, int D, int pv_mode) {
   return T >= 0 && batch >= 1 && max_seqlen >= 0 && max_seqlen <= kMaxN && H >= 1 &&
          H <= 65535 && (D == 64 || D == 128) &&
@@ -127,7 +136,7 @@ sage_status_t clear_scratch(void* ws, const Layout& L, bool fp8, cudaStream_t st
   cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, L.k_sum), 0, L.v_amax - L.k_sum, st);
   if (e == cudaSuccess && fp8)
     e = cudaMemsetAsync(at<uint8_t>(ws, L.v_amax), 0, L.sync - L.v_amax, st);
-  if (e == cudaSuccess) {
+  if (e == cudaSuccess) {  // work / completion counters (dense: both launches')
     const size_t sync_end = L.blk_off ? L.blk_off : L.scratch_end;
     e = cudaMemsetAsync(at<uint8_t>(ws, L.sync), 0, sync_end - L.sync, st);
   }
@@ -135,22 +144,35 @@ sage_status_t clear_scratch(void* ws, const Layout& L, bool fp8, cudaStream_t st
 }
 
 // Dense stage 1 into explicit buffers.
+// Hkv < H (grouped-query attention): K (and V) are quantised over the B*Hkv
+// key/value heads and Q over the B*H query heads, in two launches.
 sage_status_t quantize_dense(const void* q, const void* k, const void* v, int in_dt, int B,
                              int H, int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
                              int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
-                             float* v_scale, void* ws, const Layout& L, cudaStream_t st) {
+                             float* v_scale, void* ws, const Layout& L, cudaStream_t st,
+                             int Hkv) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   sage_status_t r = clear_scratch(ws, L, fp8, st);
   if (r != SAGE_OK) return r;
   SeqLayout S{};
   S.varlen = 0;
   S.N = N;
-  S.H = H;
-  const dim3 grid((N + BLK - 1) / BLK, B * H);
-  cudaError_t e = launch_quant(S, grid, D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
-                               k_codes, k_scale, k_mean, v_codes, v_scale,
+  S.H = Hkv;
+  const unsigned NB = (unsigned)((N + BLK - 1) / BLK);
+  const bool grouped = Hkv != H;
+  cudaError_t e = launch_quant(S, dim3(NB, (unsigned)(B * Hkv)), D, in_dt == SAGE_BF16, fp8, q,
+                               k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
                                at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                               at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync), st);
+                               at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync),
+                               grouped ? QUANT_KV : QUANT_Q | QUANT_KV, st);
+  if (e == cudaSuccess && grouped) {
+    S.H = H;
+    e = launch_quant(S, dim3(NB, (unsigned)(B * H)), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes,
+                     q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
+                     at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
+                     at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync_q), QUANT_Q, st);
+  }
+  if (e == cudaErrorNotSupported) return SAGE_ERR_UNSUPPORTED;
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
 
@@ -158,10 +180,11 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
                          const float* k_scale, const void* v, const uint8_t* v_codes,
                          const float* v_scale, void* out, int v_dt, int out_dt, int B, int H,
                          int N, int D, int causal, float sm_scale, int pv_mode, void* ws,
-                         cudaStream_t st) {
+                         cudaStream_t st, int Hkv) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   AttnLaunch A{};
   A.p.H = H;
+  A.p.Hkv = Hkv;
   A.p.N = N;
   A.p.BH = B * H;
   A.p.NB = (N + BLK - 1) / BLK;
@@ -183,6 +206,7 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
   A.v = fp8 ? static_cast<const void*>(v_codes) : v;
   A.code_rows = A.p.NB * BLK;
   A.code_z = B * H;
+  A.code_z_kv = B * Hkv;
   A.T = 0;
   A.grid = dim3((unsigned)((long long)B * H * A.p.NPAIR), 1, 1);
   cudaError_t e = launch_attn(A, st);
@@ -261,7 +285,7 @@ sage_status_t sage_quantize(const void* q, const void* k, const void* v, int in_
   const Layout L = dense_layout(B, H, N, D, fp8);
   if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
   return quantize_dense(q, k, v, in_dt, B, H, N, D, pv_mode, q_codes, q_scale, k_codes, k_scale,
-                        k_mean, v_codes, v_scale, ws, L, as_stream(stream));
+                        k_mean, v_codes, v_scale, ws, L, as_stream(stream), H);
 }
 
 sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
@@ -280,31 +304,53 @@ sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
     return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
   return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
-                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream));
+                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), H);
 }
 
-sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int in_dt,
-                            int out_dt, int B, int H, int N, int D, int causal, float sm_scale,
-                            int pv_mode, void* ws, size_t ws_bytes, void* stream) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
-      !std::isfinite(sm_scale))
+// Whole dense path for H query heads over Hkv key/value heads per batch.
+static sage_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* out,
+                                    int in_dt, int out_dt, int B, int H, int Hkv, int N, int D,
+                                    int causal, float sm_scale, int pv_mode, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !in_dtype_ok(in_dt) ||
+      !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
     return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
-  const Layout L = dense_layout(B, H, N, D, fp8);
+  const Layout L = dense_layout(B, H, N, D, fp8, Hkv);
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   sage_status_t r = quantize_dense(
       q, k, v, in_dt, B, H, N, D, pv_mode, at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
       at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
       fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr, fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L,
-      st);
+      st, Hkv);
   if (r != SAGE_OK) return r;
   return attn_dense(at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale), at<int8_t>(ws, L.k_codes),
                     at<float>(ws, L.k_scale), v, fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
                     fp8 ? at<float>(ws, L.v_scale) : nullptr, out, in_dt, out_dt, B, H, N, D,
-                    causal, sm_scale, pv_mode, ws, st);
+                    causal, sm_scale, pv_mode, ws, st, Hkv);
+}
+
+sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int in_dt,
+                            int out_dt, int B, int H, int N, int D, int causal, float sm_scale,
+                            int pv_mode, void* ws, size_t ws_bytes, void* stream) {
+  return attn_fwd_dense(q, k, v, out, in_dt, out_dt, B, H, H, N, D, causal, sm_scale, pv_mode, ws,
+                        ws_bytes, stream);
+}
+
+size_t sage_workspace_bytes_gqa(int B, int H, int Hkv, int N, int D, int pv_mode) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv)) return 0;
+  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv).total;
+}
+
+sage_status_t sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* out, int in_dt,
+                                int out_dt, int B, int H, int Hkv, int N, int D, int causal,
+                                float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return attn_fwd_dense(q, k, v, out, in_dt, out_dt, B, H, Hkv, N, D, causal, sm_scale, pv_mode,
+                        ws, ws_bytes, stream);
 }
 
 static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, int in_dt,
@@ -331,7 +377,7 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
   e = launch_quant(S, dim3((unsigned)TB, H), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
                    k_codes, k_scale, k_mean, v_codes, v_scale,
                    at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                   at<uint32_t>(ws, 0), nullptr, st);
+                   at<uint32_t>(ws, 0), nullptr, QUANT_Q | QUANT_KV, st);
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
 
@@ -404,6 +450,8 @@ sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, 
   A.v = fp8 ? static_cast<const void*>(at<uint8_t>(ws, L.v_codes)) : v;
   A.code_rows = (int)(TB * BLK);
   A.code_z = H;
+  A.code_z_kv = H;
+  A.p.Hkv = H;
   A.T = total_tokens;
   A.grid = dim3((unsigned)PM, H, 1);
   cudaError_t e = launch_attn(A, st);

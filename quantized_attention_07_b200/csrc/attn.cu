@@ -123,7 +123,8 @@ struct Work {
   int valid;
   int n;                 // sequence length (queries = keys)
   int pair;              // query tile pair index within the sequence
-  int code_z;            // z coordinate of this head in the Q^/K^ code maps
+  int code_z;            // z coordinate of this query head in the Q^ code map
+  int k_z;               // z coordinate of its key/value head in the K^ code map
   int q_y0;              // y coordinate of query tile 0 in the code map
   int k_y0;              // y coordinate of key tile 0 in the code map
   int v_y0, v_z0;        // TMA coordinates of V tile 0 (x = column)
@@ -151,17 +152,22 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
       pair = idx % p.NPAIR;
     }
     n = p.N;
+    // grouped-query attention: query head h of batch b reads key/value head
+    // h / (H / Hkv) of the same batch (the repeat_kv grouping)
+    const int b = bh / p.H, hq = bh - b * p.H;
+    const int bkv = b * p.Hkv + hq / (p.H / p.Hkv);
     w.code_z = bh;
+    w.k_z = bkv;
     w.q_y0 = pair * 2 * BLK;
     w.k_y0 = 0;
     w.v_y0 = 0;
-    w.v_z0 = bh;
+    w.v_z0 = bkv;
     w.v_tok_on_z = 0;
     w.qs_idx0 = (long long)bh * p.NB + 2 * pair;
-    w.ks_idx0 = (long long)bh * p.NB;
+    w.ks_idx0 = (long long)bkv * p.NB;
     w.out_row0 = (long long)bh * p.N;
     w.out_stride = 1;
-    w.vs_idx = bh;
+    w.vs_idx = bkv;
   } else {
     const int item = blockIdx.x;
     const int h = blockIdx.y;
@@ -174,6 +180,7 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
     pair = npairs - 1 - (item - __ldg(p.pair_off + s));  // diagonal-heavy pairs first
     const int blk0 = __ldg(p.blk_off + s);
     w.code_z = h;
+    w.k_z = h;
     w.q_y0 = (blk0 + 2 * pair) * BLK;
     w.k_y0 = blk0 * BLK;
     w.v_y0 = h;
@@ -221,7 +228,7 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
     if (j >= C::NS && !wait_bar(B, &B->kv_empty[s], ((j / C::NS) - 1) & 1, status, true)) break;
     if (ptx::elect_one()) {
       ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT);
-      ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.code_z);
+      ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
       ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
       uint8_t* dst = sV + s * C::VT;
       const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
@@ -800,8 +807,8 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
   const CUtensorMapSwizzle cs = swz_for(D);
   if (!make_map3(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.q_codes, D, L.code_rows, L.code_z, D,
                  (uint64_t)D * L.code_rows, D, BLK, 1, cs) ||
-      !make_map3(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.k_codes, D, L.code_rows, L.code_z, D,
-                 (uint64_t)D * L.code_rows, D, BLK, 1, cs))
+      !make_map3(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.k_codes, D, L.code_rows, L.code_z_kv,
+                 D, (uint64_t)D * L.code_rows, D, BLK, 1, cs))
     return cudaErrorInvalidValue;
   const int esz = PV8 ? 1 : 2;
   const CUtensorMapDataType vdt = PV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
@@ -811,7 +818,7 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
   const CUtensorMapSwizzle vs = swz_for(vbox0 * esz);
   bool okv;
   if (!L.p.varlen)
-    okv = make_map3(&tv, vdt, esz, L.v, D, L.p.N, L.p.BH, (uint64_t)D * esz,
+    okv = make_map3(&tv, vdt, esz, L.v, D, L.p.N, L.code_z_kv, (uint64_t)D * esz,
                     (uint64_t)D * esz * L.p.N, vbox0, BLK, 1, vs);
   else
     okv = make_map3(&tv, vdt, esz, L.v, D, L.p.H, L.T, (uint64_t)D * esz,

@@ -6,7 +6,8 @@
 namespace sage {
 
 struct AttnParams {
-  int H, N, BH;          // dense: N, BH = B*H
+  int H, N, BH;          // dense: N, BH = B*H (query heads)
+  int Hkv;               // dense: key/value heads (H is a multiple; query head h reads h / (H/Hkv))
   int NB;                // dense: key blocks per head = ceil(N/128)
   int NPAIR;             // dense: query tile pairs per head = ceil(N/256)
   int causal;
@@ -33,7 +34,8 @@ struct AttnLaunch {
   const int8_t* k_codes;
   const void* v;         // 16-bit V (FP16 mode) or E4M3 codes (FP8 mode)
   int code_rows;         // rows per z-slice of the code arrays (NP or TBmax*128)
-  int code_z;            // BH (dense) or H (varlen)
+  int code_z;            // Q^ z-slices: BH (dense) or H (varlen)
+  int code_z_kv;         // K^ (and dense V) z-slices: B*Hkv (dense) or H (varlen)
   int T;                 // varlen tokens
   dim3 grid;
 };

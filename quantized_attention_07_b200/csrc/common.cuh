@@ -39,6 +39,10 @@ struct VarlenMeta {
 
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t bits) { atomicOr(st, bits); }
 
+// Tensors a quantisation launch covers (launch_quant's `parts`).
+constexpr int QUANT_Q = 1;
+constexpr int QUANT_KV = 2;
+
 // Binary search: the s with off[s] <= x < off[s+1] (off non-decreasing, off[0] = 0).
 __device__ __forceinline__ int find_segment(const int32_t* off, int n, int x) {
   int lo = 0, hi = n;  // answer in [lo, hi)

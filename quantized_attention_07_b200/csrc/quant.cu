@@ -413,9 +413,29 @@ struct Stream {
   static constexpr int CTAS_PER_SM = 2;
 };
 
-template <int N>
-__device__ __forceinline__ int tensors_of(int pass) {
-  return pass == 1 ? N : N - 1;  // p1: Q, K (, V);  p2: K (, V)
+// What a launch quantises: Q, K (with V for FP8 P.V), or both.  Grouped-
+// query attention quantises Q over the query heads and K, V over the key /
+// value heads in two launches.
+enum Parts { PART_Q = 1, PART_KV = 2 };
+
+// Slabs of one work item: pass 1 = (Q,) (K, V), pass 2 = K (, V).
+__device__ __forceinline__ int tensors_of(int pass, int parts, bool fp8) {
+  const int nkv = fp8 ? 2 : 1;
+  if (pass == 2) return nkv;
+  return ((parts & PART_Q) ? 1 : 0) + ((parts & PART_KV) ? nkv : 0);
+}
+
+// Work item x -> (pass, unit, block).  Without K there is no pass 2 and the
+// items are simply the blocks in order.
+__device__ __forceinline__ void item_of(int x, int NB, int U, int lag, int parts, int& pass,
+                                        int& u, int& b) {
+  if (parts & PART_KV) {
+    fused_item(x, NB, U, lag, pass, u, b);
+  } else {
+    pass = 1;
+    u = x / NB;
+    b = x - u * NB;
+  }
 }
 
 // 1.5 * 2^23: for |y| < 2^22, the fp32 sum y + kMagic is kMagic + rint(y)
@@ -580,15 +600,15 @@ __device__ __forceinline__ void release_slot(uint64_t* empty) {
 // sync[0]: work counter; sync[1 + u]: pass-1 blocks of head u completed.
 template <int D, bool BF16, bool FP8>
 __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) quant_stream_kernel(
-    SeqLayout L, int U, int lag, const void* __restrict__ q, const void* __restrict__ k,
-    const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
-    int8_t* __restrict__ k_codes, float* __restrict__ k_scale, float* __restrict__ k_mean,
-    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale, unsigned long long* k_sum,
-    uint32_t* v_amax, uint32_t* status, unsigned int* sync) {
+    SeqLayout L, int U, int lag, int parts, const void* __restrict__ q,
+    const void* __restrict__ k, const void* __restrict__ v, int8_t* __restrict__ q_codes,
+    float* __restrict__ q_scale, int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
+    float* __restrict__ k_mean, uint8_t* __restrict__ v_codes, float* __restrict__ v_scale,
+    unsigned long long* k_sum, uint32_t* v_amax, uint32_t* status, unsigned int* sync) {
   using S = Stream<D>;
   using T = Tile<D>;
   constexpr int NS = S::NS;
-  constexpr int NT = FP8 ? 3 : 2;
+  const bool has_q = (parts & PART_Q) != 0, has_kv = (parts & PART_KV) != 0;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full[NS], empty[NS];
   __shared__ int info[NS];
@@ -602,7 +622,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
   __shared__ int s_abort, s_filled, s_consumed;
 
   const int NB = (L.N + BLK - 1) / BLK;
-  const int total = 2 * U * NB;
+  const int total = (has_kv ? 2 : 1) * U * NB;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -626,7 +646,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
       x = __shfl_sync(0xffffffffu, x, 0);
       const bool end = x >= total;
       int pass = 0, u = 0, b = 0;
-      if (!end) fused_item(x, NB, U, lag, pass, u, b);
+      if (!end) item_of(x, NB, U, lag, parts, pass, u, b);
       const unsigned target = (unsigned)NB;
       if (!end && pass == 2 && lane == 0) {
         const uint32_t* done = sync + 1 + u;
@@ -643,7 +663,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
         }
       }
       __syncwarp();
-      const int nt = end ? 1 : tensors_of<NT>(pass);
+      const int nt = end ? 1 : tensors_of(pass, parts, FP8);
       const long long row0 = (long long)u * L.N + (long long)b * BLK;
       const int rows = end ? 0 : min(BLK, L.N - b * BLK);
       bool ok = true;
@@ -654,8 +674,8 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
           ok = __shfl_sync(0xffffffffu, ok, 0);
         }
         if (!ok) break;
-        // tensor t of this item: p1 = (Q, K, V), p2 = (K, V)
-        const int which = pass == 1 ? t : t + 1;
+        // tensor t of this item (0 = Q, 1 = K, 2 = V)
+        const int which = (pass == 1 && has_q) ? t : t + 1;
         if (lane == 0) {
           info[slot] = end ? -1 : x;
           if (!end) {
@@ -719,8 +739,8 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
         break;
       }
       int pass, u, b;
-      fused_item(x, NB, U, lag, pass, u, b);
-      const int nt = tensors_of<NT>(pass);
+      item_of(x, NB, U, lag, parts, pass, u, b);
+      const int nt = tensors_of(pass, parts, FP8);
       for (int t = 1; t < nt; ++t) ok = ptx::mbar_wait(&full[(cidx + t) % NS], ((cidx + t) / NS) & 1) && ok;
       ok = ptx::named_all<256>(ok);
       if (!ok) break;
@@ -747,8 +767,9 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
       };
 
       if (pass == 1) {
+        const int tk = has_q ? 1 : 0;  // slab index of K (V follows it)
         // Q: per-block quantiser
-        {
+        if (has_q) {
           take(0);
           const float amax = consumer_block_max(regs_absmax<D, BF16>(rg), red, par);
           codes(amax, zero8, q_codes, std::false_type{});
@@ -756,8 +777,8 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
             q_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
         }
         // K: exact fixed-point channel sums
-        {
-          take(1);
+        if (has_kv) {
+          take(tk);
           float2 hi[4], fr[4];
           uint32_t absbits;
           regs_fixed_sums<D, BF16>(rg, hi, fr, absbits);
@@ -797,8 +818,8 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
           }
         }
         // V: per-channel max|v| (FP8 P.V only)
-        if constexpr (FP8) {
-          take(2);
+        if (FP8 && has_kv) {
+          take(tk + 1);
           uint32_t m2[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
           for (int i = 0; i < T::NIT; ++i) {
@@ -833,8 +854,10 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
           }
         }
         // count this block done once every consumer's atomics are issued
-        ptx::named_sync<256>();
-        if (threadIdx.x == 0) ptx::red_release_add_gpu(sync + 1 + u, 1u);
+        if (has_kv) {
+          ptx::named_sync<256>();
+          if (threadIdx.x == 0) ptx::red_release_add_gpu(sync + 1 + u, 1u);
+        }
       } else {
         // K: smoothing + per-block quantiser (channel means from the producer)
         {
@@ -938,11 +961,12 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
                                   int8_t* k_codes, float* k_scale, float* k_mean,
                                   uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                                   uint32_t* v_amax, uint32_t* status, unsigned int* sync,
-                                  cudaStream_t st) {
+                                  int parts, cudaStream_t st) {
   const int U = grid.y, NB = grid.x;
-  const long long items = 2LL * U * NB;
+  const long long items = ((parts & PART_KV) ? 2LL : 1LL) * U * NB;
   // Dense: one persistent launch in an L2-friendly order (its work counter is
-  // 32-bit).  Variable-length batches, and any larger problem: two launches.
+  // 32-bit).  Variable-length batches, and any larger problem: two launches,
+  // which handle Q and K (, V) together only.
   if (!L.varlen && items + 4096 < (1LL << 31)) {
     using S = Stream<D>;
     static int sms = 0;  // per template instance
@@ -968,10 +992,11 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
     if (lag > U) lag = U;
     if (lag < 1) lag = 1;
     quant_stream_kernel<D, BF16, FP8><<<blocks, S::THREADS, S::SMEM, st>>>(
-        L, U, (int)lag, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
-        k_sum, v_amax, status, sync);
+        L, U, (int)lag, parts, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes,
+        v_scale, k_sum, v_amax, status, sync);
     return cudaGetLastError();
   }
+  if (parts != (PART_Q | PART_KV)) return cudaErrorNotSupported;
   quant_pass1_kernel<D, BF16, FP8>
       <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status);
   cudaError_t e = cudaGetLastError();
@@ -981,19 +1006,21 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
   return cudaGetLastError();
 }
 
-// Runs both passes.  k_sum / v_amax and (dense) sync[0 .. B*H] must be zero on
-// entry (the caller clears them on the stream).  grid = (blocks per head or
-// TBmax, B*H or H).
+// Runs both passes.  k_sum / v_amax and (dense) sync[0 .. units] must be zero
+// on entry (the caller clears them on the stream).  grid = (blocks per head or
+// TBmax, units = B*H or H).  parts: QUANT_Q and/or QUANT_KV (both unless the
+// query and key/value heads differ).
 cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool fp8,
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
-                         uint32_t* v_amax, uint32_t* status, unsigned int* sync,
+                         uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
                          cudaStream_t st) {
+  static_assert(QUANT_Q == PART_Q && QUANT_KV == PART_KV, "part flags");
 #define SAGE_Q(DD, BB, FF)                                                                    \
   return launch_quant_t<DD, BB, FF>(L, grid, q, k, v, q_codes, q_scale, k_codes, k_scale,    \
                                     k_mean, v_codes, v_scale, k_sum, v_amax, status, sync,   \
-                                    st)
+                                    parts, st)
   if (D == 64) {
     if (bf16) { if (fp8) SAGE_Q(64, true, true); else SAGE_Q(64, true, false); }
     else { if (fp8) SAGE_Q(64, false, true); else SAGE_Q(64, false, false); }

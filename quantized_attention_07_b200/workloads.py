@@ -20,6 +20,8 @@ Recipe (per workload):
     picks entries that are multiplied by a factor (after the bias is added).
   * varlen: sequence lengths are drawn uniformly (inclusive) from a range, and
     ``cu_seqlens`` is their prefix sum; the packed layout is [T, H, D].
+  * grouped-query attention (Hkv < H): Q, K, V are drawn for H heads as above
+    and K, V keep their first Hkv heads ([B, Hkv, N, D]).
 """
 from __future__ import annotations
 
@@ -50,6 +52,11 @@ class Workload:
     len_lo: int = 0
     len_hi: int = 0
     seed: int = 0
+    Hkv: int = 0                # key/value heads (grouped-query attention); 0: = H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
 
     @property
     def sm_scale(self) -> float:
@@ -72,6 +79,10 @@ WORKLOADS = {
     "varlen_8seq": Workload("varlen_8seq", B=1, H=32, N=8192, D=128, dtype="bf16", causal=True,
                             pv_mode="fp8", bias_sigma=3.0, varlen=True, n_seqs=8, len_lo=512,
                             len_hi=8192, seed=20260005),
+    # LLM prefill with grouped-query attention (32 query heads over 8 key/value
+    # heads, the repeat_kv layout of the DeepSeek-VL2 page's attention code)
+    "llm_gqa_8k": Workload("llm_gqa_8k", B=1, H=32, N=8192, D=128, dtype="bf16", causal=True,
+                           pv_mode="fp16", bias_sigma=3.0, seed=20260006, Hkv=8),
 }
 
 
@@ -147,6 +158,8 @@ def make_inputs(wl: Workload) -> Inputs:
         return Inputs(q, k, v, cu, wl)
     q, k, v = make_dense(wl.B, wl.H, wl.N, wl.D, wl.dtype, wl.bias_sigma, wl.outlier_p,
                          wl.outlier_scale, seed=wl.seed)
+    if wl.kv_heads != wl.H:
+        k, v = k[:, :wl.kv_heads].contiguous(), v[:, :wl.kv_heads].contiguous()
     return Inputs(q, k, v, None, wl)
 
 

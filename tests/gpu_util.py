@@ -102,11 +102,16 @@ def cosine(a: np.ndarray, b: np.ndarray) -> float:
 def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
                          ref_cos_bar=0.999):
     """GPU fp32 output vs the oracle's emulation (max-abs tolerance) and the fp64
-    reference (cosine).  Also checks a 16-bit output run.  Returns a stats dict."""
+    reference (cosine).  Also checks a 16-bit output run.  Returns a stats dict.
+    Dense k, v with fewer heads than q run grouped-query attention on the GPU;
+    the oracle sees them repeated (its repeat_kv)."""
     D = q.shape[-1]
     if cu is None:
         out32 = run_dense(q, k, v, causal, pv_mode, torch.float32, sm_scale)
         out16 = run_dense(q, k, v, causal, pv_mode, q.dtype, sm_scale)
+        if k.shape[1] != q.shape[1]:
+            g = q.shape[1] // k.shape[1]
+            k, v = heads.repeat_kv(k, g), heads.repeat_kv(v, g)
     else:
         out32 = run_varlen(q, k, v, cu, causal, pv_mode, torch.float32, sm_scale)
         out16 = run_varlen(q, k, v, cu, causal, pv_mode, q.dtype, sm_scale)

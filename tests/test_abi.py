@@ -103,3 +103,22 @@ def test_varlen_and_stage_validation(lib):
     t = (ctypes.c_int32 * 3)(0, 5, 0)   # tile row out of range for NP = 256
     assert lib.sage_qk_int8_tiles(FAKE, FAKE, 1, 256, 64, ctypes.cast(t, ctypes.c_void_p), 1,
                                   FAKE, FAKE, 1 << 20, None) == 1
+
+
+def test_grouped_query_sizes_and_validation(lib):
+    B, H, N, D = 1, 8, 1024, 128
+    full = lib.sage_workspace_bytes(B, H, N, D, 1)
+    assert lib.sage_workspace_bytes_gqa(B, H, H, N, D, 1) == full   # Hkv = H: the plain layout
+    g4 = lib.sage_workspace_bytes_gqa(B, H, 2, N, D, 1)
+    # K codes and FP8 V codes shrink with the key/value heads; Q codes do not
+    assert full - g4 >= (H - 2) * N * D * 2 and g4 > B * H * N * D
+    for hkv in (0, 3, 16, -1):                                    # must divide H, 1 <= Hkv <= H
+        assert lib.sage_workspace_bytes_gqa(B, H, hkv, N, D, 0) == 0
+    f = lib.sage_attn_fwd_gqa
+    args = [FAKE, FAKE, FAKE, FAKE, 0, 0, 1, 8, 2, 256, 64, 0, 0.0, 0, FAKE, 1 << 40, None]
+    bad = list(args); bad[8] = 3
+    assert f(*bad) == 1
+    bad = list(args); bad[10] = 96
+    assert f(*bad) == 1
+    small = list(args); small[15] = lib.sage_workspace_bytes_gqa(1, 8, 2, 256, 64, 0) - 1
+    assert f(*small) == 3

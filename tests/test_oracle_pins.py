@@ -410,3 +410,29 @@ def test_emulation_rescale_threshold_changes_rounding_only(causal):
     ref = oracle.attn_ref_rows(q, k, v, float(np.float32(sm)), causal, np.arange(n))
     assert np.abs(outs[8.0] - ref).max() <= bound
     assert not np.array_equal(outs[0.0], outs[8.0])   # the threshold is in effect
+
+
+# ------------------------------------------------------ grouped-query heads --
+
+def test_repeat_kv_matches_repeat_interleave():
+    """The oracle's head mapping equals the library routine it restates."""
+    x = torch.randn(2, 3, 5, 4, generator=torch.Generator().manual_seed(3))
+    for g in (1, 2, 4):
+        assert torch.equal(heads.repeat_kv(x, g), torch.repeat_interleave(x, g, dim=1))
+
+
+def test_grouped_reference_uses_the_kv_head_of_each_group():
+    """Brute force: with each key/value head filled with its own constant value
+    vector, every query head's output is the value of key/value head h // g."""
+    B, Hkv, g, N, D = 1, 3, 2, 7, 4
+    gen = torch.Generator().manual_seed(5)
+    q = torch.randn(B, Hkv * g, N, D, generator=gen)
+    k = torch.randn(B, Hkv, N, D, generator=gen)
+    v = torch.zeros(B, Hkv, N, D)
+    for h in range(Hkv):
+        v[:, h] = float(h + 1)  # softmax weights sum to 1: output = h + 1
+    kr, vr = heads.repeat_kv(k, g), heads.repeat_kv(v, g)
+    for hq in range(Hkv * g):
+        out = oracle.attn_ref_rows(q[0, hq].numpy(), kr[0, hq].numpy(), vr[0, hq].numpy(),
+                                   oracle.default_sm_scale(D), False, np.arange(N))
+        assert np.allclose(out, hq // g + 1.0, atol=1e-12)
