@@ -258,6 +258,23 @@ sage_status_t sage_qk_int8_tiles(const int8_t* q_codes, const int8_t* k_codes, i
                                  void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Full-precision attention rows, the reference of the accuracy-driven choice
+ * between 16-bit and FP8 P.V ("SageAttention v1/v2/v2++/v3 overview",
+ * SageAttention v1: a faster variant serves a layer only where its cosine
+ * similarity to full-precision attention exceeds 99.8 %).
+ *   q : [B, H, N, D], k, v : [B, Hkv, N, D] (Hkv divides H; query head h
+ *       reads key/value head h / (H / Hkv)), 16-bit of type in_dt, DEVICE.
+ *   rows : DEVICE int32 [n_rows][3] = (b, h, i) query rows to evaluate.
+ *   out  : DEVICE fp32 [n_rows][D], softmax(sm_scale q_i K^T) V in fp32
+ *          (causal: keys j <= i); a row outside the input gets NaN.
+ * No quantisation: this is the plain definition, for calibration and checks,
+ * not a hot path.  sm_scale <= 0 selects 1/sqrt(D).
+ */
+sage_status_t sage_attn_ref_rows(const void* q, const void* k, const void* v, int in_dt, int B,
+                                 int H, int Hkv, int N, int D, int causal, float sm_scale,
+                                 const int32_t* rows, int n_rows, float* out, void* stream);
+
+/*
  * Self-test of device-side failure reporting: launches one CTA that waits on
  * a barrier nothing signals, gives up after wait_cycles (1 .. 2^31) SM clock
  * cycles and records SAGE_ERR_TIMEOUT in the workspace's status word, which

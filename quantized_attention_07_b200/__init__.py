@@ -7,7 +7,9 @@ ABI declared in include/sage.h (libsageb200.so).  This package is the Python
 binding of that library.
 """
 from .api import (  # noqa: F401
-    BLOCK, PV_MODES, Quantized, SageError, Workspace, alloc_quantized, attn_fwd, attn_fwd_varlen,
-    attn_quantized, qk_int8_tiles, quantize, quantize_varlen, sageattn, sync_status,
-    workspace_bytes, workspace_bytes_gqa, workspace_bytes_varlen,
+    BLOCK, PV_COSINE_THRESHOLD, PV_MODES, Quantized, SageError, Workspace, alloc_quantized,
+    attn_fwd, attn_fwd_varlen, attn_quantized, attn_ref_rows, calibrate_pv_modes,
+    choose_pv_mode, cosine_similarity, pv_mode_similarity, qk_int8_tiles, quantize,
+    quantize_varlen, sageattn, sync_status, workspace_bytes, workspace_bytes_gqa,
+    workspace_bytes_varlen,
 )

@@ -314,6 +314,89 @@ def qk_int8_tiles(q_codes: torch.Tensor, k_codes: torch.Tensor,
     return out
 
 
+# ------------------------------------------------ accuracy-driven P.V mode --
+#
+# "SageAttention v1/v2/v2++/v3 overview", SageAttention v1, adaptive
+# quantisation: the faster kernel variant is tested layer by layer on several
+# inputs, and a layer uses it only where its cosine similarity to
+# full-precision attention is above 99.8 % (the lowest similarity of the
+# accurate variant); the other layers keep the accurate variant.  Here the
+# faster variant is FP8 P.V and the accurate one 16-bit P.V.
+
+PV_COSINE_THRESHOLD = 0.998
+
+
+def attn_ref_rows(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rows,
+                  causal: bool = False, sm_scale: Optional[float] = None) -> torch.Tensor:
+    """Full-precision (fp32, unquantised) attention for the (b, h, i) query rows
+    `rows` of dense [B, H, N, D] q over [B, Hkv, N, D] k, v; returns [n, D] fp32."""
+    _need_cuda_contig(q, k, v)
+    B, H, N, D = q.shape
+    r = torch.as_tensor(rows, dtype=torch.int32).reshape(-1, 3).contiguous().to(q.device)
+    out = torch.empty((r.shape[0], D), dtype=torch.float32, device=q.device)
+    _check(_lib.load().sage_attn_ref_rows(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, H, k.shape[1], N, D,
+        int(bool(causal)), float(sm_scale) if sm_scale else 0.0, _ptr(r), int(r.shape[0]),
+        _ptr(out), _stream(q.device)), "sage_attn_ref_rows")
+    return out
+
+
+def cosine_similarity(a: torch.Tensor, b: torch.Tensor) -> float:
+    """Cosine similarity of two tensors taken as flat vectors (host, float64)."""
+    x = a.detach().double().cpu().flatten()
+    y = b.detach().double().cpu().flatten()
+    return float((x @ y) / (x.norm() * y.norm()))
+
+
+def choose_pv_mode(cos_fp8: float, threshold: float = PV_COSINE_THRESHOLD) -> str:
+    """FP8 P.V where its cosine similarity to full precision is above the
+    threshold, 16-bit P.V otherwise."""
+    return "fp8" if cos_fp8 > threshold else "fp16"
+
+
+def sample_query_rows(B: int, H: int, N: int, n_rows: int, seed: int = 0) -> list:
+    """Seeded (b, h, i) rows: the first and last row of every head plus uniform draws."""
+    g = torch.Generator().manual_seed(seed)
+    picks = {(b, h, i) for b in range(B) for h in range(H) for i in (0, N - 1)}
+    total = B * H * N
+    while len(picks) < min(max(n_rows, len(picks)), total):
+        u = int(torch.randint(0, total, (1,), generator=g))
+        picks.add((u // (H * N), (u // N) % H, u % N))
+    return sorted(picks)
+
+
+def pv_mode_similarity(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                       sm_scale: Optional[float] = None, n_rows: int = 256,
+                       seed: int = 0) -> dict:
+    """Cosine similarity to full-precision attention of both P.V modes on
+    sampled query rows of one input."""
+    B, H, N, D = q.shape
+    rows = sample_query_rows(B, H, N, n_rows, seed)
+    ref = attn_ref_rows(q, k, v, rows, causal, sm_scale)
+    idx = torch.tensor(rows, dtype=torch.long, device=q.device)
+    res = {}
+    for mode in ("fp16", "fp8"):
+        o = attn_fwd(q, k, v, causal=causal, sm_scale=sm_scale, pv_mode=mode,
+                     out_dtype=torch.float32)
+        res[mode] = cosine_similarity(o[idx[:, 0], idx[:, 1], idx[:, 2]], ref)
+    return res
+
+
+def calibrate_pv_modes(layers: dict, threshold: float = PV_COSINE_THRESHOLD,
+                       measure=pv_mode_similarity) -> dict:
+    """Per-layer P.V mode from sample inputs: `layers` maps a layer name to a
+    list of (q, k, v, causal) inputs seen at that layer.  A layer gets FP8 P.V
+    only if its lowest FP8 similarity over the inputs is above the threshold.
+    Returns {name: (mode, lowest FP8 similarity, lowest 16-bit similarity)}."""
+    out = {}
+    for name, inputs in layers.items():
+        sims = [measure(q, k, v, causal) for (q, k, v, causal) in inputs]
+        lo8 = min(s["fp8"] for s in sims)
+        lo16 = min(s["fp16"] for s in sims)
+        out[name] = (choose_pv_mode(lo8, threshold), lo8, lo16)
+    return out
+
+
 def sync_status(workspace: Optional[Workspace] = None, device=None) -> None:
     """Synchronise and raise if any call on the workspace recorded a device error."""
     if workspace is None:
