@@ -68,7 +68,7 @@ def lib():
         L.oracle_attn_ref_rows.argtypes = [P, P, P, i64, i32, i64, i64, i64, f64, i32, P, i64, P]
         L.oracle_attn_ref_rows.restype = None
         L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, i32, f32, f32,
-                                            i32, i32, i32, P, i64, P]
+                                            i32, i32, i32, P, i64, P, i32]
         L.oracle_attn_emul_rows.restype = None
         _lib = L
     return _lib
@@ -178,10 +178,12 @@ def attn_ref_rows(q, k, v, sm_scale: float, causal: bool, rows) -> np.ndarray:
 
 def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, causal: bool,
                    pv_mode: str, rows, v=None, p16: str = "fp16", vc=None, vdelta=None,
-                   blk: int = 128, kv: int = KV_TILE, tau=None) -> np.ndarray:
+                   blk: int = 128, kv: int = KV_TILE, tau=None,
+                   per_token: bool = False) -> np.ndarray:
     """The quantised method's output rows (fp32) for one head; see sage_oracle.c.
-    blk: quantisation block (tokens); kv: key tile of the online softmax."""
-    if blk % kv:
+    blk: quantisation block (tokens); kv: key tile of the online softmax;
+    per_token: qdelta / kdelta hold one delta per token (blk is then unused)."""
+    if not per_token and blk % kv:
         raise ValueError("the key tile must divide the quantisation block")
     qc = np.ascontiguousarray(qc, dtype=np.int8)
     kc = np.ascontiguousarray(kc, dtype=np.int8)
@@ -198,5 +200,6 @@ def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, caus
     lib().oracle_attn_emul_rows(_p(qc), _p(qdelta), _p(kc), _p(kdelta), v_p, ldv, vc_p, vd_p, n,
                                 D, blk, kv, float(kappa(sm_scale)),
                                 float(TAU[pv_mode] if tau is None else tau), int(causal), mode,
-                                1 if p16 == "bf16" else 0, _p(rows), len(rows), _p(out))
+                                1 if p16 == "bf16" else 0, _p(rows), len(rows), _p(out),
+                                int(bool(per_token)))
     return out

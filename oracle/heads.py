@@ -69,21 +69,37 @@ def repeat_kv(x: torch.Tensor, groups: int) -> torch.Tensor:
 
 
 def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
-             cu_seqlens: Optional[torch.Tensor] = None, pv_mode: str = "fp16") -> Quantized:
+             cu_seqlens: Optional[torch.Tensor] = None, pv_mode: str = "fp16",
+             gran: str = "block") -> Quantized:
+    """gran "block": one delta per 128-token block (deltas [B,H,NB]); "token"
+    (dense only): one delta per token, the quantiser applied to one-row blocks
+    (deltas [B,H,NP], padding rows 0)."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     status = 0
+    tok = gran == "token"
+    if tok and cu is not None:
+        raise ValueError("per-token scales are built for dense inputs")
     if cu is None:
         B, H, N, D = q.shape
         NB = (N + BLK - 1) // BLK
-        qc = np.zeros((B, H, NB * BLK, D), np.int8); qd = np.zeros((B, H, NB), np.float32)
+        qc = np.zeros((B, H, NB * BLK, D), np.int8)
+        qd = np.zeros((B, H, NB * BLK if tok else NB), np.float32)
         kc = np.zeros_like(qc); kd = np.zeros_like(qd)
         ks = np.zeros((B, H, D), np.int64); km = np.zeros((B, H, D), np.float32)
         for b, h, x in _heads(q, None):
-            qc[b, h], qd[b, h] = quant_head(x, None, BLK)
+            if tok:
+                c, d = quant_head(x, None, 1)
+                qc[b, h, :N], qd[b, h, :N] = c, d
+            else:
+                qc[b, h], qd[b, h] = quant_head(x, None, BLK)
         for b, h, x in _heads(k, None):
             ks[b, h], km[b, h], st = k_mean(x)
             status |= st
-            kc[b, h], kd[b, h] = quant_head(x, km[b, h], BLK)
+            if tok:
+                c, d = quant_head(x, km[b, h], 1)
+                kc[b, h, :N], kd[b, h, :N] = c, d
+            else:
+                kc[b, h], kd[b, h] = quant_head(x, km[b, h], BLK)
         vc = vd = None
         if pv_mode == "fp8":
             vc = np.zeros((B, H, N, D), np.uint8); vd = np.zeros((B, H, D), np.float32)
@@ -141,7 +157,7 @@ def _group(picks):
 
 def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, causal: bool,
                  pv_mode: str, sm_scale: Optional[float] = None,
-                 seqlens: Optional[list[int]] = None) -> dict:
+                 seqlens: Optional[list[int]] = None, gran: str = "block") -> dict:
     """E for the listed (seq, head, row) picks -> {pick: fp32 [D]}."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     sm_scale = default_sm_scale(D) if sm_scale is None else sm_scale
@@ -155,7 +171,7 @@ def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, caus
         if pv_mode == "fp16":
             vv = vf[s, h] if cu is None else np.ascontiguousarray(vf[cu[s]:cu[s + 1], h])
         o = attn_emul_rows(qc, qd, kc, kd, n, D, sm_scale, causal, pv_mode, rows, v=vv, p16=p16,
-                           vc=vc, vdelta=vd)
+                           vc=vc, vdelta=vd, per_token=gran == "token")
         for r, i in enumerate(rows):
             out[(s, h, i)] = o[r]
     return out

@@ -364,12 +364,23 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *
  * p16_format: 0 = fp16, 1 = bf16 (V's own format, used for P in pv_mode 0).
  * out: [nrows][D] fp32.
+ *
+ * per_token = 1: the other quantisation granularity of the dtcms.com page
+ * (SageAttention v1 item (1): "per-block or per-token"; the postsniper.ru
+ * post quantises "each row separately"): qdelta[i] and kdelta[j] are one delta
+ * per token, and the dequantisation is taken key first, then query:
+ *   y_ij   = fp32(S_ij * deltaK_j)
+ *   c_i    = fp32(deltaQ_i * kappa)
+ *   mb     = fp32(max_j y_ij * c_i)
+ *   arg_ij = fmaf(y_ij, c_i, -m_new)
+ * (the product (A^ B^) deltaA deltaB of the quantisation intro, step 3, with a
+ * per-row deltaA and a per-column deltaB); everything else as above.
  */
 void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* kc,
                            const float* kdelta, const float* v, long ldv, const uint8_t* vc,
                            const float* vdelta, long n, int D, int blk, int kv, float kappa,
                            float tau, int causal, int pv_mode, int p16_format, const long* rows,
-                           long nrows, float* out)
+                           long nrows, float* out, int per_token)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (long r = 0; r < nrows; ++r) {
@@ -382,6 +393,7 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
         double* part = (double*)malloc(sizeof(double) * (size_t)D);
         int32_t* S = (int32_t*)malloc(sizeof(int32_t) * (size_t)kv);
         float* p = (float*)malloc(sizeof(float) * (size_t)kv);
+        float* y = (float*)malloc(sizeof(float) * (size_t)kv);
         for (long T = 0; T < Tend; ++T) {
             long j0 = T * kv;
             long J = j0 / blk;
@@ -396,13 +408,27 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
                 S[jj] = acc;
                 if (acc > smax) smax = acc;
             }
-            float c = (qdelta[I] * kdelta[J]) * kappa;
-            float mblk = (float)smax * c;
+            float c, mblk;
+            if (!per_token) {
+                /* one delta per 128-token block of Q and of K */
+                c = (qdelta[I] * kdelta[J]) * kappa;
+                mblk = (float)smax * c;
+            } else {
+                /* one delta per token: S_ij deltaK_j first (a key's own
+                 * scale), then the query row's deltaQ_i kappa */
+                c = qdelta[i] * kappa;
+                float ymax = -INFINITY;
+                for (int jj = 0; jj < nj; ++jj) {
+                    y[jj] = (float)S[jj] * kdelta[j0 + jj];
+                    if (y[jj] > ymax) ymax = y[jj];
+                }
+                mblk = ymax * c;
+            }
             float m_new = mblk > m + tau ? mblk : m;
             float alpha = (float)exp2((double)(m - m_new));
             double psum = 0.0;
             for (int jj = 0; jj < nj; ++jj) {
-                float arg = fmaf((float)S[jj], c, -m_new);
+                float arg = per_token ? fmaf(y[jj], c, -m_new) : fmaf((float)S[jj], c, -m_new);
                 p[jj] = (float)exp2((double)arg);
                 psum += (double)p[jj];
             }
@@ -430,6 +456,6 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
             if (pv_mode == 0) o[d] = O[d] / l;
             else o[d] = (O[d] * (vdelta[d] / 448.0f)) / l;
         }
-        free(O); free(part); free(S); free(p);
+        free(O); free(part); free(S); free(p); free(y);
     }
 }

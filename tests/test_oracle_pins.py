@@ -436,3 +436,93 @@ def test_grouped_reference_uses_the_kv_head_of_each_group():
         out = oracle.attn_ref_rows(q[0, hq].numpy(), kr[0, hq].numpy(), vr[0, hq].numpy(),
                                    oracle.default_sm_scale(D), False, np.arange(N))
         assert np.allclose(out, hq // g + 1.0, atol=1e-12)
+
+
+# ------------------------------------------------------- per-token deltas --
+
+def test_per_token_quantiser_is_the_block_quantiser_on_each_row():
+    """Per-token granularity = the quantiser with one-row blocks: every row's
+    delta and codes match the exact rational quantiser of that row alone."""
+    gen = torch.Generator().manual_seed(21)
+    x = (torch.randn(37, 16, generator=gen) * 3).half().float().numpy()
+    x[5] = 0.0                                     # an all-zero row: delta 0, codes 0
+    codes, delta = oracle.quant_head(x, None, 1)
+    assert codes.shape == (37, 16) and delta.shape == (37,)
+    for r in range(37):
+        amax = float(np.abs(x[r]).max())
+        for d in range(16):
+            c, dl = quantize_exact(float(x[r, d]), amax)
+            assert codes[r, d] == c
+        assert delta[r] == (dl if amax > 0 else 0.0)
+
+
+def _per_token_lossless(n, D, seed):
+    """Rows of integer codes with a +-127 in channel 0 (so each row's delta is
+    its power-of-two scale exactly); K rows in pairs (r, r+1) with opposite
+    codes and equal scales, so every channel of K sums to zero (mean 0)."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-126, 127, size=(n, D)).astype(np.float64)
+    q[:, 0] = 127
+    qs = np.array([2.0 ** ((r % 3) - 1) for r in range(n)])
+    k = np.zeros((n, D))
+    ks = np.zeros(n)
+    for r in range(0, n, 2):
+        row = rng.integers(-126, 127, size=D).astype(np.float64)
+        row[0] = 127
+        k[r], k[r + 1] = row, -row
+        ks[r] = ks[r + 1] = 2.0 ** ((r // 2) % 3 - 1)
+    return (q * qs[:, None]).astype(np.float32), (k * ks[:, None]).astype(np.float32), qs, ks
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_per_token_emulation_lossless_matches_reference(causal):
+    """Exact per-token codes: the only approximation left (16-bit P.V) is P's
+    fp16 rounding; per-row and per-key deltas that differ by powers of two make
+    a wrong index visible."""
+    n, D = 200, 16
+    q, k, qs, ks = _per_token_lossless(n, D, 4)
+    v = np.random.default_rng(5).standard_normal((n, D)).astype(np.float32)
+    qt, kt, vt = (torch.from_numpy(a)[None, None].half() for a in (q, k, v))
+    assert torch.equal(qt.float()[0, 0], torch.from_numpy(q))
+    assert torch.equal(kt.float()[0, 0], torch.from_numpy(k))
+    qz = heads.quantize(qt, kt, vt, None, "fp16", gran="token")
+    assert np.array_equal(qz.q_delta[0, 0, :n], qs.astype(np.float32))
+    assert np.array_equal(qz.k_delta[0, 0, :n], ks.astype(np.float32))
+    assert not qz.k_mean.any() and not qz.q_delta[0, 0, n:].any()
+    sm = 1.0 / 12000.0
+    picks = [(0, 0, i) for i in range(n)]
+    emu = heads.emulate_rows(qz, vt, None, picks, D, causal, "fp16", sm, gran="token")
+    out = np.stack([emu[p] for p in picks])
+    ref = oracle.attn_ref_rows(q, k, vt[0, 0].float().numpy(), float(np.float32(sm)), causal,
+                               np.arange(n))
+    assert np.abs(out - ref).max() <= 2.0 ** -10 * np.abs(v).max() + 1e-5
+
+
+def test_per_token_emulation_follows_its_rounding_sequence():
+    """One query row over three keys in one tile, computed with exact rationals
+    along the documented steps (y = fp32(S dK_j), c = fp32(dQ kappa),
+    mb = fp32(max y * c), arg = fp32(y c - mb), p = fp32(2^arg), P = fp16(p),
+    out = fp32(fp32(sum P v) / fp32(sum p))): the C emulation agrees exactly."""
+    from fractions import Fraction as Fr
+    import math
+    qc = np.array([[3, -7, 11, 2]], np.int8)
+    kc = np.array([[5, 1, -2, 9], [-4, 8, 3, 1], [7, 7, -7, 0]], np.int8)
+    qd = np.array([0.0123], np.float32)
+    kd = np.array([0.031, 0.0207, 0.0444], np.float32)
+    v = np.array([[1.5, -2.0, 0.25, 3.0], [0.5, 1.0, -1.0, 2.0], [-0.75, 0.125, 2.5, -1.5]],
+                 np.float32)
+    sm = 0.5
+    kap = oracle.kappa(sm)
+    got = oracle.attn_emul_rows(qc, qd, kc, kd, 3, 4, sm, False, "fp16", [0], v=v,
+                                per_token=True, tau=8.0)[0]
+    S = [int(np.dot(qc[0].astype(np.int64), kc[j].astype(np.int64))) for j in range(3)]
+    y = [fp32(Fr(S[j]) * Fr(float(kd[j]))) for j in range(3)]
+    c = fp32(Fr(float(qd[0])) * Fr(float(kap)))
+    mb = fp32(Fr(max(y)) * Fr(c))
+    args = [fp32(Fr(y[j]) * Fr(c) - Fr(mb)) for j in range(3)]
+    p = [float(np.float32(math.pow(2.0, a))) for a in args]
+    P = [float(np.float16(x)) for x in p]
+    l = fp32(sum(Fr(x) for x in p))
+    want = [fp32(fp32(sum(Fr(P[j]) * Fr(float(v[j, d])) for j in range(3))) / Fr(l))
+            for d in range(4)]
+    assert got.tolist() == want
