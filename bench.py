@@ -211,12 +211,12 @@ def run_ours(args, rank, world, local):
         launches_per_step = 3  # quant_stream_kernel (K, V), quant_stream_kernel (Q), attn_fwd
     elif not wl.varlen:
         B, H, N, D = q.shape
-        qz = api.alloc_quantized(B, H, N, D, wl.pv_mode, dev)
+        qz = api.alloc_quantized(B, H, N, D, wl.pv_mode, dev, qk_gran=wl.qk_gran)
         out = torch.empty_like(q)
         ws = sage.Workspace(sage.workspace_bytes(B, H, N, D, wl.pv_mode), dev)
 
         def stage1():
-            api.quantize(q, k, v, wl.pv_mode, qz=qz, workspace=ws)
+            api.quantize(q, k, v, wl.pv_mode, qz=qz, workspace=ws, qk_gran=wl.qk_gran)
 
         def stage2():
             api.attn_quantized(qz, v, causal=wl.causal, out=out, workspace=ws)
@@ -280,7 +280,8 @@ def run_ours(args, rank, world, local):
                 o = sage.attn_fwd_varlen(dq, dk, dv, dcu, max(inp.seqlens), causal=wl.causal,
                                          pv_mode=wl.pv_mode, workspace=ws)
             else:
-                o = sage.attn_fwd(dq, dk, dv, causal=wl.causal, pv_mode=wl.pv_mode, workspace=ws)
+                o = sage.attn_fwd(dq, dk, dv, causal=wl.causal, pv_mode=wl.pv_mode, workspace=ws,
+                                  qk_gran=wl.qk_gran)
             hout.copy_(o, non_blocking=True)
 
         for _ in range(2):
@@ -331,7 +332,7 @@ def run_ours(args, rank, world, local):
         "dtype": "int8/fp8" if wl.pv_mode == "fp8" else "int8/fp16",
         "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D,
-                   "Hkv": wl.kv_heads,
+                   "Hkv": wl.kv_heads, "qk_gran": wl.qk_gran,
                    "in_dtype": wl.dtype, "causal": wl.causal, "pv_mode": wl.pv_mode,
                    "seqlens": inp.seqlens if wl.varlen else None,
                    "l2": f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB of q,k,v > 126 MiB)"
@@ -377,12 +378,13 @@ def cpu_oracle_throughput(wl, inp, budget_rows: int, quant_heads: int, seed: int
     sl = lambda x: x[:, :hs].contiguous()
     qh, kh, vh = sl(inp.q), sl(k_in), sl(v_in)
     t0 = time.perf_counter()
-    qz = heads.quantize(qh, kh, vh, inp.cu_seqlens, wl.pv_mode)
+    qz = heads.quantize(qh, kh, vh, inp.cu_seqlens, wl.pv_mode, gran=wl.qk_gran)
     t_quant = time.perf_counter() - t0
     # emulated rows, drawn over the quantised heads
     picks = [p for p in W.sample_rows(lens, hs, budget_rows, seed) if p[1] < hs]
     t0 = time.perf_counter()
-    heads.emulate_rows(qz, vh, inp.cu_seqlens, picks, wl.D, wl.causal, wl.pv_mode)
+    heads.emulate_rows(qz, vh, inp.cu_seqlens, picks, wl.D, wl.causal, wl.pv_mode,
+                       gran=wl.qk_gran)
     t_rows = time.perf_counter() - t0
 
     def work(i):  # key pairs of row i

@@ -72,6 +72,13 @@ typedef enum {
   SAGE_PV_FP8 = 1   /* P, V in FP8 E4M3, per-block fp32 two-level accumulation */
 } sage_pv_mode_t;
 
+/* Granularity of the Q and K deltas ("SageAttention v1/v2/v2++/v3 overview",
+ * SageAttention v1 item (1): per-block or per-token quantisation of q, k). */
+typedef enum {
+  SAGE_QK_PER_BLOCK = 0, /* one delta per 128-token block (and head)             */
+  SAGE_QK_PER_TOKEN = 1  /* one delta per token; dense inputs only                */
+} sage_qk_gran_t;
+
 /* Token count of one quantisation block and of one attention key/query tile. */
 #define SAGE_BLOCK 128
 
@@ -124,6 +131,23 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
                             int in_dt, int out_dt, int B, int H, int N, int D, int causal,
                             float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
                             void* stream);
+
+/*
+ * General dense forward pass: grouped-query heads (Hkv divides H; Hkv = H
+ * without grouping, see sage_attn_fwd_gqa) and the Q/K delta granularity
+ * qk_gran (sage_qk_gran_t).  With SAGE_QK_PER_TOKEN every query row and key
+ * has its own delta = max over its D channels / 127, and the scores are
+ * dequantised as y = fp32(S_ij * deltaK_j), arg = fmaf(y, fp32(deltaQ_i *
+ * sm_scale * log2 e), -m) (per block: c = fp32(fp32(deltaQ*deltaK) * kappa),
+ * arg = fmaf(S, c, -m)).
+ *   ws : at least sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, qk_gran).
+ * sage_attn_fwd(...) = sage_attn_fwd_ex(..., Hkv = H, ..., SAGE_QK_PER_BLOCK).
+ */
+size_t sage_workspace_bytes_ex(int B, int H, int Hkv, int N, int D, int pv_mode, int qk_gran);
+sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
+                               int in_dt, int out_dt, int B, int H, int Hkv, int N, int D,
+                               int causal, float sm_scale, int pv_mode, int qk_gran, void* ws,
+                               size_t ws_bytes, void* stream);
 
 /*
  * Grouped-query variant: q and out are [B, H, N, D]; k and v are
@@ -193,6 +217,27 @@ sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
                                   int v_dt, int out_dt, int B, int H, int N, int D, int causal,
                                   float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
                                   void* stream);
+
+/*
+ * The two stages for grouped-query heads and either delta granularity (see
+ * sage_attn_fwd_ex).  Layouts as sage_quantize with H query heads for Q and
+ * Hkv key/value heads for K, k_mean and (FP8) V; with SAGE_QK_PER_TOKEN the
+ * deltas are fp32 [B, H, NP] (Q) and [B, Hkv, NP] (K), one per code row,
+ * padding rows 0.  sage_attn_quantized_ex needs k_scale 16-byte aligned (the
+ * kernel copies 128 deltas at a time).  ws: at least sage_scratch_bytes(B, H,
+ * D), which covers every Hkv <= H (SAGE_ERR_WORKSPACE when too small).
+ */
+sage_status_t sage_quantize_ex(const void* q, const void* k, const void* v, int in_dt, int B,
+                               int H, int Hkv, int N, int D, int pv_mode, int qk_gran,
+                               int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
+                               float* k_mean, uint8_t* v_codes, float* v_scale, void* ws,
+                               size_t ws_bytes, void* stream);
+sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale,
+                                     const int8_t* k_codes, const float* k_scale, const void* v,
+                                     const uint8_t* v_codes, const float* v_scale, void* out,
+                                     int v_dt, int out_dt, int B, int H, int Hkv, int N, int D,
+                                     int causal, float sm_scale, int pv_mode, int qk_gran,
+                                     void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Stage 1 for a packed varlen batch.  Layouts (TB = number of 128-token blocks

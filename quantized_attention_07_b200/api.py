@@ -132,11 +132,12 @@ def workspace_bytes_varlen(total_tokens: int, batch: int, H: int, D: int,
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              sm_scale: Optional[float] = None, pv_mode: str = "fp16",
              out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
-             workspace: Optional[Workspace] = None) -> torch.Tensor:
+             workspace: Optional[Workspace] = None, qk_gran: str = "block") -> torch.Tensor:
     """SageAttention forward over dense [B, H, N, D] fp16/bf16 tensors.
 
     k and v may have fewer heads than q ([B, Hkv, N, D], H a multiple of Hkv):
     grouped-query attention, query head h reading key/value head h // (H // Hkv).
+    qk_gran: "block" (one Q/K delta per 128 tokens) or "token" (one per token).
     """
     _need_cuda_contig(q, k, v)
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
@@ -154,7 +155,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     mode = _pv(pv_mode)
     scale = float(sm_scale) if sm_scale else 0.0
     lib = _lib.load()
-    if Hkv == H:
+    gran = _gran(qk_gran)
+    if gran:
+        ws = _workspace(q.device, int(lib.sage_workspace_bytes_ex(B, H, Hkv, N, D, mode, gran)),
+                        workspace)
+        _check(lib.sage_attn_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+            _dtype_code(out.dtype, True), B, H, Hkv, N, D, int(bool(causal)), scale, mode, gran,
+            ws.ptr, ws.nbytes, _stream(q.device)), "sage_attn_fwd_ex")
+    elif Hkv == H:
         ws = _workspace(q.device, workspace_bytes(B, H, N, D, pv_mode), workspace)
         _check(lib.sage_attn_fwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
@@ -198,9 +207,20 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
 
 # ---------------------------------------------------------------- stages --
 
+QK_GRANS = {"block": 0, "token": 1}
+
+
+def _gran(g: str) -> int:
+    if g not in QK_GRANS:
+        raise ValueError(f"qk_gran must be one of {sorted(QK_GRANS)}")
+    return QK_GRANS[g]
+
+
 @dataclasses.dataclass
 class Quantized:
-    """Outputs of the smoothing + quantisation stage (all device tensors)."""
+    """Outputs of the smoothing + quantisation stage (all device tensors).
+    Dense: q_codes [B, H, NP, D], k_codes [B, Hkv, NP, D]; deltas [.., NB]
+    per 128-token block or [.., NP] per token (qk_gran)."""
     q_codes: torch.Tensor
     q_scale: torch.Tensor
     k_codes: torch.Tensor
@@ -209,41 +229,48 @@ class Quantized:
     v_codes: Optional[torch.Tensor]
     v_scale: Optional[torch.Tensor]
     pv_mode: str
+    qk_gran: str = "block"
 
 
-def alloc_quantized(B: int, H: int, N: int, D: int, pv_mode: str, device) -> Quantized:
+def alloc_quantized(B: int, H: int, N: int, D: int, pv_mode: str, device,
+                    Hkv: Optional[int] = None, qk_gran: str = "block") -> Quantized:
     NB = (N + BLOCK - 1) // BLOCK
+    NS = NB * BLOCK if _gran(qk_gran) else NB
+    Hk = Hkv or H
     fp8 = pv_mode == "fp8"
     e = dict(device=device)
     return Quantized(
         torch.empty((B, H, NB * BLOCK, D), dtype=torch.int8, **e),
-        torch.empty((B, H, NB), dtype=torch.float32, **e),
-        torch.empty((B, H, NB * BLOCK, D), dtype=torch.int8, **e),
-        torch.empty((B, H, NB), dtype=torch.float32, **e),
-        torch.empty((B, H, D), dtype=torch.float32, **e),
-        torch.empty((B, H, N, D), dtype=torch.uint8, **e) if fp8 else None,
-        torch.empty((B, H, D), dtype=torch.float32, **e) if fp8 else None,
-        pv_mode)
+        torch.empty((B, H, NS), dtype=torch.float32, **e),
+        torch.empty((B, Hk, NB * BLOCK, D), dtype=torch.int8, **e),
+        torch.empty((B, Hk, NS), dtype=torch.float32, **e),
+        torch.empty((B, Hk, D), dtype=torch.float32, **e),
+        torch.empty((B, Hk, N, D), dtype=torch.uint8, **e) if fp8 else None,
+        torch.empty((B, Hk, D), dtype=torch.float32, **e) if fp8 else None,
+        pv_mode, qk_gran)
 
 
 def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
              pv_mode: str = "fp16", qz: Optional[Quantized] = None,
-             workspace: Optional[Workspace] = None) -> Quantized:
-    """Stage 1 (K smoothing, per-block INT8 Q/K, FP8 V) of a dense problem."""
+             workspace: Optional[Workspace] = None, qk_gran: str = "block") -> Quantized:
+    """Stage 1 (K smoothing, INT8 Q/K per block or per token, FP8 V) of a dense
+    problem; k, v may have fewer heads than q (grouped-query)."""
     _need_cuda_contig(q, k)
     B, H, N, D = q.shape
+    Hkv = k.shape[1]
     mode = _pv(pv_mode)
+    gran = _gran(qk_gran)
     if mode == 1:
         if v is None:
             raise ValueError("FP8 P.V needs v")
         _need_cuda_contig(v)
-    qz = qz or alloc_quantized(B, H, N, D, pv_mode, q.device)
+    qz = qz or alloc_quantized(B, H, N, D, pv_mode, q.device, Hkv, qk_gran)
     ws = _workspace(q.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
-    _check(_lib.load().sage_quantize(
-        _ptr(q), _ptr(k), _ptr(v) if mode == 1 else None, _dtype_code(q.dtype), B, H, N, D, mode,
-        _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(qz.k_mean),
-        _ptr(qz.v_codes), _ptr(qz.v_scale), ws.ptr, ws.nbytes, _stream(q.device)),
-        "sage_quantize")
+    _check(_lib.load().sage_quantize_ex(
+        _ptr(q), _ptr(k), _ptr(v) if mode == 1 else None, _dtype_code(q.dtype), B, H, Hkv, N, D,
+        mode, gran, _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale),
+        _ptr(qz.k_mean), _ptr(qz.v_codes), _ptr(qz.v_scale), ws.ptr, ws.nbytes,
+        _stream(q.device)), "sage_quantize_ex")
     return qz
 
 
@@ -253,18 +280,19 @@ def attn_quantized(qz: Quantized, v: torch.Tensor, causal: bool = False,
                    workspace: Optional[Workspace] = None) -> torch.Tensor:
     """Stage 2 (fused INT8 QK^T, online softmax, P.V) from stage-1 outputs."""
     _need_cuda_contig(v)
-    B, H, N, D = v.shape
+    B, H, NP, D = qz.q_codes.shape
+    Hkv, N = v.shape[1], v.shape[2]
     mode = _pv(qz.pv_mode)
     od = out_dtype or v.dtype
     if out is None:
         out = torch.empty((B, H, N, D), dtype=od, device=v.device)
     ws = _workspace(v.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
-    _check(_lib.load().sage_attn_quantized(
+    _check(_lib.load().sage_attn_quantized_ex(
         _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(v),
         _ptr(qz.v_codes), _ptr(qz.v_scale), _ptr(out), _dtype_code(v.dtype),
-        _dtype_code(out.dtype, True), B, H, N, D, int(bool(causal)),
-        float(sm_scale) if sm_scale else 0.0, mode, ws.ptr, ws.nbytes, _stream(v.device)),
-        "sage_attn_quantized")
+        _dtype_code(out.dtype, True), B, H, Hkv, N, D, int(bool(causal)),
+        float(sm_scale) if sm_scale else 0.0, mode, _gran(qz.qk_gran), ws.ptr, ws.nbytes,
+        _stream(v.device)), "sage_attn_quantized_ex")
     return out
 
 
@@ -412,7 +440,7 @@ def sync_status(workspace: Optional[Workspace] = None, device=None) -> None:
 
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, attn_mask=None,
              dropout_p: float = 0.0, is_causal: bool = False, scale: Optional[float] = None,
-             pv_mode: str = "fp16") -> torch.Tensor:
+             pv_mode: str = "fp16", qk_gran: str = "block") -> torch.Tensor:
     """Drop-in for scaled_dot_product_attention on [B, H, N, D] fp16/bf16 inputs.
 
     Arbitrary masks and dropout are not part of the method; passing them raises
@@ -424,7 +452,7 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, attn_mask=None,
     if attn_mask is not None or dropout_p:
         raise SageError(2, "sageattn: attn_mask / dropout_p")
     q, k, v = (t if t.is_contiguous() else t.contiguous() for t in (q, k, v))
-    return attn_fwd(q, k, v, causal=is_causal, sm_scale=scale, pv_mode=pv_mode)
+    return attn_fwd(q, k, v, causal=is_causal, sm_scale=scale, pv_mode=pv_mode, qk_gran=qk_gran)
 
 
 def default_sm_scale(D: int) -> float:

@@ -17,7 +17,7 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                          uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
-                         cudaStream_t st);
+                         int per_token, cudaStream_t st);
 cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
                             const int32_t* tiles, int n, int32_t* out, uint32_t* status,
                             cudaStream_t st);
@@ -61,9 +61,9 @@ struct Layout {
 // without grouping).  sync: work counter + one completion counter per
 // key/value head for the launch that quantises K (and Q when Hkv = H);
 // sync_q: the work counter of the separate Q launch when Hkv < H.
-Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv) {
+Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, bool per_token = false) {
   const size_t BH = (size_t)B * H, BK = (size_t)B * Hkv, NB = ((size_t)N + BLK - 1) / BLK,
-               NP = NB * BLK;
+               NP = NB * BLK, NS = per_token ? NP : NB;  // deltas per head
   Layout L{};
   size_t o = kHeader;
   L.k_sum = o; o += al(BK * D * 8);
@@ -73,8 +73,8 @@ Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv) {
   L.scratch_end = o;
   L.q_codes = o; o += al(BH * NP * D);
   L.k_codes = o; o += al(BK * NP * D);
-  L.q_scale = o; o += al(BH * NB * 4);
-  L.k_scale = o; o += al(BK * NB * 4);
+  L.q_scale = o; o += al(BH * NS * 4);
+  L.k_scale = o; o += al(BK * NS * 4);
   L.k_mean = o; o += al(BK * D * 4);
   if (fp8) {
     L.v_codes = o; o += al(BK * (size_t)N * D);
@@ -117,6 +117,7 @@ bool dense_args_ok(int B, int H, int N, int D, int pv_mode) {
 }
 
 bool gqa_heads_ok(int H, int Hkv) { return Hkv >= 1 && Hkv <= H && H % Hkv == 0; }
+bool gran_ok(int g) { return g == SAGE_QK_PER_BLOCK || g == SAGE_QK_PER_TOKEN; }
 
 bool varlen_args_ok(int T, int batch, int max_seqlen, int H, int D, int pv_mode) {
   return T >= 0 && batch >= 1 && max_seqlen >= 0 && max_seqlen <= kMaxN && H >= 1 &&
@@ -150,7 +151,7 @@ sage_status_t quantize_dense(const void* q, const void* k, const void* v, int in
                              int H, int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
                              int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
                              float* v_scale, void* ws, const Layout& L, cudaStream_t st,
-                             int Hkv) {
+                             int Hkv, int per_token = 0) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   sage_status_t r = clear_scratch(ws, L, fp8, st);
   if (r != SAGE_OK) return r;
@@ -164,13 +165,13 @@ sage_status_t quantize_dense(const void* q, const void* k, const void* v, int in
                                k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
                                at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
                                at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync),
-                               grouped ? QUANT_KV : QUANT_Q | QUANT_KV, st);
+                               grouped ? QUANT_KV : QUANT_Q | QUANT_KV, per_token, st);
   if (e == cudaSuccess && grouped) {
     S.H = H;
     e = launch_quant(S, dim3(NB, (unsigned)(B * H)), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes,
                      q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
                      at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                     at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync_q), QUANT_Q, st);
+                     at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync_q), QUANT_Q, per_token, st);
   }
   if (e == cudaErrorNotSupported) return SAGE_ERR_UNSUPPORTED;
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
@@ -180,11 +181,12 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
                          const float* k_scale, const void* v, const uint8_t* v_codes,
                          const float* v_scale, void* out, int v_dt, int out_dt, int B, int H,
                          int N, int D, int causal, float sm_scale, int pv_mode, void* ws,
-                         cudaStream_t st, int Hkv) {
+                         cudaStream_t st, int Hkv, int per_token = 0) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   AttnLaunch A{};
   A.p.H = H;
   A.p.Hkv = Hkv;
+  A.p.per_token = per_token;
   A.p.N = N;
   A.p.BH = B * H;
   A.p.NB = (N + BLK - 1) / BLK;
@@ -272,20 +274,54 @@ sage_status_t sage_sync_status(void* ws, void* stream) {
   return SAGE_OK;
 }
 
-sage_status_t sage_quantize(const void* q, const void* k, const void* v, int in_dt, int B, int H,
-                            int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
-                            int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
-                            float* v_scale, void* ws, size_t ws_bytes, void* stream) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !in_dtype_ok(in_dt)) return SAGE_ERR_INVALID_ARG;
+sage_status_t sage_quantize_ex(const void* q, const void* k, const void* v, int in_dt, int B,
+                               int H, int Hkv, int N, int D, int pv_mode, int qk_gran,
+                               int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
+                               float* k_mean, uint8_t* v_codes, float* v_scale, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran) ||
+      !in_dtype_ok(in_dt))
+    return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes) ||
       !q_scale || !k_scale || !k_mean || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
   if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
-  const Layout L = dense_layout(B, H, N, D, fp8);
+  const bool tok = qk_gran == SAGE_QK_PER_TOKEN;
+  const Layout L = dense_layout(B, H, N, D, fp8, Hkv, tok);
   if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
   return quantize_dense(q, k, v, in_dt, B, H, N, D, pv_mode, q_codes, q_scale, k_codes, k_scale,
-                        k_mean, v_codes, v_scale, ws, L, as_stream(stream), H);
+                        k_mean, v_codes, v_scale, ws, L, as_stream(stream), Hkv, tok ? 1 : 0);
+}
+
+sage_status_t sage_quantize(const void* q, const void* k, const void* v, int in_dt, int B, int H,
+                            int N, int D, int pv_mode, int8_t* q_codes, float* q_scale,
+                            int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
+                            float* v_scale, void* ws, size_t ws_bytes, void* stream) {
+  return sage_quantize_ex(q, k, v, in_dt, B, H, H, N, D, pv_mode, SAGE_QK_PER_BLOCK, q_codes,
+                          q_scale, k_codes, k_scale, k_mean, v_codes, v_scale, ws, ws_bytes,
+                          stream);
+}
+
+sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale,
+                                     const int8_t* k_codes, const float* k_scale, const void* v,
+                                     const uint8_t* v_codes, const float* v_scale, void* out,
+                                     int v_dt, int out_dt, int B, int H, int Hkv, int N, int D,
+                                     int causal, float sm_scale, int pv_mode, int qk_gran,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran) ||
+      !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !aligned16(k_scale) ||
+      !aligned16(out) || !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+    return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
+  return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
+                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), Hkv,
+                    qk_gran == SAGE_QK_PER_TOKEN ? 1 : 0);
 }
 
 sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
@@ -294,63 +330,58 @@ sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
                                   int v_dt, int out_dt, int B, int H, int N, int D, int causal,
                                   float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
                                   void* stream) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
-    return SAGE_ERR_INVALID_ARG;
-  const bool fp8 = pv_mode == SAGE_PV_FP8;
-  if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !k_scale || !aligned16(out) ||
-      !aligned16(ws))
-    return SAGE_ERR_INVALID_ARG;
-  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
-    return SAGE_ERR_INVALID_ARG;
-  if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
-  return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
-                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), H);
+  return sage_attn_quantized_ex(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out,
+                                v_dt, out_dt, B, H, H, N, D, causal, sm_scale, pv_mode,
+                                SAGE_QK_PER_BLOCK, ws, ws_bytes, stream);
 }
 
-// Whole dense path for H query heads over Hkv key/value heads per batch.
-static sage_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* out,
-                                    int in_dt, int out_dt, int B, int H, int Hkv, int N, int D,
-                                    int causal, float sm_scale, int pv_mode, void* ws,
-                                    size_t ws_bytes, void* stream) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !in_dtype_ok(in_dt) ||
-      !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
+size_t sage_workspace_bytes_ex(int B, int H, int Hkv, int N, int D, int pv_mode, int qk_gran) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran)) return 0;
+  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv, qk_gran == SAGE_QK_PER_TOKEN).total;
+}
+
+sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int in_dt,
+                               int out_dt, int B, int H, int Hkv, int N, int D, int causal,
+                               float sm_scale, int pv_mode, int qk_gran, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran) ||
+      !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
     return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
-  const bool fp8 = pv_mode == SAGE_PV_FP8;
-  const Layout L = dense_layout(B, H, N, D, fp8, Hkv);
+  const bool fp8 = pv_mode == SAGE_PV_FP8, tok = qk_gran == SAGE_QK_PER_TOKEN;
+  const Layout L = dense_layout(B, H, N, D, fp8, Hkv, tok);
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   sage_status_t r = quantize_dense(
       q, k, v, in_dt, B, H, N, D, pv_mode, at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
       at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
       fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr, fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L,
-      st, Hkv);
+      st, Hkv, tok ? 1 : 0);
   if (r != SAGE_OK) return r;
   return attn_dense(at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale), at<int8_t>(ws, L.k_codes),
                     at<float>(ws, L.k_scale), v, fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
                     fp8 ? at<float>(ws, L.v_scale) : nullptr, out, in_dt, out_dt, B, H, N, D,
-                    causal, sm_scale, pv_mode, ws, st, Hkv);
+                    causal, sm_scale, pv_mode, ws, st, Hkv, tok ? 1 : 0);
 }
 
 sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int in_dt,
                             int out_dt, int B, int H, int N, int D, int causal, float sm_scale,
                             int pv_mode, void* ws, size_t ws_bytes, void* stream) {
-  return attn_fwd_dense(q, k, v, out, in_dt, out_dt, B, H, H, N, D, causal, sm_scale, pv_mode, ws,
-                        ws_bytes, stream);
+  return sage_attn_fwd_ex(q, k, v, out, in_dt, out_dt, B, H, H, N, D, causal, sm_scale, pv_mode,
+                          SAGE_QK_PER_BLOCK, ws, ws_bytes, stream);
 }
 
 size_t sage_workspace_bytes_gqa(int B, int H, int Hkv, int N, int D, int pv_mode) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv)) return 0;
-  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv).total;
+  return sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, SAGE_QK_PER_BLOCK);
 }
 
 sage_status_t sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* out, int in_dt,
                                 int out_dt, int B, int H, int Hkv, int N, int D, int causal,
                                 float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
                                 void* stream) {
-  return attn_fwd_dense(q, k, v, out, in_dt, out_dt, B, H, Hkv, N, D, causal, sm_scale, pv_mode,
-                        ws, ws_bytes, stream);
+  return sage_attn_fwd_ex(q, k, v, out, in_dt, out_dt, B, H, Hkv, N, D, causal, sm_scale, pv_mode,
+                          SAGE_QK_PER_BLOCK, ws, ws_bytes, stream);
 }
 
 static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, int in_dt,
@@ -377,7 +408,7 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
   e = launch_quant(S, dim3((unsigned)TB, H), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes, q_scale,
                    k_codes, k_scale, k_mean, v_codes, v_scale,
                    at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                   at<uint32_t>(ws, 0), nullptr, QUANT_Q | QUANT_KV, st);
+                   at<uint32_t>(ws, 0), nullptr, QUANT_Q | QUANT_KV, 0, st);
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
 

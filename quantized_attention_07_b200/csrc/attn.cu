@@ -48,7 +48,7 @@ namespace {
 
 constexpr int SUB = 64;  // keys per softmax sub-tile
 
-template <int D, bool PV8>
+template <int D, bool PV8, bool TOK>
 struct Cfg {
   // warpgroups: 2 softmax, 1 control
   static constexpr int WGS = 3;
@@ -63,11 +63,12 @@ struct Cfg {
 
   static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
   static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
+  static constexpr int KS = TOK ? BLK * 4 : 0;          // per-token K deltas of a stage
   static constexpr int AUX = 1024;                      // barriers
   static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - AUX;
-  static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT);
+  static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT + KS);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;    // pipeline stages (128 keys each)
-  static constexpr int SMEM = 1024 + 2 * QT + NS * (QT + VT) + AUX;
+  static constexpr int SMEM = 1024 + 2 * QT + NS * (QT + VT + KS) + AUX;
   // int8 code tiles: rows of D bytes
   static constexpr uint32_t QK_SWZ = (D == 128) ? 2u : 4u;  // 128B : 64B swizzle
   static constexpr uint32_t QK_SBO = 8 * D;                 // 8 rows
@@ -205,11 +206,11 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
 
 // --------------------------------------------------------------- producer --
 
-template <int D, bool PV8>
+template <int D, bool PV8, bool TOK>
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const Work& w, Bars* B, uint8_t* sQ, uint8_t* sK, uint8_t* sV,
-                         uint32_t* status) {
-  using C = Cfg<D, PV8>;
+                         float* sKs, const float* k_scale, uint32_t* status) {
+  using C = Cfg<D, PV8, TOK>;
   // The whole warp runs this loop (uniform control flow); one elected lane
   // issues each TMA instruction.
   if (ptx::elect_one()) {
@@ -227,8 +228,11 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
     const int s = j % C::NS;
     if (j >= C::NS && !wait_bar(B, &B->kv_empty[s], ((j / C::NS) - 1) & 1, status, true)) break;
     if (ptx::elect_one()) {
-      ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT);
+      ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);
       ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
+      if constexpr (TOK)  // the stage's 128 per-token K deltas, on the same barrier
+        ptx::bulk_load_plain(sKs + s * BLK, k_scale + (w.ks_idx0 + j) * BLK, C::KS,
+                             &B->k_full[s]);
       ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
       uint8_t* dst = sV + s * C::VT;
       const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
@@ -258,10 +262,10 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
 // Issue order per thread is execution order, so S_t(i+2) never overwrites
 // P_t(i) before P.V has read it.  A 128-key stage is released to the producer
 // when both tiles' warps have committed it (kv_empty counts two arrivals).
-template <int D, bool PV8, bool BF16V>
+template <int D, bool PV8, bool BF16V, bool TOK>
 __device__ void mma_issuer(const Work& w, Bars* B, uint32_t tmem, const uint8_t* sQ,
                            const uint8_t* sK, const uint8_t* sV, int t, uint32_t* status) {
-  using C = Cfg<D, PV8>;
+  using C = Cfg<D, PV8, TOK>;
   constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, SUB);
   constexpr uint32_t IDESC_PV =
       PV8 ? ptx::instr_desc(1, 0, 0, 0, 1, 128, D)
@@ -396,20 +400,46 @@ __device__ __forceinline__ int row_max_masked(const uint32_t* v, int acc, int fi
   return acc;
 }
 
+// Per-token deltas: y_j = fp32(S_j * deltaK_j) in place (as fp32 bits) for NC
+// columns, returning max_j y_j over the unmasked keys (-inf if none).
+template <int NC, bool MASKED>
+__device__ __forceinline__ float row_scale_max(uint32_t* v, const float* dk, int first_key,
+                                               int limit) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < NC; j += 4) {
+    const float4 d = *reinterpret_cast<const float4*>(dk + j);
+    const float dd[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float y = __fmul_rn((float)(int)v[j + e], dd[e]);
+      v[j + e] = __float_as_uint(y);
+      if (!MASKED || first_key + j + e < limit) {
+        if (e & 1) m1 = fmaxf(m1, y);
+        else m0 = fmaxf(m0, y);
+      }
+    }
+  }
+  return fmaxf(m0, m1);
+}
+
 // Share of the exponentials computed by the FMA-pipe polynomial: one pair in
 // POLY_EVERY (0 = none; every 2^x on the special-function unit).
 constexpr int POLY_EVERY = 0;
 
 // p for NC columns: p = 2^fma(S, c, -m) (masked columns give 0); returns the
 // sum of p.  Results are written to p[].
-template <bool MASKED, int NC>
+template <bool MASKED, int NC, bool FIN = false>
 __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m, int first_key,
                                          int limit, float* p) {
   const float2 c2 = make_float2(c, c), n2 = make_float2(neg_m, neg_m);
   float2 s2a = make_float2(0.0f, 0.0f), s2b = make_float2(0.0f, 0.0f);
 #pragma unroll
   for (int i = 0; i < NC; i += 2) {
-    const float2 a = __ffma2_rn(s32x2_to_f32x2(v[i], v[i + 1]), c2, n2);
+    // FIN: v holds fp32 bit patterns (per-token dequantised scores), else int32 S
+    const float2 x = FIN ? make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1]))
+                         : s32x2_to_f32x2(v[i], v[i + 1]);
+    const float2 a = __ffma2_rn(x, c2, n2);
     float p0, p1;
     if (POLY_EVERY > 0 && (i / 2) % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1) {
       const float2 e = exp2_poly2(a);  // FMA-pipe 2^x for a share of the pairs
@@ -432,9 +462,10 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
   return s.x + s.y;
 }
 
-template <int D, bool PV8, bool BF16V>
-__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t tmem, int t) {
-  using C = Cfg<D, PV8>;
+template <int D, bool PV8, bool BF16V, bool TOK>
+__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t tmem, int t,
+                           const float* sKs) {
+  using C = Cfg<D, PV8, TOK>;
   using In = In16<BF16V>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
@@ -447,8 +478,10 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
   const int nsub = t == 0 ? w.nsub0 : w.nsub1;
   if (nsub == 0) return;
 
-  const float qd = __ldg(p.q_scale + w.qs_idx0 + t);
+  // deltaQ of this tile's block, or (per token) of this row
+  const float qd = __ldg(p.q_scale + (TOK ? (w.qs_idx0 + t) * BLK + r : w.qs_idx0 + t));
   float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f, c = 0.0f;
+  if constexpr (TOK) c = __fmul_rn(qd, p.kappa);  // fp32(deltaQ_i kappa), per row
   float o32[PV8 ? D : 1];
   if constexpr (PV8) {
 #pragma unroll
@@ -459,7 +492,7 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
   for (int i = 0; i < nsub; ++i) {
     const int b = i & 1;
     const uint32_t tS = tS0 + SUB * b;
-    if ((i & 1) == 0) {  // a new 128-key quantisation block: its delta
+    if (!TOK && (i & 1) == 0) {  // a new 128-key quantisation block: its delta
       const float kd = __ldg(p.k_scale + w.ks_idx0 + i / 2);
       c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
     }
@@ -468,6 +501,24 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
     const int key0 = i * SUB;
     const bool full_tile = (key0 + SUB <= w.n) && (!p.causal || key0 + SUB - 1 <= qt * BLK);
     float alpha, rowsum = 0.0f, m_new;
+    // The sub-tile's scaled maximum (-inf when no key of it is unmasked for
+    // this row).  Per token, S is first turned into y = fp32(S deltaK_j) in
+    // place; the K deltas came with the K tile (wait on its barrier).
+    auto tile_max = [&](uint32_t (&sv)[SUB], float& m_blk) -> bool {
+      if constexpr (TOK) {
+        const int j = i / 2;
+        if (!wait_bar(B, &B->k_full[j % C::NS], (j / C::NS) & 1, p.status, true)) return false;
+        const float* dk = sKs + (j % C::NS) * BLK + (i & 1) * SUB;
+        const float ym = full_tile ? row_scale_max<SUB, false>(sv, dk, key0, limit)
+                                   : row_scale_max<SUB, true>(sv, dk, key0, limit);
+        m_blk = ym == -INFINITY ? -INFINITY : __fmul_rn(ym, c);
+      } else {
+        const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
+                                   : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
+        m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+      }
+      return true;
+    };
 
     if constexpr (!PV8) {
       uint32_t sv[SUB];
@@ -475,17 +526,16 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
       for (int cc = 0; cc < SUB / 32; ++cc)
         ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
       ptx::tmem_wait_ld();
-      const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
-                                 : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
       // a sub-tile with no unmasked key for this row leaves the maximum unchanged
-      const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+      float m_blk;
+      if (!tile_max(sv, m_blk)) return;
       m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
       alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
 #pragma unroll
       for (int cc = 0; cc < SUB / 32; ++cc) {
         float pv[32];
-        rowsum += full_tile ? row_exp<false, 32>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv)
-                            : row_exp<true, 32>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv);
+        rowsum += full_tile ? row_exp<false, 32, TOK>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv)
+                            : row_exp<true, 32, TOK>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv);
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) packed[k] = In::pack(pv[2 * k], pv[2 * k + 1]);
@@ -518,17 +568,16 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
       for (int cc = 0; cc < SUB / 32; ++cc)
         ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
       ptx::tmem_wait_ld();
-      const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
-                                 : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
-      const float m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+      float m_blk;
+      if (!tile_max(sv, m_blk)) return;
       m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
       alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
       // P^ = e4m3(448 p), four per TMEM column, written over S
 #pragma unroll
       for (int cc = 0; cc < SUB / 16; ++cc) {
         float pv[16];
-        rowsum += full_tile ? row_exp<false, 16>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv)
-                            : row_exp<true, 16>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv);
+        rowsum += full_tile ? row_exp<false, 16, TOK>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv)
+                            : row_exp<true, 16, TOK>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv);
         uint32_t packed[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -615,17 +664,18 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
 
 // ---------------------------------------------------------------- kernel --
 
-template <int D, bool PV8, bool BF16V>
-__global__ void __launch_bounds__(Cfg<D, PV8>::THREADS, 1)
+template <int D, bool PV8, bool BF16V, bool TOK>
+__global__ void __launch_bounds__(Cfg<D, PV8, TOK>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using C = Cfg<D, PV8>;
+  using C = Cfg<D, PV8, TOK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + 2 * C::QT;
   uint8_t* sV = sK + C::NS * C::QT;
-  Bars* B = reinterpret_cast<Bars*>(sV + C::NS * C::VT);
+  float* sKs = reinterpret_cast<float*>(sV + C::NS * C::VT);  // TOK: [NS][128] K deltas
+  Bars* B = reinterpret_cast<Bars*>(sV + C::NS * (C::VT + C::KS));
   static_assert(sizeof(Bars) <= C::AUX, "aux layout");
 
   const Work w = decode_work(p);
@@ -666,13 +716,13 @@ __global__ void __launch_bounds__(Cfg<D, PV8>::THREADS, 1)
   if (wg == C::WG_CTRL) {
     ptx::setmaxnreg_dec<C::REG_CTRL>();
     if (warp == warp_tma) {
-      producer<D, PV8>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, p.status);
+      producer<D, PV8, TOK>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, sKs, p.k_scale, p.status);
     } else if (warp == warp_mma || warp == warp_mma + 1) {
-      mma_issuer<D, PV8, BF16V>(w, B, tmem, sQ, sK, sV, warp - warp_mma, p.status);
+      mma_issuer<D, PV8, BF16V, TOK>(w, B, tmem, sQ, sK, sV, warp - warp_mma, p.status);
     }
   } else {
     ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
-    softmax_wg<D, PV8, BF16V>(p, w, B, tmem, wg);
+    softmax_wg<D, PV8, BF16V, TOK>(p, w, B, tmem, wg, sKs);
   }
 
   ptx::tc_fence_before();
@@ -800,9 +850,9 @@ static CUtensorMapSwizzle swz_for(int row_bytes) {
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 }
 
-template <int D, bool PV8, bool BF16V>
+template <int D, bool PV8, bool BF16V, bool TOK>
 static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
-  using C = Cfg<D, PV8>;
+  using C = Cfg<D, PV8, TOK>;
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle cs = swz_for(D);
   if (!make_map3(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.q_codes, D, L.code_rows, L.code_z, D,
@@ -824,20 +874,27 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
     okv = make_map3(&tv, vdt, esz, L.v, D, L.p.H, L.T, (uint64_t)D * esz,
                     (uint64_t)D * esz * L.p.H, vbox0, 1, BLK, vs);
   if (!okv) return cudaErrorInvalidValue;
-  auto kern = attn_fwd_kernel<D, PV8, BF16V>;
+  auto kern = attn_fwd_kernel<D, PV8, BF16V, TOK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<L.grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, L.p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st) {
+template <bool TOK>
+static cudaError_t launch_attn_g(const AttnLaunch& L, cudaStream_t st) {
   if (L.D == 64) {
-    if (L.pv8) return launch_attn_t<64, true, false>(L, st);
-    return L.bf16v ? launch_attn_t<64, false, true>(L, st) : launch_attn_t<64, false, false>(L, st);
+    if (L.pv8) return launch_attn_t<64, true, false, TOK>(L, st);
+    return L.bf16v ? launch_attn_t<64, false, true, TOK>(L, st)
+                   : launch_attn_t<64, false, false, TOK>(L, st);
   }
-  if (L.pv8) return launch_attn_t<128, true, false>(L, st);
-  return L.bf16v ? launch_attn_t<128, false, true>(L, st) : launch_attn_t<128, false, false>(L, st);
+  if (L.pv8) return launch_attn_t<128, true, false, TOK>(L, st);
+  return L.bf16v ? launch_attn_t<128, false, true, TOK>(L, st)
+                 : launch_attn_t<128, false, false, TOK>(L, st);
+}
+
+cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st) {
+  return L.p.per_token ? launch_attn_g<true>(L, st) : launch_attn_g<false>(L, st);
 }
 
 template <int D>

@@ -11,6 +11,7 @@ struct AttnParams {
   int NB;                // dense: key blocks per head = ceil(N/128)
   int NPAIR;             // dense: query tile pairs per head = ceil(N/256)
   int causal;
+  int per_token;         // dense: one delta per token ([BH][NP] / [B*Hkv][NP]), not per block
   float kappa;           // fp32(sm_scale * log2 e)
   const float* q_scale;  // dense [BH][NB]; varlen [H][TBmax]
   const float* k_scale;

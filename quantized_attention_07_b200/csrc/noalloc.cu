@@ -31,7 +31,7 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                          uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
-                         cudaStream_t st);
+                         int per_token, cudaStream_t st);
 }  // namespace sage
 
 namespace {
@@ -111,6 +111,6 @@ extern "C" sage_status_t sage_quantize_noalloc(
                          fp8, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes,
                          v_scale, reinterpret_cast<unsigned long long*>(scratch + kSumOff),
                          reinterpret_cast<uint32_t*>(scratch + kAmaxOff), status,
-                         reinterpret_cast<unsigned int*>(scratch + kSyncOff), sage::QUANT_Q | sage::QUANT_KV, st);
+                         reinterpret_cast<unsigned int*>(scratch + kSyncOff), sage::QUANT_Q | sage::QUANT_KV, 0, st);
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

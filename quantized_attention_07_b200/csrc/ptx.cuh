@@ -140,6 +140,16 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
+// The same without an L2 eviction hint.
+__device__ __forceinline__ void bulk_load_plain(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                                uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1], %2, [%3];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Named barrier 1 over the first `n` threads of the CTA (a multiple of 32),
 // optionally AND-reducing a predicate.
 template <int N>

@@ -546,6 +546,49 @@ __device__ __forceinline__ float regs_absmax_sub(const uint4 (&u)[Tile<D>::NIT],
   return a;
 }
 
+// Per-token quantiser: every row gets its own delta, the max |x - mean| over
+// its D channels (held by the D/8 consecutive lanes that own the row, combined
+// with shuffles); codes as in the block quantiser.  Padding rows get code 0
+// and delta 0.  delta[code_row0 + r] receives the row deltas.
+template <int D, bool BF16, bool SUB, bool FULL>
+__device__ __forceinline__ void regs_codes_per_row(const uint4 (&u)[Tile<D>::NIT], int rows,
+                                                   const float (&mean)[8], int8_t* codes,
+                                                   float* delta, long long code_row0) {
+  using T = Tile<D>;
+  const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
+  float2 nm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) nm[e] = make_float2(-mean[2 * e], -mean[2 * e + 1]);
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i) {
+    const int r = r0 + i * T::RS;
+    const bool valid = FULL || r < rows;
+    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+    float2 f[4];
+    float a = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      f[e] = In16<BF16>::to_float2(w[e]);
+      if constexpr (SUB) f[e] = __fadd2_rn(f[e], nm[e]);
+      a = fmaxf(a, fmaxf(fabsf(f[e].x), fabsf(f[e].y)));
+    }
+    if (!valid) a = 0.0f;
+#pragma unroll
+    for (int o = T::CPR / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const float s = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    float2 y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      y[e] = make_float2(__fadd_rn(__fmul_rn(f[e].x, s), kMagic),
+                         __fadd_rn(__fmul_rn(f[e].y, s), kMagic));
+    uint2 out = make_uint2(low_bytes4(y[0].x, y[0].y, y[1].x, y[1].y),
+                           low_bytes4(y[2].x, y[2].y, y[3].x, y[3].y));
+    if (!valid) out = make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(codes + (code_row0 + r) * D + 8 * c) = out;
+    if (c == 0) delta[code_row0 + r] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  }
+}
+
 // Exact sums of rint(x * 2^24) over the thread's rows, per channel, as two
 // fp32 sums: hi = sum of h = rint(16x), fr = sum of d = 16x - h, so that the
 // total is 2^20 (hi + fr).  For |x| < 2^16: |h| <= 2^20 and d is exact with
@@ -600,7 +643,7 @@ __device__ __forceinline__ void release_slot(uint64_t* empty) {
 // sync[0]: work counter; sync[1 + u]: pass-1 blocks of head u completed.
 template <int D, bool BF16, bool FP8>
 __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) quant_stream_kernel(
-    SeqLayout L, int U, int lag, int parts, const void* __restrict__ q,
+    SeqLayout L, int U, int lag, int parts, int tok, const void* __restrict__ q,
     const void* __restrict__ k, const void* __restrict__ v, int8_t* __restrict__ q_codes,
     float* __restrict__ q_scale, int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
     float* __restrict__ k_mean, uint8_t* __restrict__ v_codes, float* __restrict__ v_scale,
@@ -768,8 +811,12 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
 
       if (pass == 1) {
         const int tk = has_q ? 1 : 0;  // slab index of K (V follows it)
-        // Q: per-block quantiser
-        if (has_q) {
+        // Q: per-block (or per-token) quantiser
+        if (has_q && tok) {
+          take(0);
+          if (full_blk) regs_codes_per_row<D, BF16, false, true>(rg, P.rows, zero8, q_codes, q_scale, P.code_row0);
+          else regs_codes_per_row<D, BF16, false, false>(rg, P.rows, zero8, q_codes, q_scale, P.code_row0);
+        } else if (has_q) {
           take(0);
           const float amax = consumer_block_max(regs_absmax<D, BF16>(rg), red, par);
           codes(amax, zero8, q_codes, std::false_type{});
@@ -865,12 +912,17 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
 #pragma unroll
           for (int e = 0; e < 8; ++e) m[e] = s_side[slot0][8 * c + e];
           take(0);
+          if (tok) {  // one delta per token: no block-wide maximum
+            if (full_blk) regs_codes_per_row<D, BF16, true, true>(rg, P.rows, m, k_codes, k_scale, P.code_row0);
+            else regs_codes_per_row<D, BF16, true, false>(rg, P.rows, m, k_codes, k_scale, P.code_row0);
+          } else {
           const float a = full_blk ? regs_absmax_sub<D, BF16, true>(rg, P.rows, m)
                                    : regs_absmax_sub<D, BF16, false>(rg, P.rows, m);
           const float amax = consumer_block_max(a, red, par);
           codes(amax, m, k_codes, std::true_type{});
           if (threadIdx.x == 0)
             k_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+          }
         }
         // V: FP8 E4M3 codes with a per-channel scale
         if constexpr (FP8) {
@@ -961,7 +1013,7 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
                                   int8_t* k_codes, float* k_scale, float* k_mean,
                                   uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                                   uint32_t* v_amax, uint32_t* status, unsigned int* sync,
-                                  int parts, cudaStream_t st) {
+                                  int parts, int tok, cudaStream_t st) {
   const int U = grid.y, NB = grid.x;
   const long long items = ((parts & PART_KV) ? 2LL : 1LL) * U * NB;
   // Dense: one persistent launch in an L2-friendly order (its work counter is
@@ -992,11 +1044,11 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
     if (lag > U) lag = U;
     if (lag < 1) lag = 1;
     quant_stream_kernel<D, BF16, FP8><<<blocks, S::THREADS, S::SMEM, st>>>(
-        L, U, (int)lag, parts, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes,
+        L, U, (int)lag, parts, tok, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes,
         v_scale, k_sum, v_amax, status, sync);
     return cudaGetLastError();
   }
-  if (parts != (PART_Q | PART_KV)) return cudaErrorNotSupported;
+  if (parts != (PART_Q | PART_KV) || tok) return cudaErrorNotSupported;
   quant_pass1_kernel<D, BF16, FP8>
       <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status);
   cudaError_t e = cudaGetLastError();
@@ -1009,18 +1061,19 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
 // Runs both passes.  k_sum / v_amax and (dense) sync[0 .. units] must be zero
 // on entry (the caller clears them on the stream).  grid = (blocks per head or
 // TBmax, units = B*H or H).  parts: QUANT_Q and/or QUANT_KV (both unless the
-// query and key/value heads differ).
+// query and key/value heads differ).  per_token: one delta per token (dense
+// only; deltas indexed like the code rows).
 cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool fp8,
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                          uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
-                         cudaStream_t st) {
+                         int per_token, cudaStream_t st) {
   static_assert(QUANT_Q == PART_Q && QUANT_KV == PART_KV, "part flags");
 #define SAGE_Q(DD, BB, FF)                                                                    \
   return launch_quant_t<DD, BB, FF>(L, grid, q, k, v, q_codes, q_scale, k_codes, k_scale,    \
                                     k_mean, v_codes, v_scale, k_sum, v_amax, status, sync,   \
-                                    parts, st)
+                                    parts, per_token, st)
   if (D == 64) {
     if (bf16) { if (fp8) SAGE_Q(64, true, true); else SAGE_Q(64, true, false); }
     else { if (fp8) SAGE_Q(64, false, true); else SAGE_Q(64, false, false); }

@@ -53,6 +53,7 @@ class Workload:
     len_hi: int = 0
     seed: int = 0
     Hkv: int = 0                # key/value heads (grouped-query attention); 0: = H
+    qk_gran: str = "block"      # Q/K deltas per 128-token block or per token
 
     @property
     def kv_heads(self) -> int:
@@ -83,6 +84,11 @@ WORKLOADS = {
     # heads, the repeat_kv layout of the DeepSeek-VL2 page's attention code)
     "llm_gqa_8k": Workload("llm_gqa_8k", B=1, H=32, N=8192, D=128, dtype="bf16", causal=True,
                            pv_mode="fp16", bias_sigma=3.0, seed=20260006, Hkv=8),
+    # the video-DiT shape with one Q/K delta per token (the accurate option for
+    # channel outliers)
+    "dit_8k_fp8_tok": Workload("dit_8k_fp8_tok", B=1, H=24, N=8192, D=64, dtype="fp16",
+                               causal=False, pv_mode="fp8", bias_sigma=3.0, outlier_p=0.01,
+                               outlier_scale=20.0, seed=20260003, qk_gran="token"),
 }
 
 

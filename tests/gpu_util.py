@@ -21,9 +21,10 @@ def half_ulp(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
     return 0.5 * np.exp2(e - mant)
 
 
-def gpu_quantize_dense(q, k, v, pv_mode):
+def gpu_quantize_dense(q, k, v, pv_mode, qk_gran="block"):
     dev = torch.device("cuda")
-    qz = sage.quantize(q.to(dev), k.to(dev), v.to(dev) if v is not None else None, pv_mode)
+    qz = sage.quantize(q.to(dev), k.to(dev), v.to(dev) if v is not None else None, pv_mode,
+                       qk_gran=qk_gran)
     torch.cuda.synchronize()
     sage.sync_status()
     return qz
@@ -66,10 +67,11 @@ def compare_quant_varlen(qz_gpu, qz_ref, cu, pv_mode):
         assert_same("v codes", c(qz_gpu.v_codes), qz_ref.v_codes)
 
 
-def run_dense(q, k, v, causal, pv_mode, out_dtype=torch.float32, sm_scale=None):
+def run_dense(q, k, v, causal, pv_mode, out_dtype=torch.float32, sm_scale=None,
+              qk_gran="block"):
     dev = torch.device("cuda")
     out = sage.attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=causal, sm_scale=sm_scale,
-                        pv_mode=pv_mode, out_dtype=out_dtype)
+                        pv_mode=pv_mode, out_dtype=out_dtype, qk_gran=qk_gran)
     torch.cuda.synchronize()
     sage.sync_status()
     return out.cpu()
@@ -100,23 +102,23 @@ def cosine(a: np.ndarray, b: np.ndarray) -> float:
 
 
 def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
-                         ref_cos_bar=0.999):
+                         ref_cos_bar=0.999, qk_gran="block"):
     """GPU fp32 output vs the oracle's emulation (max-abs tolerance) and the fp64
     reference (cosine).  Also checks a 16-bit output run.  Returns a stats dict.
     Dense k, v with fewer heads than q run grouped-query attention on the GPU;
     the oracle sees them repeated (its repeat_kv)."""
     D = q.shape[-1]
     if cu is None:
-        out32 = run_dense(q, k, v, causal, pv_mode, torch.float32, sm_scale)
-        out16 = run_dense(q, k, v, causal, pv_mode, q.dtype, sm_scale)
+        out32 = run_dense(q, k, v, causal, pv_mode, torch.float32, sm_scale, qk_gran)
+        out16 = run_dense(q, k, v, causal, pv_mode, q.dtype, sm_scale, qk_gran)
         if k.shape[1] != q.shape[1]:
             g = q.shape[1] // k.shape[1]
             k, v = heads.repeat_kv(k, g), heads.repeat_kv(v, g)
     else:
         out32 = run_varlen(q, k, v, cu, causal, pv_mode, torch.float32, sm_scale)
         out16 = run_varlen(q, k, v, cu, causal, pv_mode, q.dtype, sm_scale)
-    qz = heads.quantize(q, k, v, cu, pv_mode)
-    emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale)
+    qz = heads.quantize(q, k, v, cu, pv_mode, gran=qk_gran)
+    emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran)
     ref = heads.reference_rows(q, k, v, cu, picks, causal, sm_scale)
     E = np.stack([emu[p] for p in picks])
     R = np.stack([ref[p] for p in picks])

@@ -49,7 +49,7 @@ def test_quantize_bit_exact_full_workloads(name):
     are checked through the attention tests in test_gpu_gqa.py.)"""
     wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl)
-    ref = heads.quantize(inp.q, inp.k, inp.v, inp.cu_seqlens, wl.pv_mode)
+    ref = heads.quantize(inp.q, inp.k, inp.v, inp.cu_seqlens, wl.pv_mode, gran=wl.qk_gran)
     if wl.varlen:
         dev = torch.device("cuda")
         qz = sage.quantize_varlen(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev),
@@ -58,7 +58,7 @@ def test_quantize_bit_exact_full_workloads(name):
         sage.sync_status()
         U.compare_quant_varlen(qz, ref, inp.cu_seqlens, wl.pv_mode)
     else:
-        qz = U.gpu_quantize_dense(inp.q, inp.k, inp.v, wl.pv_mode)
+        qz = U.gpu_quantize_dense(inp.q, inp.k, inp.v, wl.pv_mode, wl.qk_gran)
         U.compare_quant_dense(qz, ref, wl.pv_mode)
 
 
@@ -169,5 +169,5 @@ def test_attention_full_workloads_sampled_rows(name):
         flat = W.sample_rows([wl.N] * wl.B, wl.H, 512, seed=wl.seed)
         picks = flat
     stats = U.check_against_oracle(inp.q, inp.k, inp.v, inp.cu_seqlens, wl.causal, wl.pv_mode,
-                                   picks)
+                                   picks, qk_gran=wl.qk_gran)
     print(name, stats)
