@@ -274,15 +274,16 @@ def run_ours(args, rank, world, local):
         hcu = inp.cu_seqlens.pin_memory() if inp.cu_seqlens is not None else None
 
         def e2e_step():
-            dq, dk, dv = (x.to(dev, non_blocking=True) for x in (hq, hk, hv))
             if wl.varlen:
+                dq, dk, dv = (x.to(dev, non_blocking=True) for x in (hq, hk, hv))
                 dcu = hcu.to(dev, non_blocking=True)
                 o = sage.attn_fwd_varlen(dq, dk, dv, dcu, max(inp.seqlens), causal=wl.causal,
                                          pv_mode=wl.pv_mode, workspace=ws)
+                hout.copy_(o, non_blocking=True)
             else:
-                o = sage.attn_fwd(dq, dk, dv, causal=wl.causal, pv_mode=wl.pv_mode, workspace=ws,
-                                  qk_gran=wl.qk_gran)
-            hout.copy_(o, non_blocking=True)
+                # uploads, compute and downloads of independent head groups overlapped
+                sage.attn_fwd_host(hq, hk, hv, hout, causal=wl.causal, pv_mode=wl.pv_mode,
+                                   qk_gran=wl.qk_gran, device=dev)
 
         for _ in range(2):
             e2e_step()
