@@ -185,6 +185,20 @@ sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, 
                                    float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
                                    void* stream);
 
+/*
+ * Grouped-query variant of sage_attn_fwd_varlen: q, out are [T, H, D]; k, v
+ * are [T, Hkv, D] with Hkv dividing H; query head h reads key/value head
+ * h / (H / Hkv) of its sequence (the repeat_kv grouping, see
+ * sage_attn_fwd_gqa).  ws: at least sage_workspace_bytes_varlen_gqa(...).
+ */
+size_t sage_workspace_bytes_varlen_gqa(int total_tokens, int batch, int H, int Hkv, int D,
+                                       int pv_mode);
+sage_status_t sage_attn_fwd_varlen_gqa(const void* q, const void* k, const void* v, void* out,
+                                       int in_dt, int out_dt, const int32_t* cu_seqlens,
+                                       int batch, int max_seqlen, int total_tokens, int H,
+                                       int Hkv, int D, int causal, float sm_scale, int pv_mode,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------ the two stages, separately -- */
 
 /*

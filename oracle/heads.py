@@ -68,6 +68,16 @@ def repeat_kv(x: torch.Tensor, groups: int) -> torch.Tensor:
     return out
 
 
+def repeat_kv_packed(x: torch.Tensor, groups: int) -> torch.Tensor:
+    """repeat_kv for packed [T, Hkv, D] tensors: head h of the result is key/value
+    head h // groups."""
+    T, Hkv, D = x.shape
+    out = torch.empty((T, Hkv * groups, D), dtype=x.dtype)
+    for h in range(Hkv * groups):
+        out[:, h] = x[:, h // groups]
+    return out
+
+
 def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
              cu_seqlens: Optional[torch.Tensor] = None, pv_mode: str = "fp16",
              gran: str = "block") -> Quantized:

@@ -261,25 +261,40 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     pv_mode: str = "fp16", out_dtype: Optional[torch.dtype] = None,
                     out: Optional[torch.Tensor] = None,
                     workspace: Optional[Workspace] = None) -> torch.Tensor:
-    """SageAttention forward over packed [T, H, D] tensors with int32 cu_seqlens."""
+    """SageAttention forward over packed [T, H, D] tensors with int32 cu_seqlens.
+    k, v may be [T, Hkv, D] with Hkv dividing H (grouped-query attention)."""
     _need_cuda_contig(q, k, v, cu_seqlens)
-    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must share one [T, H, D] shape")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("q must be [T, H, D] and k, v one [T, Hkv, D] shape")
     if cu_seqlens.dtype != torch.int32:
         raise ValueError("cu_seqlens must be int32")
     T, H, D = q.shape
+    Hkv = k.shape[1]
+    if (k.shape[0], k.shape[2]) != (T, D) or H % Hkv:
+        raise ValueError("k, v must be [T, Hkv, D] with Hkv dividing H")
     batch = cu_seqlens.numel() - 1
     od = out_dtype or q.dtype
     if out is None:
         out = torch.empty((T, H, D), dtype=od, device=q.device)
     _need_cuda_contig(out)
     mode = _pv(pv_mode)
-    ws = _workspace(q.device, workspace_bytes_varlen(T, batch, H, D, pv_mode), workspace)
-    _check(_lib.load().sage_attn_fwd_varlen(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype), _dtype_code(out.dtype, True),
-        _ptr(cu_seqlens), batch, int(max_seqlen), T, H, D, int(bool(causal)),
-        float(sm_scale) if sm_scale else 0.0, mode, ws.ptr, ws.nbytes, _stream(q.device)),
-        "sage_attn_fwd_varlen")
+    lib = _lib.load()
+    scale = float(sm_scale) if sm_scale else 0.0
+    if Hkv == H:
+        ws = _workspace(q.device, workspace_bytes_varlen(T, batch, H, D, pv_mode), workspace)
+        _check(lib.sage_attn_fwd_varlen(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+            _dtype_code(out.dtype, True), _ptr(cu_seqlens), batch, int(max_seqlen), T, H, D,
+            int(bool(causal)), scale, mode, ws.ptr, ws.nbytes, _stream(q.device)),
+            "sage_attn_fwd_varlen")
+    else:
+        ws = _workspace(q.device, int(lib.sage_workspace_bytes_varlen_gqa(T, batch, H, Hkv, D,
+                                                                          mode)), workspace)
+        _check(lib.sage_attn_fwd_varlen_gqa(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+            _dtype_code(out.dtype, True), _ptr(cu_seqlens), batch, int(max_seqlen), T, H, Hkv, D,
+            int(bool(causal)), scale, mode, ws.ptr, ws.nbytes, _stream(q.device)),
+            "sage_attn_fwd_varlen_gqa")
     return out
 
 

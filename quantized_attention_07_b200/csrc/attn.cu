@@ -180,18 +180,19 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
     const int npairs = __ldg(p.pair_off + s + 1) - __ldg(p.pair_off + s);
     pair = npairs - 1 - (item - __ldg(p.pair_off + s));  // diagonal-heavy pairs first
     const int blk0 = __ldg(p.blk_off + s);
+    const int hk = h / (p.H / p.Hkv);  // its key/value head (grouped-query)
     w.code_z = h;
-    w.k_z = h;
+    w.k_z = hk;
     w.q_y0 = (blk0 + 2 * pair) * BLK;
     w.k_y0 = blk0 * BLK;
-    w.v_y0 = h;
+    w.v_y0 = hk;
     w.v_z0 = tok0;
     w.v_tok_on_z = 1;
     w.qs_idx0 = (long long)h * p.TBmax + blk0 + 2 * pair;
-    w.ks_idx0 = (long long)h * p.TBmax + blk0;
+    w.ks_idx0 = (long long)hk * p.TBmax + blk0;
     w.out_row0 = (long long)tok0 * p.H + h;
     w.out_stride = p.H;
-    w.vs_idx = (long long)s * p.H + h;
+    w.vs_idx = (long long)s * p.Hkv + hk;
   }
   w.valid = 1;
   w.n = n;
@@ -871,8 +872,8 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
     okv = make_map3(&tv, vdt, esz, L.v, D, L.p.N, L.code_z_kv, (uint64_t)D * esz,
                     (uint64_t)D * esz * L.p.N, vbox0, BLK, 1, vs);
   else
-    okv = make_map3(&tv, vdt, esz, L.v, D, L.p.H, L.T, (uint64_t)D * esz,
-                    (uint64_t)D * esz * L.p.H, vbox0, 1, BLK, vs);
+    okv = make_map3(&tv, vdt, esz, L.v, D, L.code_z_kv, L.T, (uint64_t)D * esz,
+                    (uint64_t)D * esz * L.code_z_kv, vbox0, 1, BLK, vs);
   if (!okv) return cudaErrorInvalidValue;
   auto kern = attn_fwd_kernel<D, PV8, BF16V, TOK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

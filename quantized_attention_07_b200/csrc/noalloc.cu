@@ -111,6 +111,7 @@ extern "C" sage_status_t sage_quantize_noalloc(
                          fp8, q, k, v, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes,
                          v_scale, reinterpret_cast<unsigned long long*>(scratch + kSumOff),
                          reinterpret_cast<uint32_t*>(scratch + kAmaxOff), status,
-                         reinterpret_cast<unsigned int*>(scratch + kSyncOff), sage::QUANT_Q | sage::QUANT_KV, 0, st);
+                         reinterpret_cast<unsigned int*>(scratch + kSyncOff),
+                         sage::QUANT_Q | sage::QUANT_KV, 0, st);
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

@@ -178,20 +178,23 @@ __device__ __forceinline__ void pass1_block(
     const BlockPos& P, const void* __restrict__ q, const void* __restrict__ k,
     const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
     unsigned long long* __restrict__ k_sum, uint32_t* __restrict__ v_amax,
-    uint32_t* __restrict__ status) {
+    uint32_t* __restrict__ status, int parts) {
   using T = Tile<D>;
   __shared__ float red[THREADS / 32];
   __shared__ long long red64[THREADS / 32][D];
   const int c = threadIdx.x % T::CPR;
   const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const bool has_q = (parts & QUANT_Q) != 0, has_kv = (parts & QUANT_KV) != 0;
 
   uint4 rq[T::NIT], rk[T::NIT], rv[FP8 ? T::NIT : 1];
-  load_raw<D>(q, P, rq);
-  load_raw<D>(k, P, rk);
-  if constexpr (FP8) load_raw<D>(v, P, rv);
+  if (has_q) load_raw<D>(q, P, rq);
+  if (has_kv) load_raw<D>(k, P, rk);
+  if constexpr (FP8) {
+    if (has_kv) load_raw<D>(v, P, rv);
+  }
 
   // --- Q: per-block quantiser
-  {
+  if (has_q) {
     float x[T::NIT][8];
     to_float<D, BF16>(rq, x);
     float a = 0.0f;
@@ -205,7 +208,7 @@ __device__ __forceinline__ void pass1_block(
   }
 
   // --- K: exact fixed-point channel sums
-  {
+  if (has_kv) {
     float x[T::NIT][8];
     to_float<D, BF16>(rk, x);
     long long acc[8];
@@ -238,7 +241,7 @@ __device__ __forceinline__ void pass1_block(
   }
 
   // --- V: per-channel max|v| (FP8 P.V only)
-  if constexpr (FP8) {
+  if constexpr (FP8) if (has_kv) {
     float x[T::NIT][8];
     to_float<D, BF16>(rv, x);
     float m[8];
@@ -273,10 +276,10 @@ __global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
     SeqLayout L, const void* __restrict__ q, const void* __restrict__ k,
     const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
     unsigned long long* __restrict__ k_sum, uint32_t* __restrict__ v_amax,
-    uint32_t* __restrict__ status) {
+    uint32_t* __restrict__ status, int parts) {
   BlockPos P;
   if (!block_pos(L, P)) return;
-  pass1_block<D, BF16, FP8>(P, q, k, v, q_codes, q_scale, k_sum, v_amax, status);
+  pass1_block<D, BF16, FP8>(P, q, k, v, q_codes, q_scale, k_sum, v_amax, status, parts);
 }
 
 // ------------------------------------------------------------------ pass 2 --
@@ -814,8 +817,12 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
         // Q: per-block (or per-token) quantiser
         if (has_q && tok) {
           take(0);
-          if (full_blk) regs_codes_per_row<D, BF16, false, true>(rg, P.rows, zero8, q_codes, q_scale, P.code_row0);
-          else regs_codes_per_row<D, BF16, false, false>(rg, P.rows, zero8, q_codes, q_scale, P.code_row0);
+          if (full_blk)
+            regs_codes_per_row<D, BF16, false, true>(rg, P.rows, zero8, q_codes, q_scale,
+                                                     P.code_row0);
+          else
+            regs_codes_per_row<D, BF16, false, false>(rg, P.rows, zero8, q_codes, q_scale,
+                                                      P.code_row0);
         } else if (has_q) {
           take(0);
           const float amax = consumer_block_max(regs_absmax<D, BF16>(rg), red, par);
@@ -913,8 +920,12 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
           for (int e = 0; e < 8; ++e) m[e] = s_side[slot0][8 * c + e];
           take(0);
           if (tok) {  // one delta per token: no block-wide maximum
-            if (full_blk) regs_codes_per_row<D, BF16, true, true>(rg, P.rows, m, k_codes, k_scale, P.code_row0);
-            else regs_codes_per_row<D, BF16, true, false>(rg, P.rows, m, k_codes, k_scale, P.code_row0);
+            if (full_blk)
+              regs_codes_per_row<D, BF16, true, true>(rg, P.rows, m, k_codes, k_scale,
+                                                      P.code_row0);
+            else
+              regs_codes_per_row<D, BF16, true, false>(rg, P.rows, m, k_codes, k_scale,
+                                                       P.code_row0);
           } else {
           const float a = full_blk ? regs_absmax_sub<D, BF16, true>(rg, P.rows, m)
                                    : regs_absmax_sub<D, BF16, false>(rg, P.rows, m);
@@ -1017,8 +1028,8 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
   const int U = grid.y, NB = grid.x;
   const long long items = ((parts & PART_KV) ? 2LL : 1LL) * U * NB;
   // Dense: one persistent launch in an L2-friendly order (its work counter is
-  // 32-bit).  Variable-length batches, and any larger problem: two launches,
-  // which handle Q and K (, V) together only.
+  // 32-bit).  Variable-length batches, and any larger problem: two launches
+  // (pass 1 alone for Q only; per-block deltas only).
   if (!L.varlen && items + 4096 < (1LL << 31)) {
     using S = Stream<D>;
     static int sms = 0;  // per template instance
@@ -1048,11 +1059,11 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
         v_scale, k_sum, v_amax, status, sync);
     return cudaGetLastError();
   }
-  if (parts != (PART_Q | PART_KV) || tok) return cudaErrorNotSupported;
+  if (tok) return cudaErrorNotSupported;
   quant_pass1_kernel<D, BF16, FP8>
-      <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status);
+      <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status, parts);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || !(parts & PART_KV)) return e;
   quant_pass2_kernel<D, BF16, FP8><<<grid, THREADS, 0, st>>>(L, k, v, k_sum, v_amax, k_codes,
                                                              k_scale, k_mean, v_codes, v_scale);
   return cudaGetLastError();

@@ -114,12 +114,16 @@ extern "C" sage_status_t sage_attn_ref_rows(const void* q, const void* k, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dim3 grid(n_rows), block(32 * sage::RR_WARPS);
   const bool bf16 = in_dt == SAGE_BF16;
+#define SAGE_RR(DD, BB)                                                                  \
+  sage::ref_rows_kernel<DD, BB><<<grid, block, 0, st>>>(q16, k16, v16, B, H, Hkv, N, causal, \
+                                                        scale, rows, n_rows, out)
   if (D == 64) {
-    if (bf16) sage::ref_rows_kernel<64, true><<<grid, block, 0, st>>>(q16, k16, v16, B, H, Hkv, N, causal, scale, rows, n_rows, out);
-    else sage::ref_rows_kernel<64, false><<<grid, block, 0, st>>>(q16, k16, v16, B, H, Hkv, N, causal, scale, rows, n_rows, out);
+    if (bf16) SAGE_RR(64, true);
+    else SAGE_RR(64, false);
   } else {
-    if (bf16) sage::ref_rows_kernel<128, true><<<grid, block, 0, st>>>(q16, k16, v16, B, H, Hkv, N, causal, scale, rows, n_rows, out);
-    else sage::ref_rows_kernel<128, false><<<grid, block, 0, st>>>(q16, k16, v16, B, H, Hkv, N, causal, scale, rows, n_rows, out);
+    if (bf16) SAGE_RR(128, true);
+    else SAGE_RR(128, false);
   }
+#undef SAGE_RR
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

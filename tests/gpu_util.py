@@ -117,6 +117,9 @@ def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
     else:
         out32 = run_varlen(q, k, v, cu, causal, pv_mode, torch.float32, sm_scale)
         out16 = run_varlen(q, k, v, cu, causal, pv_mode, q.dtype, sm_scale)
+        if k.shape[1] != q.shape[1]:
+            g = q.shape[1] // k.shape[1]
+            k, v = heads.repeat_kv_packed(k, g), heads.repeat_kv_packed(v, g)
     qz = heads.quantize(q, k, v, cu, pv_mode, gran=qk_gran)
     emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran)
     ref = heads.reference_rows(q, k, v, cu, picks, causal, sm_scale)

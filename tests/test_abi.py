@@ -122,3 +122,13 @@ def test_grouped_query_sizes_and_validation(lib):
     assert f(*bad) == 1
     small = list(args); small[15] = lib.sage_workspace_bytes_gqa(1, 8, 2, 256, 64, 0) - 1
     assert f(*small) == 3
+
+
+def test_grouped_varlen_sizes_and_validation(lib):
+    full = lib.sage_workspace_bytes_varlen(5000, 4, 8, 128, 1)
+    assert lib.sage_workspace_bytes_varlen_gqa(5000, 4, 8, 8, 128, 1) == full
+    assert 0 < lib.sage_workspace_bytes_varlen_gqa(5000, 4, 8, 2, 128, 1) < full
+    assert lib.sage_workspace_bytes_varlen_gqa(5000, 4, 8, 3, 128, 1) == 0
+    f = lib.sage_attn_fwd_varlen_gqa
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 4, 100, 300, 8, 3, 64, 0, 0.0, 0, FAKE, 1 << 40,
+             None) == 1

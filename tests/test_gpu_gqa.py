@@ -71,3 +71,25 @@ def test_gqa_sageattn_shim_needs_no_repeat():
                         is_causal=True)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("causal,pv_mode,dtype,H,Hkv", [(True, "fp16", "bf16", 8, 2),
+                                                       (False, "fp8", "fp16", 4, 1),
+                                                       (True, "fp8", "bf16", 6, 3)])
+def test_varlen_gqa_equals_repeated_and_oracle(causal, pv_mode, dtype, H, Hkv):
+    lens = [1, 300, 129, 0, 517]
+    D = 128 if pv_mode == "fp8" else 64
+    q, k, v, cu = W.make_varlen(lens, H, D, dtype, seed=H * 7 + Hkv)
+    k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
+    dev = torch.device("cuda")
+    g = H // Hkv
+    kr, vr = heads.repeat_kv_packed(k, g), heads.repeat_kv_packed(v, g)
+    a = sage.attn_fwd_varlen(q.to(dev), k.to(dev), v.to(dev), cu.to(dev), max(lens), causal=causal,
+                             pv_mode=pv_mode, out_dtype=torch.float32)
+    b = sage.attn_fwd_varlen(q.to(dev), kr.to(dev), vr.to(dev), cu.to(dev), max(lens),
+                             causal=causal, pv_mode=pv_mode, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    sage.sync_status()
+    assert torch.equal(a, b)
+    picks = [(s, h, i) for s, n in enumerate(lens) for h in range(H) for i in range(0, n, 3)]
+    U.check_against_oracle(q, k, v, cu, causal, pv_mode, picks)
