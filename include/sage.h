@@ -76,7 +76,7 @@ typedef enum {
  * SageAttention v1 item (1): per-block or per-token quantisation of q, k). */
 typedef enum {
   SAGE_QK_PER_BLOCK = 0, /* one delta per 128-token block (and head)             */
-  SAGE_QK_PER_TOKEN = 1  /* one delta per token; dense inputs only                */
+  SAGE_QK_PER_TOKEN = 1  /* one delta per token                                   */
 } sage_qk_gran_t;
 
 /* Token count of one quantisation block and of one attention key/query tile. */
@@ -198,6 +198,20 @@ sage_status_t sage_attn_fwd_varlen_gqa(const void* q, const void* k, const void*
                                        int batch, int max_seqlen, int total_tokens, int H,
                                        int Hkv, int D, int causal, float sm_scale, int pv_mode,
                                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * General variable-length forward pass: grouped-query heads (as
+ * sage_attn_fwd_varlen_gqa) and the Q/K delta granularity qk_gran (as
+ * sage_attn_fwd_ex; per token, every packed token has its own Q and K delta).
+ *   ws : at least sage_workspace_bytes_varlen_ex(...).
+ */
+size_t sage_workspace_bytes_varlen_ex(int total_tokens, int batch, int H, int Hkv, int D,
+                                      int pv_mode, int qk_gran);
+sage_status_t sage_attn_fwd_varlen_ex(const void* q, const void* k, const void* v, void* out,
+                                      int in_dt, int out_dt, const int32_t* cu_seqlens, int batch,
+                                      int max_seqlen, int total_tokens, int H, int Hkv, int D,
+                                      int causal, float sm_scale, int pv_mode, int qk_gran,
+                                      void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------ the two stages, separately -- */
 

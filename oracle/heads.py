@@ -81,14 +81,13 @@ def repeat_kv_packed(x: torch.Tensor, groups: int) -> torch.Tensor:
 def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
              cu_seqlens: Optional[torch.Tensor] = None, pv_mode: str = "fp16",
              gran: str = "block") -> Quantized:
-    """gran "block": one delta per 128-token block (deltas [B,H,NB]); "token"
-    (dense only): one delta per token, the quantiser applied to one-row blocks
-    (deltas [B,H,NP], padding rows 0)."""
+    """gran "block": one delta per 128-token block (deltas [B,H,NB] dense,
+    [H, TB] varlen); "token": one delta per token, the quantiser applied to
+    one-row blocks, stored like the code rows (deltas [B,H,NP] dense,
+    [H, TB*128] varlen; padding rows 0)."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     status = 0
     tok = gran == "token"
-    if tok and cu is not None:
-        raise ValueError("per-token scales are built for dense inputs")
     if cu is None:
         B, H, N, D = q.shape
         NB = (N + BLK - 1) // BLK
@@ -121,19 +120,28 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
     nblk = [(cu[s + 1] - cu[s] + BLK - 1) // BLK for s in range(S)]
     boff = np.concatenate([[0], np.cumsum(nblk)]).astype(np.int64)
     TB = int(boff[-1])
-    qc = np.zeros((H, TB * BLK, D), np.int8); qd = np.zeros((H, TB), np.float32)
+    qc = np.zeros((H, TB * BLK, D), np.int8)
+    qd = np.zeros((H, TB * BLK if tok else TB), np.float32)
     kc = np.zeros_like(qc); kd = np.zeros_like(qd)
     ks = np.zeros((S, H, D), np.int64); km = np.zeros((S, H, D), np.float32)
     for s, h, x in _heads(q, cu):
         r0 = boff[s] * BLK
-        c, d = quant_head(x, None, BLK)
-        qc[h, r0:r0 + c.shape[0]] = c; qd[h, boff[s]:boff[s + 1]] = d
+        if tok:
+            c, d = quant_head(x, None, 1)
+            qc[h, r0:r0 + c.shape[0]] = c; qd[h, r0:r0 + d.shape[0]] = d
+        else:
+            c, d = quant_head(x, None, BLK)
+            qc[h, r0:r0 + c.shape[0]] = c; qd[h, boff[s]:boff[s + 1]] = d
     for s, h, x in _heads(k, cu):
         ks[s, h], km[s, h], st = k_mean(x)
         status |= st
         r0 = boff[s] * BLK
-        c, d = quant_head(x, km[s, h], BLK)
-        kc[h, r0:r0 + c.shape[0]] = c; kd[h, boff[s]:boff[s + 1]] = d
+        if tok:
+            c, d = quant_head(x, km[s, h], 1)
+            kc[h, r0:r0 + c.shape[0]] = c; kd[h, r0:r0 + d.shape[0]] = d
+        else:
+            c, d = quant_head(x, km[s, h], BLK)
+            kc[h, r0:r0 + c.shape[0]] = c; kd[h, boff[s]:boff[s + 1]] = d
     vc = vd = None
     if pv_mode == "fp8":
         vc = np.zeros((T, H, D), np.uint8); vd = np.zeros((S, H, D), np.float32)
@@ -142,8 +150,9 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
     return Quantized(qc, qd, kc, kd, ks, km, vc, vd, status)
 
 
-def _head_view(qz: Quantized, cu, s: int, h: int):
-    """Per-head slices of the quantised tensors for sequence s, head h."""
+def _head_view(qz: Quantized, cu, s: int, h: int, tok: bool = False):
+    """Per-head slices of the quantised tensors for sequence s, head h (tok:
+    deltas stored per code row)."""
     if cu is None:
         qc, qd, kc, kd = qz.q_codes[s, h], qz.q_delta[s, h], qz.k_codes[s, h], qz.k_delta[s, h]
         vc = None if qz.v_codes is None else qz.v_codes[s, h]
@@ -152,7 +161,10 @@ def _head_view(qz: Quantized, cu, s: int, h: int):
     nblk = [(cu[i + 1] - cu[i] + BLK - 1) // BLK for i in range(len(cu) - 1)]
     b0 = sum(nblk[:s]); b1 = b0 + nblk[s]
     qc = qz.q_codes[h, b0 * BLK:b1 * BLK]; kc = qz.k_codes[h, b0 * BLK:b1 * BLK]
-    qd = qz.q_delta[h, b0:b1]; kd = qz.k_delta[h, b0:b1]
+    if tok:
+        qd = qz.q_delta[h, b0 * BLK:b1 * BLK]; kd = qz.k_delta[h, b0 * BLK:b1 * BLK]
+    else:
+        qd = qz.q_delta[h, b0:b1]; kd = qz.k_delta[h, b0:b1]
     vc = None if qz.v_codes is None else np.ascontiguousarray(qz.v_codes[cu[s]:cu[s + 1], h])
     vd = None if qz.v_delta is None else qz.v_delta[s, h]
     return qc, qd, kc, kd, vc, vd
@@ -176,7 +188,7 @@ def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, caus
     vf = v.float().numpy() if pv_mode == "fp16" else None
     for (s, h), rows in _group(picks).items():
         n = (cu[s + 1] - cu[s]) if cu is not None else (seqlens[s] if seqlens else v.shape[2])
-        qc, qd, kc, kd, vc, vd = _head_view(qz, cu, s, h)
+        qc, qd, kc, kd, vc, vd = _head_view(qz, cu, s, h, gran == "token")
         vv = None
         if pv_mode == "fp16":
             vv = vf[s, h] if cu is None else np.ascontiguousarray(vf[cu[s]:cu[s + 1], h])

@@ -260,9 +260,10 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     max_seqlen: int, causal: bool = False, sm_scale: Optional[float] = None,
                     pv_mode: str = "fp16", out_dtype: Optional[torch.dtype] = None,
                     out: Optional[torch.Tensor] = None,
-                    workspace: Optional[Workspace] = None) -> torch.Tensor:
+                    workspace: Optional[Workspace] = None, qk_gran: str = "block") -> torch.Tensor:
     """SageAttention forward over packed [T, H, D] tensors with int32 cu_seqlens.
-    k, v may be [T, Hkv, D] with Hkv dividing H (grouped-query attention)."""
+    k, v may be [T, Hkv, D] with Hkv dividing H (grouped-query attention);
+    qk_gran: one Q/K delta per 128-token block ("block") or per token ("token")."""
     _need_cuda_contig(q, k, v, cu_seqlens)
     if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
         raise ValueError("q must be [T, H, D] and k, v one [T, Hkv, D] shape")
@@ -280,7 +281,16 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     mode = _pv(pv_mode)
     lib = _lib.load()
     scale = float(sm_scale) if sm_scale else 0.0
-    if Hkv == H:
+    gran = _gran(qk_gran)
+    if gran:
+        ws = _workspace(q.device, int(lib.sage_workspace_bytes_varlen_ex(T, batch, H, Hkv, D, mode,
+                                                                         gran)), workspace)
+        _check(lib.sage_attn_fwd_varlen_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
+            _dtype_code(out.dtype, True), _ptr(cu_seqlens), batch, int(max_seqlen), T, H, Hkv, D,
+            int(bool(causal)), scale, mode, gran, ws.ptr, ws.nbytes, _stream(q.device)),
+            "sage_attn_fwd_varlen_ex")
+    elif Hkv == H:
         ws = _workspace(q.device, workspace_bytes_varlen(T, batch, H, D, pv_mode), workspace)
         _check(lib.sage_attn_fwd_varlen(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),

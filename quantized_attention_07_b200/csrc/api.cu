@@ -90,9 +90,11 @@ long long pair_max(long long T, long long batch) { return (T + (2 * BLK - 1) * b
 
 // Varlen layout for H query heads and Hkv key/value heads (Hkv = H without
 // grouping): Q codes / deltas over H heads, everything of K and V over Hkv.
-Layout varlen_layout(int T, int batch, int H, int D, bool fp8, int Hkv = 0) {
+Layout varlen_layout(int T, int batch, int H, int D, bool fp8, int Hkv = 0,
+                     bool per_token = false) {
   if (Hkv <= 0) Hkv = H;
   const size_t SH = (size_t)batch * Hkv, TB = (size_t)tb_max(T, batch);
+  const size_t NS = per_token ? TB * BLK : TB;  // deltas per head
   Layout L{};
   size_t o = kHeader;
   L.k_sum = o; o += al(SH * D * 8);
@@ -103,8 +105,8 @@ Layout varlen_layout(int T, int batch, int H, int D, bool fp8, int Hkv = 0) {
   L.scratch_end = o;
   L.q_codes = o; o += al((size_t)H * TB * BLK * D);
   L.k_codes = o; o += al((size_t)Hkv * TB * BLK * D);
-  L.q_scale = o; o += al((size_t)H * TB * 4);
-  L.k_scale = o; o += al((size_t)Hkv * TB * 4);
+  L.q_scale = o; o += al((size_t)H * NS * 4);
+  L.k_scale = o; o += al((size_t)Hkv * NS * 4);
   L.k_mean = o; o += al(SH * D * 4);
   if (fp8) {
     L.v_codes = o; o += al((size_t)T * Hkv * D);
@@ -392,7 +394,7 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
                                    int D, int pv_mode, int8_t* q_codes, float* q_scale,
                                    int8_t* k_codes, float* k_scale, float* k_mean,
                                    uint8_t* v_codes, float* v_scale, void* ws, const Layout& L,
-                                   cudaStream_t st, int Hkv = 0) {
+                                   cudaStream_t st, int Hkv = 0, int per_token = 0) {
   if (Hkv <= 0) Hkv = H;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   sage_status_t r = clear_scratch(ws, L, fp8, st);
@@ -415,13 +417,14 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
   e = launch_quant(S, dim3((unsigned)TB, Hkv), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes,
                    q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
                    at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                   at<uint32_t>(ws, 0), nullptr, grouped ? QUANT_KV : QUANT_Q | QUANT_KV, 0, st);
+                   at<uint32_t>(ws, 0), nullptr, grouped ? QUANT_KV : QUANT_Q | QUANT_KV,
+                   per_token, st);
   if (e == cudaSuccess && grouped) {
     S.H = H;
     e = launch_quant(S, dim3((unsigned)TB, H), D, in_dt == SAGE_BF16, fp8, q, k, v, q_codes,
                      q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
                      at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
-                     at<uint32_t>(ws, 0), nullptr, QUANT_Q, 0, st);
+                     at<uint32_t>(ws, 0), nullptr, QUANT_Q, per_token, st);
   }
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
@@ -451,15 +454,17 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
                                        int in_dt, int out_dt, const int32_t* cu_seqlens,
                                        int batch, int max_seqlen, int total_tokens, int H,
                                        int Hkv, int D, int causal, float sm_scale, int pv_mode,
-                                       void* ws, size_t ws_bytes, void* stream) {
+                                       int qk_gran, void* ws, size_t ws_bytes, void* stream) {
   if (!varlen_args_ok(total_tokens, batch, max_seqlen, H, D, pv_mode) || !gqa_heads_ok(H, Hkv) ||
-      !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
+      !gran_ok(qk_gran) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
+      !std::isfinite(sm_scale))
     return SAGE_ERR_INVALID_ARG;
+  const int tok = qk_gran == SAGE_QK_PER_TOKEN ? 1 : 0;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws) ||
       !cu_seqlens)
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
-  const Layout L = varlen_layout(total_tokens, batch, H, D, fp8, Hkv);
+  const Layout L = varlen_layout(total_tokens, batch, H, D, fp8, Hkv, tok != 0);
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   if (total_tokens == 0) return SAGE_OK;
   cudaStream_t st = as_stream(stream);
@@ -467,13 +472,14 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
       q, k, v, in_dt, cu_seqlens, batch, max_seqlen, total_tokens, H, D, pv_mode,
       at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale), at<int8_t>(ws, L.k_codes),
       at<float>(ws, L.k_scale), at<float>(ws, L.k_mean), fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
-      fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L, st, Hkv);
+      fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L, st, Hkv, tok);
   if (r != SAGE_OK) return r;
   const long long TB = tb_max(total_tokens, batch), PM = pair_max(total_tokens, batch);
   if (PM == 0) return SAGE_OK;
   AttnLaunch A{};
   A.p.H = H;
   A.p.Hkv = Hkv;
+  A.p.per_token = tok;
   A.p.causal = causal ? 1 : 0;
   A.p.kappa = kappa_of(sm_scale, D);
   A.p.q_scale = at<float>(ws, L.q_scale);
@@ -509,13 +515,33 @@ sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, 
                                    float sm_scale, int pv_mode, void* ws, size_t ws_bytes,
                                    void* stream) {
   return attn_fwd_varlen_g(q, k, v, out, in_dt, out_dt, cu_seqlens, batch, max_seqlen,
-                           total_tokens, H, H, D, causal, sm_scale, pv_mode, ws, ws_bytes, stream);
+                           total_tokens, H, H, D, causal, sm_scale, pv_mode, SAGE_QK_PER_BLOCK, ws,
+                           ws_bytes, stream);
+}
+
+size_t sage_workspace_bytes_varlen_ex(int total_tokens, int batch, int H, int Hkv, int D,
+                                      int pv_mode, int qk_gran) {
+  if (!varlen_args_ok(total_tokens, batch, 0, H, D, pv_mode) || !gqa_heads_ok(H, Hkv) ||
+      !gran_ok(qk_gran))
+    return 0;
+  return varlen_layout(total_tokens, batch, H, D, pv_mode == SAGE_PV_FP8, Hkv,
+                       qk_gran == SAGE_QK_PER_TOKEN).total;
+}
+
+sage_status_t sage_attn_fwd_varlen_ex(const void* q, const void* k, const void* v, void* out,
+                                      int in_dt, int out_dt, const int32_t* cu_seqlens, int batch,
+                                      int max_seqlen, int total_tokens, int H, int Hkv, int D,
+                                      int causal, float sm_scale, int pv_mode, int qk_gran,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  return attn_fwd_varlen_g(q, k, v, out, in_dt, out_dt, cu_seqlens, batch, max_seqlen,
+                           total_tokens, H, Hkv, D, causal, sm_scale, pv_mode, qk_gran, ws,
+                           ws_bytes, stream);
 }
 
 size_t sage_workspace_bytes_varlen_gqa(int total_tokens, int batch, int H, int Hkv, int D,
                                        int pv_mode) {
-  if (!varlen_args_ok(total_tokens, batch, 0, H, D, pv_mode) || !gqa_heads_ok(H, Hkv)) return 0;
-  return varlen_layout(total_tokens, batch, H, D, pv_mode == SAGE_PV_FP8, Hkv).total;
+  return sage_workspace_bytes_varlen_ex(total_tokens, batch, H, Hkv, D, pv_mode,
+                                        SAGE_QK_PER_BLOCK);
 }
 
 sage_status_t sage_attn_fwd_varlen_gqa(const void* q, const void* k, const void* v, void* out,
@@ -524,8 +550,8 @@ sage_status_t sage_attn_fwd_varlen_gqa(const void* q, const void* k, const void*
                                        int Hkv, int D, int causal, float sm_scale, int pv_mode,
                                        void* ws, size_t ws_bytes, void* stream) {
   return attn_fwd_varlen_g(q, k, v, out, in_dt, out_dt, cu_seqlens, batch, max_seqlen,
-                           total_tokens, H, Hkv, D, causal, sm_scale, pv_mode, ws, ws_bytes,
-                           stream);
+                           total_tokens, H, Hkv, D, causal, sm_scale, pv_mode, SAGE_QK_PER_BLOCK,
+                           ws, ws_bytes, stream);
 }
 
 sage_status_t sage_qk_int8_tiles(const int8_t* q_codes, const int8_t* k_codes, int BH, int NP,

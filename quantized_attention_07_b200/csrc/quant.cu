@@ -171,6 +171,60 @@ __device__ __forceinline__ void store_codes(const float (&x)[Tile<D>::NIT][8], f
   }
 }
 
+// 1.5 * 2^23: for |y| < 2^22, the fp32 sum y + kMagic is kMagic + rint(y)
+// (round to nearest even), and its low mantissa byte is rint(y) mod 256.
+constexpr float kMagic = 12582912.0f;
+
+// Low bytes of four floats' bit patterns, packed (a in byte 0).
+__device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float d) {
+  const uint32_t ab = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
+  const uint32_t cd = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
+}
+
+// Per-token quantiser: every row gets its own delta, the max |x - mean| over
+// its D channels (held by the D/8 consecutive lanes that own the row, combined
+// with shuffles); codes as in the block quantiser.  Padding rows get code 0
+// and delta 0.  delta[code_row0 + r] receives the row deltas.
+template <int D, bool BF16, bool SUB, bool FULL>
+__device__ __forceinline__ void regs_codes_per_row(const uint4 (&u)[Tile<D>::NIT], int rows,
+                                                   const float (&mean)[8], int8_t* codes,
+                                                   float* delta, long long code_row0) {
+  using T = Tile<D>;
+  const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
+  float2 nm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) nm[e] = make_float2(-mean[2 * e], -mean[2 * e + 1]);
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i) {
+    const int r = r0 + i * T::RS;
+    const bool valid = FULL || r < rows;
+    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+    float2 f[4];
+    float a = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      f[e] = In16<BF16>::to_float2(w[e]);
+      if constexpr (SUB) f[e] = __fadd2_rn(f[e], nm[e]);
+      a = fmaxf(a, fmaxf(fabsf(f[e].x), fabsf(f[e].y)));
+    }
+    if (!valid) a = 0.0f;
+#pragma unroll
+    for (int o = T::CPR / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const float s = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    float2 y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      y[e] = make_float2(__fadd_rn(__fmul_rn(f[e].x, s), kMagic),
+                         __fadd_rn(__fmul_rn(f[e].y, s), kMagic));
+    uint2 out = make_uint2(low_bytes4(y[0].x, y[0].y, y[1].x, y[1].y),
+                           low_bytes4(y[2].x, y[2].y, y[3].x, y[3].y));
+    if (!valid) out = make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(codes + (code_row0 + r) * D + 8 * c) = out;
+    if (c == 0) delta[code_row0 + r] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  }
+}
+
 // ------------------------------------------------------------------ pass 1 --
 
 template <int D, bool BF16, bool FP8>
@@ -178,7 +232,7 @@ __device__ __forceinline__ void pass1_block(
     const BlockPos& P, const void* __restrict__ q, const void* __restrict__ k,
     const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
     unsigned long long* __restrict__ k_sum, uint32_t* __restrict__ v_amax,
-    uint32_t* __restrict__ status, int parts) {
+    uint32_t* __restrict__ status, int parts, int tok) {
   using T = Tile<D>;
   __shared__ float red[THREADS / 32];
   __shared__ long long red64[THREADS / 32][D];
@@ -193,8 +247,11 @@ __device__ __forceinline__ void pass1_block(
     if (has_kv) load_raw<D>(v, P, rv);
   }
 
-  // --- Q: per-block quantiser
-  if (has_q) {
+  // --- Q: per-token quantiser, or per-block below
+  if (has_q && tok) {
+    const float zero8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    regs_codes_per_row<D, BF16, false, false>(rq, P.rows, zero8, q_codes, q_scale, P.code_row0);
+  } else if (has_q) {
     float x[T::NIT][8];
     to_float<D, BF16>(rq, x);
     float a = 0.0f;
@@ -276,10 +333,10 @@ __global__ void __launch_bounds__(THREADS) quant_pass1_kernel(
     SeqLayout L, const void* __restrict__ q, const void* __restrict__ k,
     const void* __restrict__ v, int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
     unsigned long long* __restrict__ k_sum, uint32_t* __restrict__ v_amax,
-    uint32_t* __restrict__ status, int parts) {
+    uint32_t* __restrict__ status, int parts, int tok) {
   BlockPos P;
   if (!block_pos(L, P)) return;
-  pass1_block<D, BF16, FP8>(P, q, k, v, q_codes, q_scale, k_sum, v_amax, status, parts);
+  pass1_block<D, BF16, FP8>(P, q, k, v, q_codes, q_scale, k_sum, v_amax, status, parts, tok);
 }
 
 // ------------------------------------------------------------------ pass 2 --
@@ -295,7 +352,7 @@ __device__ __forceinline__ void pass2_block(
     const BlockPos& P, const void* __restrict__ k, const void* __restrict__ v,
     const unsigned long long* k_sum, const uint32_t* v_amax,
     int8_t* __restrict__ k_codes, float* __restrict__ k_scale, float* __restrict__ k_mean,
-    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale) {
+    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale, int tok) {
   using T = Tile<D>;
   __shared__ float red[THREADS / 32];
   __shared__ float s_chan[2][D];  // K channel means, V scale factors
@@ -318,8 +375,13 @@ __device__ __forceinline__ void pass2_block(
   }
   __syncthreads();
 
-  // --- K: smoothing + per-block quantiser
-  {
+  // --- K: smoothing + per-token quantiser, or per-block below
+  if (tok) {
+    float m[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = s_chan[0][8 * c + e];
+    regs_codes_per_row<D, BF16, true, false>(rk, P.rows, m, k_codes, k_scale, P.code_row0);
+  } else {
     float m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = s_chan[0][8 * c + e];
@@ -367,10 +429,11 @@ __global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
     SeqLayout L, const void* __restrict__ k, const void* __restrict__ v,
     const unsigned long long* __restrict__ k_sum, const uint32_t* __restrict__ v_amax,
     int8_t* __restrict__ k_codes, float* __restrict__ k_scale, float* __restrict__ k_mean,
-    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale) {
+    uint8_t* __restrict__ v_codes, float* __restrict__ v_scale, int tok) {
   BlockPos P;
   if (!block_pos(L, P)) return;
-  pass2_block<D, BF16, FP8>(P, k, v, k_sum, v_amax, k_codes, k_scale, k_mean, v_codes, v_scale);
+  pass2_block<D, BF16, FP8>(P, k, v, k_sum, v_amax, k_codes, k_scale, k_mean, v_codes, v_scale,
+                            tok);
 }
 
 // ---------------------------------------------------------- streamed, dense --
@@ -439,17 +502,6 @@ __device__ __forceinline__ void item_of(int x, int NB, int U, int lag, int parts
     u = x / NB;
     b = x - u * NB;
   }
-}
-
-// 1.5 * 2^23: for |y| < 2^22, the fp32 sum y + kMagic is kMagic + rint(y)
-// (round to nearest even), and its low mantissa byte is rint(y) mod 256.
-constexpr float kMagic = 12582912.0f;
-
-// Low bytes of four floats' bit patterns, packed (a in byte 0).
-__device__ __forceinline__ uint32_t low_bytes4(float a, float b, float c, float d) {
-  const uint32_t ab = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
-  const uint32_t cd = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
-  return __byte_perm(ab, cd, 0x5410);
 }
 
 // Consumer-side helpers.  Thread t owns the 16-byte chunk c = t % (D/8) of
@@ -547,49 +599,6 @@ __device__ __forceinline__ float regs_absmax_sub(const uint4 (&u)[Tile<D>::NIT],
     }
   }
   return a;
-}
-
-// Per-token quantiser: every row gets its own delta, the max |x - mean| over
-// its D channels (held by the D/8 consecutive lanes that own the row, combined
-// with shuffles); codes as in the block quantiser.  Padding rows get code 0
-// and delta 0.  delta[code_row0 + r] receives the row deltas.
-template <int D, bool BF16, bool SUB, bool FULL>
-__device__ __forceinline__ void regs_codes_per_row(const uint4 (&u)[Tile<D>::NIT], int rows,
-                                                   const float (&mean)[8], int8_t* codes,
-                                                   float* delta, long long code_row0) {
-  using T = Tile<D>;
-  const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
-  float2 nm[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) nm[e] = make_float2(-mean[2 * e], -mean[2 * e + 1]);
-#pragma unroll
-  for (int i = 0; i < T::NIT; ++i) {
-    const int r = r0 + i * T::RS;
-    const bool valid = FULL || r < rows;
-    const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
-    float2 f[4];
-    float a = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      f[e] = In16<BF16>::to_float2(w[e]);
-      if constexpr (SUB) f[e] = __fadd2_rn(f[e], nm[e]);
-      a = fmaxf(a, fmaxf(fabsf(f[e].x), fabsf(f[e].y)));
-    }
-    if (!valid) a = 0.0f;
-#pragma unroll
-    for (int o = T::CPR / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float s = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-    float2 y[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      y[e] = make_float2(__fadd_rn(__fmul_rn(f[e].x, s), kMagic),
-                         __fadd_rn(__fmul_rn(f[e].y, s), kMagic));
-    uint2 out = make_uint2(low_bytes4(y[0].x, y[0].y, y[1].x, y[1].y),
-                           low_bytes4(y[2].x, y[2].y, y[3].x, y[3].y));
-    if (!valid) out = make_uint2(0u, 0u);
-    *reinterpret_cast<uint2*>(codes + (code_row0 + r) * D + 8 * c) = out;
-    if (c == 0) delta[code_row0 + r] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
-  }
 }
 
 // Exact sums of rint(x * 2^24) over the thread's rows, per channel, as two
@@ -1059,21 +1068,20 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
         v_scale, k_sum, v_amax, status, sync);
     return cudaGetLastError();
   }
-  if (tok) return cudaErrorNotSupported;
   quant_pass1_kernel<D, BF16, FP8>
-      <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status, parts);
+      <<<grid, THREADS, 0, st>>>(L, q, k, v, q_codes, q_scale, k_sum, v_amax, status, parts, tok);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !(parts & PART_KV)) return e;
-  quant_pass2_kernel<D, BF16, FP8><<<grid, THREADS, 0, st>>>(L, k, v, k_sum, v_amax, k_codes,
-                                                             k_scale, k_mean, v_codes, v_scale);
+  quant_pass2_kernel<D, BF16, FP8><<<grid, THREADS, 0, st>>>(
+      L, k, v, k_sum, v_amax, k_codes, k_scale, k_mean, v_codes, v_scale, tok);
   return cudaGetLastError();
 }
 
 // Runs both passes.  k_sum / v_amax and (dense) sync[0 .. units] must be zero
 // on entry (the caller clears them on the stream).  grid = (blocks per head or
 // TBmax, units = B*H or H).  parts: QUANT_Q and/or QUANT_KV (both unless the
-// query and key/value heads differ).  per_token: one delta per token (dense
-// only; deltas indexed like the code rows).
+// query and key/value heads differ).  per_token: one delta per token (deltas
+// indexed like the code rows).
 cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool fp8,
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,

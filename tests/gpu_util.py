@@ -77,12 +77,13 @@ def run_dense(q, k, v, causal, pv_mode, out_dtype=torch.float32, sm_scale=None,
     return out.cpu()
 
 
-def run_varlen(q, k, v, cu, causal, pv_mode, out_dtype=torch.float32, sm_scale=None):
+def run_varlen(q, k, v, cu, causal, pv_mode, out_dtype=torch.float32, sm_scale=None,
+               qk_gran="block"):
     dev = torch.device("cuda")
     lens = (cu[1:] - cu[:-1]).tolist()
     out = sage.attn_fwd_varlen(q.to(dev), k.to(dev), v.to(dev), cu.to(dev), max(lens) if lens else 0,
                                causal=causal, sm_scale=sm_scale, pv_mode=pv_mode,
-                               out_dtype=out_dtype)
+                               out_dtype=out_dtype, qk_gran=qk_gran)
     torch.cuda.synchronize()
     sage.sync_status()
     return out.cpu()
@@ -115,8 +116,8 @@ def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
             g = q.shape[1] // k.shape[1]
             k, v = heads.repeat_kv(k, g), heads.repeat_kv(v, g)
     else:
-        out32 = run_varlen(q, k, v, cu, causal, pv_mode, torch.float32, sm_scale)
-        out16 = run_varlen(q, k, v, cu, causal, pv_mode, q.dtype, sm_scale)
+        out32 = run_varlen(q, k, v, cu, causal, pv_mode, torch.float32, sm_scale, qk_gran)
+        out16 = run_varlen(q, k, v, cu, causal, pv_mode, q.dtype, sm_scale, qk_gran)
         if k.shape[1] != q.shape[1]:
             g = q.shape[1] // k.shape[1]
             k, v = heads.repeat_kv_packed(k, g), heads.repeat_kv_packed(v, g)

@@ -74,3 +74,14 @@ def test_per_token_deltas_help_with_outliers():
         cos[gran] = sage.cosine_similarity(o[idx[:, 0], idx[:, 1], idx[:, 2]], ref)
     print(cos)
     assert cos["token"] > cos["block"] + 0.01 and cos["token"] > 0.98
+
+
+@pytest.mark.parametrize("causal,pv_mode,dtype,H,Hkv", [(True, "fp16", "bf16", 4, 2),
+                                                       (False, "fp8", "fp16", 2, 2)])
+def test_per_token_varlen_against_oracle(causal, pv_mode, dtype, H, Hkv):
+    lens = [1, 300, 0, 129, 517]
+    D = 128 if pv_mode == "fp8" else 64
+    q, k, v, cu = W.make_varlen(lens, H, D, dtype, seed=31 + H)
+    k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
+    picks = [(s, h, i) for s, n in enumerate(lens) for h in range(H) for i in range(0, n, 2)]
+    U.check_against_oracle(q, k, v, cu, causal, pv_mode, picks, qk_gran="token")

@@ -526,3 +526,29 @@ def test_per_token_emulation_follows_its_rounding_sequence():
     want = [fp32(fp32(sum(Fr(P[j]) * Fr(float(v[j, d])) for j in range(3))) / Fr(l))
             for d in range(4)]
     assert got.tolist() == want
+
+
+def test_per_token_varlen_layout_matches_dense_per_sequence():
+    """Packed per-token quantisation = the dense per-token quantisation of each
+    sequence, placed at the sequence's code rows (deltas one per code row)."""
+    lens = [5, 130, 0, 3]
+    gen = torch.Generator().manual_seed(8)
+    T, H, D = sum(lens), 2, 16
+    q = (torch.randn(T, H, D, generator=gen) * 2).half()
+    k = (torch.randn(T, H, D, generator=gen) + 1).half()
+    cu = torch.tensor([0, 5, 135, 135, 138], dtype=torch.int32)
+    qz = heads.quantize(q, k, None, cu, "fp16", gran="token")
+    r0 = 0
+    for s, n in enumerate(lens):
+        if n == 0:
+            continue
+        qs, ks = q[cu[s]:cu[s + 1]], k[cu[s]:cu[s + 1]]
+        dz = heads.quantize(qs.permute(1, 0, 2)[None].contiguous(),
+                            ks.permute(1, 0, 2)[None].contiguous(), None, None, "fp16",
+                            gran="token")
+        for h in range(H):
+            assert np.array_equal(qz.q_codes[h, r0:r0 + n], dz.q_codes[0, h, :n])
+            assert np.array_equal(qz.q_delta[h, r0:r0 + n], dz.q_delta[0, h, :n])
+            assert np.array_equal(qz.k_codes[h, r0:r0 + n], dz.k_codes[0, h, :n])
+            assert np.array_equal(qz.k_delta[h, r0:r0 + n], dz.k_delta[0, h, :n])
+        r0 += ((n + 127) // 128) * 128
