@@ -429,6 +429,7 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8/fp8" if wl.pv_mode == "fp8" else "int8/fp16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D,
+                   "Hkv": wl.kv_heads, "qk_gran": wl.qk_gran,
                    "in_dtype": wl.dtype, "causal": wl.causal, "pv_mode": wl.pv_mode},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": vals[0]["cores"],
                          "kind": "oracle",
