@@ -37,8 +37,10 @@
  *     outside the exact-mean range) are OR-ed into a status word at the start
  *     of the workspace and reported by sage_sync_status().
  *   - Workspace: every compute call takes (ws, ws_bytes).  Its first 256 bytes
- *     hold the status word; sage_workspace_init() must zero them once before
- *     first use.  Calls on different streams must use different workspaces.
+ *     hold the status word and the attention kernel's work-item counters;
+ *     sage_workspace_init() must zero them once before first use (each
+ *     attention launch leaves the counters at zero again).  Calls on
+ *     different streams must use different workspaces.
  *   - Layouts: dense tensors are [B, H, N, D] row-major; varlen tensors are
  *     [T, H, D] row-major with T = cu_seqlens[batch].  D is 64 or 128.
  *   - Causal masking is top-left aligned (query i sees keys j <= i), per

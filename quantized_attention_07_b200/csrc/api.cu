@@ -36,7 +36,11 @@ sage_status_t cuda_fail(cudaError_t e, const char* what) {
   return SAGE_ERR_CUDA;
 }
 
+// Workspace header: the status word at byte 0 and the attention kernel's two
+// work-scheduler counters at kSchedOff (zeroed by sage_workspace_init; every
+// attention launch leaves them at zero).
 constexpr size_t kHeader = 256;
+constexpr size_t kSchedOff = 64;
 constexpr long long kMaxN = 1LL << 22;
 
 size_t al(size_t x) { return (x + 255) & ~size_t(255); }
@@ -205,6 +209,7 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
   A.p.out_dt = out_dt;
   A.p.varlen = 0;
   A.p.status = at<uint32_t>(ws, 0);
+  A.p.sched = at<unsigned int>(ws, kSchedOff);
   A.D = D;
   A.pv8 = fp8;
   A.bf16v = v_dt == SAGE_BF16;
@@ -215,7 +220,7 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
   A.code_z = B * H;
   A.code_z_kv = B * Hkv;
   A.T = 0;
-  A.grid = dim3((unsigned)((long long)B * H * A.p.NPAIR), 1, 1);
+  A.p.items = B * H * A.p.NPAIR;
   cudaError_t e = launch_attn(A, st);
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "attention launch");
 }
@@ -494,6 +499,7 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
   A.p.batch = batch;
   A.p.TBmax = (int)TB;
   A.p.status = at<uint32_t>(ws, 0);
+  A.p.sched = at<unsigned int>(ws, kSchedOff);
   A.D = D;
   A.pv8 = fp8;
   A.bf16v = in_dt == SAGE_BF16;
@@ -504,7 +510,8 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
   A.code_z = H;
   A.code_z_kv = Hkv;
   A.T = total_tokens;
-  A.grid = dim3((unsigned)PM, H, 1);
+  A.p.PM = (int)PM;
+  A.p.items = (int)(PM * H);
   cudaError_t e = launch_attn(A, st);
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "attention launch");
 }

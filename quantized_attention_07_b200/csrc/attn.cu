@@ -38,6 +38,8 @@
 // ST_TIMEOUT, raises a CTA-wide abort flag that the other roles' waits also
 // watch, and everyone falls through to the teardown, which waits (bounded) for
 // the CTA's own TMA loads and MMAs and always frees TMEM.
+#include <algorithm>
+
 #include "attn_launch.cuh"
 #include "exp2.cuh"
 #include "ptx.cuh"
@@ -92,7 +94,12 @@ struct Bars {
   uint64_t s_full[2][2];   // [tile][S buffer]: QK^T of a sub-tile landed
   uint64_t p_full[2][2];   // P of a sub-tile written, O rescaled (128 softmax threads)
   uint64_t o_full[2];      // P.V of a sub-tile completed
-  uint64_t o_done[2];      // the last P.V of a query tile completed (one phase)
+  uint64_t o_done[2];      // the last P.V of a query tile of an item completed
+  uint64_t q_empty;        // both MMA warps' last QK^T of the item completed (2 commits)
+  uint64_t item_full[2];   // work-item ring: index published by the producer
+  uint64_t item_empty[2];  // ... and read by both MMA warps and all 256 softmax threads
+  int item[2];
+  int sm_loop[8][2];       // per softmax warp: items taken, items with keys (see softmax_wg)
   uint64_t k_full[8], v_full[8], kv_empty[8];
   uint32_t tmem_base;
   volatile int abort;
@@ -139,11 +146,13 @@ struct Work {
   int nkv;               // 128-key stages to stream
 };
 
-__device__ __forceinline__ Work decode_work(const AttnParams& p) {
+// Work item idx of the launch (0 <= idx < p.items).  Dense: idx -> (head,
+// query tile pair); varlen: idx = h * PM + item, item over the sequences'
+// pairs (items past the last pair are empty).
+__device__ __forceinline__ Work decode_work(const AttnParams& p, int idx) {
   Work w{};
   int pair, n;
   if (!p.varlen) {
-    const int idx = blockIdx.x;
     int bh;
     if (p.causal) {  // heaviest pairs first
       pair = p.NPAIR - 1 - idx / p.BH;
@@ -170,8 +179,8 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
     w.out_stride = 1;
     w.vs_idx = bkv;
   } else {
-    const int item = blockIdx.x;
-    const int h = blockIdx.y;
+    const int h = idx / p.PM;
+    const int item = idx - h * p.PM;
     const int total = __ldg(p.pair_off + p.batch);
     if (item >= total) { w.valid = 0; return w; }
     const int s = find_segment(p.pair_off, p.batch + 1, item);
@@ -205,54 +214,121 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p) {
   return w;
 }
 
+// ------------------------------------------------------- work scheduling --
+//
+// Work items are handed out dynamically: the producer warp takes the next
+// index from a global counter (p.sched[0]) and publishes it to the CTA's other
+// roles through a two-slot ring in shared memory; -1 ends the loop.  The
+// counter and the count of finished CTAs (p.sched[1]) start at zero; the last
+// CTA to finish sets both back to zero for the next launch.
+
+constexpr int ITEM_READERS = 2 + 256;  // item_empty arrivals: 2 MMA warps + 256 softmax threads
+
+// Index of the r-th item taken by this CTA's consumers (false on timeout or
+// abort).  The whole warp calls it; `all_lanes` arrive individually
+// (softmax) or lane 0 for the warp (MMA warps).
+__device__ __forceinline__ bool take_item(Bars* B, int r, uint32_t* status, bool all_lanes,
+                                          int& idx) {
+  const int s = r & 1;
+  if (!wait_bar(B, &B->item_full[s], (r >> 1) & 1, status, true)) return false;
+  idx = *reinterpret_cast<volatile int*>(&B->item[s]);
+  if (all_lanes) {
+    ptx::mbar_arrive(&B->item_empty[s]);
+  } else {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&B->item_empty[s]);
+  }
+  return true;
+}
+
 // --------------------------------------------------------------- producer --
 
 template <int D, bool PV8, bool TOK>
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                         const Work& w, Bars* B, uint8_t* sQ, uint8_t* sK, uint8_t* sV,
-                         float* sKs, const float* k_scale, uint32_t* status) {
+                         const AttnParams& p, Bars* B, uint8_t* sQ, uint8_t* sK, uint8_t* sV,
+                         float* sKs) {
   using C = Cfg<D, PV8, TOK>;
   // The whole warp runs this loop (uniform control flow); one elected lane
-  // issues each TMA instruction.
+  // issues each TMA instruction.  Stages form one ring across the CTA's work
+  // items: G counts the stages loaded so far.
   if (ptx::elect_one()) {
     ptx::prefetch_tmap(tm_q);
     ptx::prefetch_tmap(tm_k);
     ptx::prefetch_tmap(tm_v);
-    // both Q^ tiles (an absent second tile reads zero-filled or padding rows)
-    ptx::mbar_arrive_expect_tx(&B->q_full, 2 * C::QT);
-    ptx::tma_load_3d(sQ, tm_q, &B->q_full, 0, w.q_y0, w.code_z);
-    ptx::tma_load_3d(sQ + C::QT, tm_q, &B->q_full, 0, w.q_y0 + BLK, w.code_z);
   }
   __syncwarp();
-  int j = 0;
-  for (; j < w.nkv; ++j) {
-    const int s = j % C::NS;
-    if (j >= C::NS && !wait_bar(B, &B->kv_empty[s], ((j / C::NS) - 1) & 1, status, true)) break;
-    if (ptx::elect_one()) {
-      ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);
-      ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
-      if constexpr (TOK)  // the stage's 128 per-token K deltas, on the same barrier
-        ptx::bulk_load_plain(sKs + s * BLK, k_scale + (w.ks_idx0 + j) * BLK, C::KS,
-                             &B->k_full[s]);
-      ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
-      uint8_t* dst = sV + s * C::VT;
-      const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
-      const int z = w.v_tok_on_z ? w.v_z0 + j * BLK : w.v_z0;
-      ptx::tma_load_3d(dst, tm_v, &B->v_full[s], 0, y, z);
-      if (!PV8 && D == 128)  // 16-bit V rows are 256 B: second 64-column box
-        ptx::tma_load_3d(dst + BLK * 128, tm_v, &B->v_full[s], 64, y, z);
+  const int lane = threadIdx.x & 31;
+  auto fetch = [&]() -> int {
+    int v = 0;
+    if (lane == 0) v = (int)atomicAdd(p.sched, 1u);
+    v = __shfl_sync(0xffffffffu, v, 0);
+    return v < p.items ? v : -1;
+  };
+  int G = 0, n = 0;
+  bool ok = true;
+  int next = fetch();
+  for (int r = 0; ok; ++r) {
+    // publish the r-th item (slot r & 1, free once item r-2 was read)
+    const int idx = next;
+    const int slot = r & 1;
+    if (r >= 2 && !wait_bar(B, &B->item_empty[slot], ((r >> 1) - 1) & 1, p.status, true)) break;
+    if (lane == 0) {
+      B->item[slot] = idx;
+      ptx::mbar_arrive(&B->item_full[slot]);
     }
     __syncwarp();
+    if (idx < 0) break;
+    const Work w = decode_work(p, idx);
+    if (!w.valid) {
+      next = fetch();
+      continue;
+    }
+    // the previous item's QK^T must have read both Q^ tiles
+    if (n > 0 && !wait_bar(B, &B->q_empty, (n - 1) & 1, p.status, true)) break;
+    if (ptx::elect_one()) {
+      // both Q^ tiles (an absent second tile reads zero-filled or padding rows)
+      ptx::mbar_arrive_expect_tx(&B->q_full, 2 * C::QT);
+      ptx::tma_load_3d(sQ, tm_q, &B->q_full, 0, w.q_y0, w.code_z);
+      ptx::tma_load_3d(sQ + C::QT, tm_q, &B->q_full, 0, w.q_y0 + BLK, w.code_z);
+    }
+    __syncwarp();
+    ++n;
+    for (int j = 0; j < w.nkv; ++j, ++G) {
+      const int s = G % C::NS;
+      if (G >= C::NS && !wait_bar(B, &B->kv_empty[s], ((G / C::NS) - 1) & 1, p.status, true)) {
+        ok = false;
+        break;
+      }
+      if (ptx::elect_one()) {
+        ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);
+        ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
+        if constexpr (TOK)  // the stage's 128 per-token K deltas, on the same barrier
+          ptx::bulk_load_plain(sKs + s * BLK, p.k_scale + (w.ks_idx0 + j) * BLK, C::KS,
+                               &B->k_full[s]);
+        ptx::mbar_arrive_expect_tx(&B->v_full[s], C::VT);
+        uint8_t* dst = sV + s * C::VT;
+        const int y = w.v_tok_on_z ? w.v_y0 : w.v_y0 + j * BLK;
+        const int z = w.v_tok_on_z ? w.v_z0 + j * BLK : w.v_z0;
+        ptx::tma_load_3d(dst, tm_v, &B->v_full[s], 0, y, z);
+        if (!PV8 && D == 128)  // 16-bit V rows are 256 B: second 64-column box
+          ptx::tma_load_3d(dst + BLK * 128, tm_v, &B->v_full[s], 64, y, z);
+      }
+      __syncwarp();
+    }
+    // The next item is taken only now, when this one's last loads are issued
+    // (a few stages before its MMAs end): taking it earlier would bind it to
+    // this CTA while another CTA may become free first.
+    next = fetch();
   }
-  // Teardown: the most recent load of every stage must have landed before
-  // this CTA may exit (the earlier ones were consumed already).
-  for (int jj = max(0, j - C::NS); jj < j; ++jj) {
+  // Teardown: the most recent load of every stage and of Q must have landed
+  // before this CTA may exit (the earlier ones were consumed already).
+  for (int jj = max(0, G - C::NS); jj < G; ++jj) {
     const int s = jj % C::NS;
     const uint32_t ph = (jj / C::NS) & 1;
     ptx::mbar_wait(&B->k_full[s], ph);
     ptx::mbar_wait(&B->v_full[s], ph);
   }
-  ptx::mbar_wait(&B->q_full, 0);
+  if (n > 0) ptx::mbar_wait(&B->q_full, (n - 1) & 1);
 }
 
 // ------------------------------------------------------------ MMA issuer --
@@ -264,49 +340,55 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
 // P_t(i) before P.V has read it.  A 128-key stage is released to the producer
 // when both tiles' warps have committed it (kv_empty counts two arrivals).
 template <int D, bool PV8, bool BF16V, bool TOK>
-__device__ void mma_issuer(const Work& w, Bars* B, uint32_t tmem, const uint8_t* sQ,
-                           const uint8_t* sK, const uint8_t* sV, int t, uint32_t* status) {
+__device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const uint8_t* sQ,
+                           const uint8_t* sK, const uint8_t* sV, int t) {
   using C = Cfg<D, PV8, TOK>;
   constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, SUB);
   constexpr uint32_t IDESC_PV =
       PV8 ? ptx::instr_desc(1, 0, 0, 0, 1, 128, D)
           : ptx::instr_desc(1, BF16V ? 1 : 0, BF16V ? 1 : 0, 0, 1, 128, D);
-  const int nt = t == 0 ? w.nsub0 : w.nsub1;
-  const int nst = w.nkv;                      // stages the producer loads
+  uint32_t* status = p.status;
   const uint32_t qa = ptx::smem_u32(sQ + t * C::QT);
   const uint32_t tO = tmem + 256 + D * t;
-  int k_ready = -1, v_ready = -1;             // highest stage known to be loaded
-  int released = 0;                           // stages this warp has committed
+  // Counts over the CTA's work items: sub-tiles of this tile (I0: S buffer
+  // and barrier phases), stages of the ring (G0), items (n: q_full phase).
+  int I0 = 0, G0 = 0, n = 0;
+  int nt = 0, released = 0;                   // this item: sub-tiles, stages committed
+  int k_ready = -1, v_ready = -1;             // highest ring stage known to be loaded
 
-  auto need_k = [&](int j) -> bool {
-    if (k_ready >= j) return true;
-    if (!wait_bar(B, &B->k_full[j % C::NS], (j / C::NS) & 1, status, true)) return false;
-    k_ready = j;
+  auto need_k = [&](int g) -> bool {
+    if (k_ready >= g) return true;
+    if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, status, true)) return false;
+    k_ready = g;
     return true;
   };
-  auto need_v = [&](int j) -> bool {
-    if (v_ready >= j) return true;
-    if (!wait_bar(B, &B->v_full[j % C::NS], (j / C::NS) & 1, status, true)) return false;
-    v_ready = j;
+  auto need_v = [&](int g) -> bool {
+    if (v_ready >= g) return true;
+    if (!wait_bar(B, &B->v_full[g % C::NS], (g / C::NS) & 1, status, true)) return false;
+    v_ready = g;
     return true;
   };
-  auto issue_qk = [&](int i) {
-    const uint32_t kb = ptx::smem_u32(sK + ((i / 2) % C::NS) * C::QT + (i & 1) * C::K_SUB_BYTES);
-    const uint32_t dst = tmem + 128 * t + SUB * (i & 1);
+  auto issue_qk = [&](int i) {  // i: sub-tile of the item
+    const int I = I0 + i, g = G0 + i / 2;
+    const uint32_t kb = ptx::smem_u32(sK + (g % C::NS) * C::QT + (i & 1) * C::K_SUB_BYTES);
+    const uint32_t dst = tmem + 128 * t + SUB * (I & 1);
     if (ptx::elect_one()) {
       const uint64_t a0 = ptx::smem_desc(qa, 16, C::QK_SBO, C::QK_SWZ);
       const uint64_t b0 = ptx::smem_desc(kb, 16, C::QK_SBO, C::QK_SWZ);
 #pragma unroll
       for (int kk = 0; kk < D / 32; ++kk)  // +32 bytes along K per step: +2 in the address field
         ptx::mma_i8_ss(dst, a0 + 2 * kk, b0 + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
-      ptx::mma_commit(&B->s_full[t][i & 1]);
+      ptx::mma_commit(&B->s_full[t][I & 1]);
+      // after the item's last QK^T the Q^ tiles may be reloaded
+      if (i == nt - 1) ptx::mma_commit(&B->q_empty);
     }
     __syncwarp();
   };
   auto issue_pv = [&](int i) {
-    const uint32_t vb = ptx::smem_u32(sV + ((i / 2) % C::NS) * C::VT + (i & 1) * C::V_SUB_BYTES);
-    const uint32_t tP = tmem + 128 * t + SUB * (i & 1);
-    const uint32_t acc0 = PV8 ? 0u : (i > 0 ? 1u : 0u);
+    const int I = I0 + i, g = G0 + i / 2;
+    const uint32_t vb = ptx::smem_u32(sV + (g % C::NS) * C::VT + (i & 1) * C::V_SUB_BYTES);
+    const uint32_t tP = tmem + 128 * t + SUB * (I & 1);
+    const uint32_t acc0 = PV8 ? 0u : (i > 0 ? 1u : 0u);  // an item's first P.V starts O
     if (ptx::elect_one()) {
       const uint64_t b0 = ptx::smem_desc(vb, C::V_LBO, C::V_SBO, C::V_SWZ);
 #pragma unroll
@@ -321,44 +403,62 @@ __device__ void mma_issuer(const Work& w, Bars* B, uint32_t tmem, const uint8_t*
     }
     __syncwarp();
   };
-  // Commit stage `released` (this warp is done with it).  For a stage this
-  // tile never reads, first wait until the stage's previous use was released,
-  // so the arrival cannot count toward that earlier phase.
+  // Commit the item's next stage (this warp is done with it).  A stage this
+  // tile never reads is first waited for like a used one: then every load
+  // this warp releases was seen complete by it, which keeps the parity of
+  // the slot's next k_full / v_full phase unambiguous for this warp in a
+  // later item, and the producer's refill of the slot (issued only after the
+  // previous release) makes the arrival count toward this stage's phase.
   auto release = [&](bool used) -> bool {
-    const int j = released;
-    if (!used && j >= C::NS &&
-        !wait_bar(B, &B->kv_empty[j % C::NS], ((j / C::NS) - 1) & 1, status, true))
-      return false;
-    if (ptx::elect_one()) ptx::mma_commit(&B->kv_empty[j % C::NS]);
+    const int g = G0 + released;
+    if (!used && !(need_k(g) && need_v(g))) return false;
+    if (ptx::elect_one()) ptx::mma_commit(&B->kv_empty[g % C::NS]);
     __syncwarp();
     ++released;
     return true;
   };
 
-  bool ok = wait_bar(B, &B->q_full, 0, status, true);
-  if (ok) ptx::tc_fence_after();
-  for (int i = 0; ok && i < 2 && i < nt; ++i) {
-    if (!need_k(i / 2)) { ok = false; break; }
+  bool ok = true;
+  for (int r = 0; ok; ++r) {
+    int idx;
+    if (!take_item(B, r, status, false, idx) || idx < 0) break;
+    const Work w = decode_work(p, idx);
+    if (!w.valid) continue;
+    nt = t == 0 ? w.nsub0 : w.nsub1;
+    released = 0;
+    ok = wait_bar(B, &B->q_full, n & 1, status, true);
+    if (!ok) break;
     ptx::tc_fence_after();
-    issue_qk(i);
-  }
-  for (int i = 0; ok && i < nt; ++i) {
-    if (!need_v(i / 2)) break;
-    if (!wait_bar(B, &B->p_full[t][i & 1], (i / 2) & 1, status, true)) break;
-    ptx::tc_fence_after();
-    issue_pv(i);
-    if (i + 2 < nt) {
-      if (!need_k((i + 2) / 2)) break;
+    if (nt == 0) {  // no key for this tile: its share of q_empty right away
+      if (ptx::elect_one()) ptx::mma_commit(&B->q_empty);
+      __syncwarp();
+    }
+    for (int i = 0; ok && i < 2 && i < nt; ++i) {
+      ok = need_k(G0 + i / 2);
+      if (!ok) break;
       ptx::tc_fence_after();
-      issue_qk(i + 2);
+      issue_qk(i);
     }
-    if ((i & 1) || i == nt - 1) {
-      if (!release(true)) break;
+    for (int i = 0; ok && i < nt; ++i) {
+      ok = need_v(G0 + i / 2) &&
+           wait_bar(B, &B->p_full[t][(I0 + i) & 1], ((I0 + i) / 2) & 1, status, true);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      issue_pv(i);
+      if (i + 2 < nt) {
+        ok = need_k(G0 + (i + 2) / 2);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_qk(i + 2);
+      }
+      if ((i & 1) || i == nt - 1) ok = release(true);
     }
-  }
-  // stages loaded for the other tile only
-  while (ok && released < nst && released >= (nt + 1) / 2) {
-    if (!release(false)) break;
+    // stages loaded for the other tile only
+    while (ok && released < w.nkv && released >= (nt + 1) / 2) ok = release(false);
+    if (!ok) break;
+    I0 += nt;
+    G0 += w.nkv;
+    ++n;
   }
   // Drain: every MMA this warp issued completes before TMEM is released.
   if (ptx::elect_one()) ptx::mma_commit(&B->done[t]);
@@ -464,8 +564,9 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
 }
 
 template <int D, bool PV8, bool BF16V, bool TOK>
-__device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t tmem, int t,
-                           const float* sKs) {
+__device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w, Bars* B,
+                                             uint32_t tmem, int t, const float* sKs, int I0,
+                                             int G0, volatile int* loop) {
   using C = Cfg<D, PV8, TOK>;
   using In = In16<BF16V>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
@@ -477,7 +578,6 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
   const uint32_t tS0 = tmem + 128 * t + lane_off;
   const uint32_t tO = tmem + 256 + D * t + lane_off;
   const int nsub = t == 0 ? w.nsub0 : w.nsub1;
-  if (nsub == 0) return;
 
   // deltaQ of this tile's block, or (per token) of this row
   const float qd = __ldg(p.q_scale + (TOK ? (w.qs_idx0 + t) * BLK + r : w.qs_idx0 + t));
@@ -491,13 +591,14 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
   const int limit = p.causal ? min(w.n, row + 1) : w.n;  // keys >= limit are masked
 
   for (int i = 0; i < nsub; ++i) {
-    const int b = i & 1;
+    const int I = I0 + i;                        // sub-tile count of this tile over the items
+    const int b = I & 1;
     const uint32_t tS = tS0 + SUB * b;
     if (!TOK && (i & 1) == 0) {  // a new 128-key quantisation block: its delta
       const float kd = __ldg(p.k_scale + w.ks_idx0 + i / 2);
       c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
     }
-    if (!wait_bar(B, &B->s_full[t][b], (i / 2) & 1, p.status, true)) return;
+    if (!wait_bar(B, &B->s_full[t][b], (I / 2) & 1, p.status, true)) return false;
     ptx::tc_fence_after();
     const int key0 = i * SUB;
     const bool full_tile = (key0 + SUB <= w.n) && (!p.causal || key0 + SUB - 1 <= qt * BLK);
@@ -507,9 +608,9 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
     // place; the K deltas came with the K tile (wait on its barrier).
     auto tile_max = [&](uint32_t (&sv)[SUB], float& m_blk) -> bool {
       if constexpr (TOK) {
-        const int j = i / 2;
-        if (!wait_bar(B, &B->k_full[j % C::NS], (j / C::NS) & 1, p.status, true)) return false;
-        const float* dk = sKs + (j % C::NS) * BLK + (i & 1) * SUB;
+        const int g = G0 + i / 2;  // ring stage of the sub-tile
+        if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, p.status, true)) return false;
+        const float* dk = sKs + (g % C::NS) * BLK + (i & 1) * SUB;
         const float ym = full_tile ? row_scale_max<SUB, false>(sv, dk, key0, limit)
                                    : row_scale_max<SUB, true>(sv, dk, key0, limit);
         m_blk = ym == -INFINITY ? -INFINITY : __fmul_rn(ym, c);
@@ -529,7 +630,7 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
       ptx::tmem_wait_ld();
       // a sub-tile with no unmasked key for this row leaves the maximum unchanged
       float m_blk;
-      if (!tile_max(sv, m_blk)) return;
+      if (!tile_max(sv, m_blk)) return false;
       m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
       alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
 #pragma unroll
@@ -545,7 +646,7 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
       // O <- alpha * O before this sub-tile's P.V accumulates into it (rare:
       // only when some row's maximum moved by more than TAU)
       if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
+        if (!wait_bar(B, &B->o_full[t], (I - 1) & 1, p.status, true)) return false;
         ptx::tc_fence_after();
         const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
@@ -570,7 +671,7 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
         ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
       ptx::tmem_wait_ld();
       float m_blk;
-      if (!tile_max(sv, m_blk)) return;
+      if (!tile_max(sv, m_blk)) return false;
       m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
       alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
       // P^ = e4m3(448 p), four per TMEM column, written over S
@@ -591,7 +692,7 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
       if (i > 0) {
         // two-level accumulation: O32 <- alpha_{i-1} O32 + Part_{i-1}, 64
         // columns of the partial per TMEM round trip
-        if (!wait_bar(B, &B->o_full[t], (i - 1) & 1, p.status, true)) return;
+        if (!wait_bar(B, &B->o_full[t], (I - 1) & 1, p.status, true)) return false;
         ptx::tc_fence_after();
         const float2 a2 = make_float2(alpha_prev, alpha_prev);
 #pragma unroll
@@ -619,8 +720,9 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
   }
 
   // ------------------------------------------------------------ epilogue --
-  // (o_full may lag by two phases here in 16-bit mode; o_done is unambiguous)
-  if (!wait_bar(B, &B->o_done[t], 0, p.status, true)) return;
+  // (o_full may lag by two phases here in 16-bit mode; o_done is unambiguous:
+  // one phase per item in which this tile has keys)
+  if (!wait_bar(B, &B->o_done[t], loop[1] & 1, p.status, true)) return false;
   ptx::tc_fence_after();
   const bool store = row < w.n;
   const long long orow = (w.out_row0 + (long long)row * w.out_stride) * D;
@@ -661,6 +763,35 @@ __device__ void softmax_wg(const AttnParams& p, const Work& w, Bars* B, uint32_t
       }
     }
   }
+  return true;
+}
+
+// One softmax warpgroup per query tile t, over the CTA's work items.  The
+// counts carried across items give the S buffer and barrier phases: I0 the
+// tile's sub-tiles so far, G0 the ring stages, loop[1] the items with keys
+// (o_done phase).  The item counts sit in a per-warp shared-memory slot
+// rather than in registers, which the per-sub-tile loop needs.
+template <int D, bool PV8, bool BF16V, bool TOK>
+__device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, const float* sKs) {
+  volatile int* loop = B->sm_loop[threadIdx.x / 32];  // [0] items taken, [1] items with keys
+  loop[0] = 0;
+  loop[1] = 0;
+  int I0 = 0, G0 = 0;
+  while (true) {
+    const int r = loop[0];
+    int idx;
+    if (!take_item(B, r, p.status, true, idx) || idx < 0) return;
+    loop[0] = r + 1;
+    const Work w = decode_work(p, idx);
+    if (!w.valid) continue;
+    const int nsub = t == 0 ? w.nsub0 : w.nsub1;
+    if (nsub > 0) {
+      if (!softmax_item<D, PV8, BF16V, TOK>(p, w, B, tmem, t, sKs, I0, G0, loop)) return;
+      loop[1] = loop[1] + 1;
+    }
+    I0 += nsub;
+    G0 += w.nkv;
+  }
 }
 
 // ---------------------------------------------------------------- kernel --
@@ -679,14 +810,17 @@ __global__ void __launch_bounds__(Cfg<D, PV8, TOK>::THREADS, 1)
   Bars* B = reinterpret_cast<Bars*>(sV + C::NS * (C::VT + C::KS));
   static_assert(sizeof(Bars) <= C::AUX, "aux layout");
 
-  const Work w = decode_work(p);
-  if (!w.valid) return;
   const int warp = threadIdx.x / 32;
   const int wg = warp / 4;
   const int warp_tma = 4 * C::WG_CTRL, warp_mma = 4 * C::WG_CTRL + 1;  // MMA warps: +1, +2
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&B->q_full, 1);
+    ptx::mbar_init(&B->q_empty, 2);  // one commit per MMA warp
+    for (int r = 0; r < 2; ++r) {
+      ptx::mbar_init(&B->item_full[r], 1);
+      ptx::mbar_init(&B->item_empty[r], ITEM_READERS);
+    }
     ptx::mbar_init(&B->done[0], 1);
     ptx::mbar_init(&B->done[1], 1);
     for (int t = 0; t < 2; ++t) {
@@ -717,19 +851,29 @@ __global__ void __launch_bounds__(Cfg<D, PV8, TOK>::THREADS, 1)
   if (wg == C::WG_CTRL) {
     ptx::setmaxnreg_dec<C::REG_CTRL>();
     if (warp == warp_tma) {
-      producer<D, PV8, TOK>(&tm_q, &tm_k, &tm_v, w, B, sQ, sK, sV, sKs, p.k_scale, p.status);
+      producer<D, PV8, TOK>(&tm_q, &tm_k, &tm_v, p, B, sQ, sK, sV, sKs);
     } else if (warp == warp_mma || warp == warp_mma + 1) {
-      mma_issuer<D, PV8, BF16V, TOK>(w, B, tmem, sQ, sK, sV, warp - warp_mma, p.status);
+      mma_issuer<D, PV8, BF16V, TOK>(p, B, tmem, sQ, sK, sV, warp - warp_mma);
     }
   } else {
     ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
-    softmax_wg<D, PV8, BF16V, TOK>(p, w, B, tmem, wg, sKs);
+    softmax_wg<D, PV8, BF16V, TOK>(p, B, tmem, wg, sKs);
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == warp_mma) ptx::tmem_dealloc(tmem, 512);
+  // Every fetch of this CTA happened before the barrier above: the last CTA
+  // to get here resets the scheduler for the next launch.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      __threadfence();
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
+  }
 }
 
 // ------------------------------------------------ QK^T tile diagnostic --
@@ -878,7 +1022,12 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
   auto kern = attn_fwd_kernel<D, PV8, BF16V, TOK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<L.grid, C::THREADS, C::SMEM, st>>>(tq, tk, tv, L.p);
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (L.p.items <= 0) return cudaSuccess;
+  kern<<<dim3((unsigned)std::min(L.p.items, std::max(sms, 1))), C::THREADS, C::SMEM, st>>>(tq, tk, tv, L.p);
   return cudaGetLastError();
 }
 

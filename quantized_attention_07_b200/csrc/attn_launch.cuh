@@ -25,6 +25,9 @@ struct AttnParams {
   const int32_t* pair_off;
   int batch;
   int TBmax;
+  int PM;                // varlen: work items per head (query tile pairs of the longest layout)
+  int items;             // work items of the launch: dense BH*NPAIR, varlen H*PM
+  unsigned int* sched;   // [2] in the workspace header: next item, CTAs finished (zero between launches)
   uint32_t* status;
 };
 
@@ -38,9 +41,10 @@ struct AttnLaunch {
   int code_z;            // Q^ z-slices: BH (dense) or H (varlen)
   int code_z_kv;         // K^ (and dense V) z-slices: B*Hkv (dense) or H (varlen)
   int T;                 // varlen tokens
-  dim3 grid;
 };
 
+// Persistent launch: min(p.items, SM count) CTAs, each taking work items
+// from the counter p.sched until none is left.
 cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st);
 
 }  // namespace sage
