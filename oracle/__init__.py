@@ -68,8 +68,10 @@ def lib():
         L.oracle_attn_ref_rows.argtypes = [P, P, P, i64, i32, i64, i64, i64, f64, i32, P, i64, P]
         L.oracle_attn_ref_rows.restype = None
         L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, i32, f32, f32,
-                                            i32, i32, i32, P, i64, P, i32]
+                                            i32, i32, i32, P, i64, P, i32, P, i64]
         L.oracle_attn_emul_rows.restype = None
+        L.oracle_q_smooth_bias.argtypes = [P, i64, P, i64, i32, i64, P, f32, P, i64]
+        L.oracle_q_smooth_bias.restype = None
         _lib = L
     return _lib
 
@@ -176,20 +178,41 @@ def attn_ref_rows(q, k, v, sm_scale: float, causal: bool, rows) -> np.ndarray:
     return out
 
 
+def q_smooth_bias(qmean: np.ndarray, k: np.ndarray, kmean: np.ndarray, sm_scale: float,
+                  ldo: Optional[int] = None) -> np.ndarray:
+    """Per-key term of Q smoothing for one head: [nb, ldo] fp32 with
+    out[I, j] = fp32(kappa * qmean[I] . (k[j] - kmean)) for j < n (0 beyond).
+    qmean: [nb, D] block means of Q; k: [n, D]; kmean: [D]."""
+    qmean, k, kmean = _f32(qmean), _f32(k), _f32(kmean)
+    nb, D = qmean.shape
+    n = k.shape[0]
+    ldo = n if ldo is None else ldo
+    out = np.zeros((nb, ldo), dtype=np.float32)
+    lib().oracle_q_smooth_bias(_p(qmean), nb, _p(k), n, D, D, _p(kmean), float(kappa(sm_scale)),
+                               _p(out), ldo)
+    return out
+
+
 def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, causal: bool,
                    pv_mode: str, rows, v=None, p16: str = "fp16", vc=None, vdelta=None,
                    blk: int = 128, kv: int = KV_TILE, tau=None,
-                   per_token: bool = False) -> np.ndarray:
+                   per_token: bool = False, bias: Optional[np.ndarray] = None) -> np.ndarray:
     """The quantised method's output rows (fp32) for one head; see sage_oracle.c.
     blk: quantisation block (tokens); kv: key tile of the online softmax;
-    per_token: qdelta / kdelta hold one delta per token (blk is then unused)."""
+    per_token: qdelta / kdelta hold one delta per token (blk is then unused);
+    bias: Q smoothing's per-key term [nb, >= n] (q_smooth_bias), per-block
+    deltas only."""
     if not per_token and blk % kv:
         raise ValueError("the key tile must divide the quantisation block")
+    if bias is not None and per_token:
+        raise ValueError("Q smoothing is defined with per-block deltas")
     qc = np.ascontiguousarray(qc, dtype=np.int8)
     kc = np.ascontiguousarray(kc, dtype=np.int8)
     qdelta, kdelta = _f32(qdelta), _f32(kdelta)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     out = np.zeros((len(rows), D), dtype=np.float32)
+    if bias is not None:
+        bias = _f32(bias)
     if pv_mode == "fp16":
         v = _f32(v)
         vc_p, vd_p, v_p, ldv, mode = None, None, _p(v), D, 0
@@ -201,5 +224,6 @@ def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, caus
                                 D, blk, kv, float(kappa(sm_scale)),
                                 float(TAU[pv_mode] if tau is None else tau), int(causal), mode,
                                 1 if p16 == "bf16" else 0, _p(rows), len(rows), _p(out),
-                                int(bool(per_token)))
+                                int(bool(per_token)), _p(bias),
+                                0 if bias is None else bias.shape[1])
     return out

@@ -19,7 +19,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import attn_emul_rows, attn_ref_rows, default_sm_scale, k_mean, quant_head, quant_v_fp8
+from . import (attn_emul_rows, attn_ref_rows, default_sm_scale, k_mean, q_smooth_bias, quant_block,
+               quant_head, quant_v_fp8)
 
 BLK = 128
 
@@ -35,6 +36,7 @@ class Quantized:
     v_codes: Optional[np.ndarray]
     v_delta: Optional[np.ndarray]
     status: int
+    q_mean: Optional[np.ndarray] = None   # gran "block_sq": Q block means [B,H,NB,D]
 
 
 def _heads(x: torch.Tensor, cu: Optional[list[int]]):
@@ -84,10 +86,29 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
     """gran "block": one delta per 128-token block (deltas [B,H,NB] dense,
     [H, TB] varlen); "token": one delta per token, the quantiser applied to
     one-row blocks, stored like the code rows (deltas [B,H,NP] dense,
-    [H, TB*128] varlen; padding rows 0)."""
+    [H, TB*128] varlen; padding rows 0); "block_sq" (dense only): per-block
+    deltas of Q smoothed by its block mean (SageAttention2's smoothing of Q),
+    the means in q_mean [B,H,NB,D]."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     status = 0
     tok = gran == "token"
+    if gran == "block_sq":
+        if cu is not None:
+            raise ValueError("Q smoothing is defined here for dense inputs")
+        qz = quantize(q, k, v, None, pv_mode, "block")  # K and V as for "block"
+        B, H, N, D = q.shape
+        NB = (N + BLK - 1) // BLK
+        qc = np.zeros((B, H, NB * BLK, D), np.int8)
+        qd = np.zeros((B, H, NB), np.float32)
+        qm = np.zeros((B, H, NB, D), np.float32)
+        for b, h, x in _heads(q, None):
+            for I in range(NB):
+                xb = np.ascontiguousarray(x[I * BLK:(I + 1) * BLK])
+                _, qm[b, h, I], st = k_mean(xb)  # the exact row mean, over this block's rows
+                status |= st
+                qc[b, h, I * BLK:I * BLK + xb.shape[0]], qd[b, h, I] = quant_block(xb, qm[b, h, I])
+        return Quantized(qc, qd, qz.k_codes, qz.k_delta, qz.k_sum, qz.k_mean, qz.v_codes,
+                         qz.v_delta, status | qz.status, qm)
     if cu is None:
         B, H, N, D = q.shape
         NB = (N + BLK - 1) // BLK
@@ -179,8 +200,11 @@ def _group(picks):
 
 def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, causal: bool,
                  pv_mode: str, sm_scale: Optional[float] = None,
-                 seqlens: Optional[list[int]] = None, gran: str = "block") -> dict:
-    """E for the listed (seq, head, row) picks -> {pick: fp32 [D]}."""
+                 seqlens: Optional[list[int]] = None, gran: str = "block",
+                 k: Optional[torch.Tensor] = None) -> dict:
+    """E for the listed (seq, head, row) picks -> {pick: fp32 [D]}.  gran
+    "block_sq" needs k (dense, [B,H,N,D], one head per query head) for the
+    per-key term of Q smoothing."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     sm_scale = default_sm_scale(D) if sm_scale is None else sm_scale
     p16 = "bf16" if v.dtype == torch.bfloat16 else "fp16"
@@ -192,8 +216,12 @@ def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, caus
         vv = None
         if pv_mode == "fp16":
             vv = vf[s, h] if cu is None else np.ascontiguousarray(vf[cu[s]:cu[s + 1], h])
+        bias = None
+        if gran == "block_sq":
+            bias = q_smooth_bias(qz.q_mean[s, h], k[s, h].float().numpy(), qz.k_mean[s, h],
+                                 sm_scale)
         o = attn_emul_rows(qc, qd, kc, kd, n, D, sm_scale, causal, pv_mode, rows, v=vv, p16=p16,
-                           vc=vc, vdelta=vd, per_token=gran == "token")
+                           vc=vc, vdelta=vd, per_token=gran == "token", bias=bias)
         for r, i in enumerate(rows):
             out[(s, h, i)] = o[r]
     return out

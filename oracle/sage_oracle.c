@@ -375,12 +375,24 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *   arg_ij = fmaf(y_ij, c_i, -m_new)
  * (the product (A^ B^) deltaA deltaB of the quantisation intro, step 3, with a
  * per-row deltaA and a per-column deltaB); everything else as above.
+ *
+ * bk != NULL: Q smoothing (SageAttention2, dtcms.com page, v2 bullet 2, and
+ * the postsniper.ru post's SageAttention2 bullet 1, which also normalise Q).
+ * The Q codes are those of q~ = q - qmean_I (per-block channel mean of Q), and
+ * the part of q.k~ that the mean carries is added back per key:
+ * bk[I*ldb + j] = fp32(kappa * qmean_I . k~_j) (see oracle_q_smooth_bias).
+ * Per-block deltas only:
+ *   c_IJ   = fp32( fp32(deltaQ_I * deltaK_J) * kappa )
+ *   y_ij   = fmaf(S_ij, c_IJ, bk_Ij)                  scaled logit
+ *   mb     = max_j y_ij
+ *   arg_ij = fp32(y_ij - m_new)
+ * everything else as above.
  */
 void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* kc,
                            const float* kdelta, const float* v, long ldv, const uint8_t* vc,
                            const float* vdelta, long n, int D, int blk, int kv, float kappa,
                            float tau, int causal, int pv_mode, int p16_format, const long* rows,
-                           long nrows, float* out, int per_token)
+                           long nrows, float* out, int per_token, const float* bk, long ldb)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (long r = 0; r < nrows; ++r) {
@@ -409,7 +421,17 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
                 if (acc > smax) smax = acc;
             }
             float c, mblk;
-            if (!per_token) {
+            if (bk) {
+                /* Q smoothing: the per-key mean term joins before the maximum */
+                const float* bI = bk + I * ldb + j0;
+                c = (qdelta[I] * kdelta[J]) * kappa;
+                float ymax = -INFINITY;
+                for (int jj = 0; jj < nj; ++jj) {
+                    y[jj] = fmaf((float)S[jj], c, bI[jj]);
+                    if (y[jj] > ymax) ymax = y[jj];
+                }
+                mblk = ymax;
+            } else if (!per_token) {
                 /* one delta per 128-token block of Q and of K */
                 c = (qdelta[I] * kdelta[J]) * kappa;
                 mblk = (float)smax * c;
@@ -428,7 +450,8 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
             float alpha = (float)exp2((double)(m - m_new));
             double psum = 0.0;
             for (int jj = 0; jj < nj; ++jj) {
-                float arg = per_token ? fmaf(y[jj], c, -m_new) : fmaf((float)S[jj], c, -m_new);
+                float arg = bk ? y[jj] - m_new
+                            : per_token ? fmaf(y[jj], c, -m_new) : fmaf((float)S[jj], c, -m_new);
                 p[jj] = (float)exp2((double)arg);
                 psum += (double)p[jj];
             }
@@ -457,5 +480,39 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
             else o[d] = (O[d] * (vdelta[d] / 448.0f)) / l;
         }
         free(O); free(part); free(S); free(p); free(y);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Q smoothing: the per-key term of the block mean.                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * With q = q~ + qmean_I for the rows of query block I (SageAttention2's
+ * smoothing of Q, dtcms.com page, v2 bullet 2), the smoothed logit splits as
+ *   q . k~_j = q~ . k~_j + qmean_I . k~_j,
+ * the first part quantised like any Q block, the second a dot product that
+ * depends on the block and the key only.  (qmean_I . m, the part through the
+ * K mean, is a constant per row and leaves the softmax unchanged, as for K
+ * smoothing; the term here uses the smoothed k~ = fp32(k - kmean) that the K
+ * codes come from.)
+ *
+ *   out[I*ldo + j] = fp32( kappa * sum_d qmean[I][d] * k~_j[d] )   (fp64 sum)
+ *
+ * qmean: [nb][D]; k: row j at k + j*ld; kmean: [D]; out: [nb][ldo], columns
+ * j < n written.
+ */
+void oracle_q_smooth_bias(const float* qmean, long nb, const float* k, long n, int D, long ld,
+                          const float* kmean, float kappa, float* out, long ldo)
+{
+    for (long I = 0; I < nb; ++I) {
+        for (long j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) {
+                const float ks = k[j * ld + d] - kmean[d];
+                acc += (double)qmean[I * D + d] * (double)ks;
+            }
+            out[I * ldo + j] = (float)(acc * (double)kappa);
+        }
     }
 }
