@@ -216,11 +216,14 @@ def run_ours(args, rank, world, local):
         ws = sage.Workspace(sage.workspace_bytes(B, H, N, D, wl.pv_mode), dev)
 
         def stage1():
-            api.quantize(q, k, v, wl.pv_mode, qz=qz, workspace=ws, qk_gran=wl.qk_gran)
+            api.quantize(q, k, v, wl.pv_mode, qz=qz, workspace=ws, qk_gran=wl.qk_gran,
+                         causal=wl.causal)
 
         def stage2():
             api.attn_quantized(qz, v, causal=wl.causal, out=out, workspace=ws)
-        launches_per_step = 2  # quant_stream_kernel, attn_fwd_kernel
+        # quant_stream_kernel, attn_fwd_kernel; Q smoothing: Q in its own
+        # kernel (quant_q_smooth_kernel) and the mean term (q_smooth_bias_kernel)
+        launches_per_step = 4 if wl.qk_gran == "block_sq" else 2
     else:
         T, H, D = q.shape
         out = torch.empty_like(q)
@@ -385,7 +388,7 @@ def cpu_oracle_throughput(wl, inp, budget_rows: int, quant_heads: int, seed: int
     picks = [p for p in W.sample_rows(lens, hs, budget_rows, seed) if p[1] < hs]
     t0 = time.perf_counter()
     heads.emulate_rows(qz, vh, inp.cu_seqlens, picks, wl.D, wl.causal, wl.pv_mode,
-                       gran=wl.qk_gran)
+                       gran=wl.qk_gran, k=kh if wl.qk_gran == "block_sq" else None)
     t_rows = time.perf_counter() - t0
 
     def work(i):  # key pairs of row i

@@ -75,10 +75,15 @@ typedef enum {
 } sage_pv_mode_t;
 
 /* Granularity of the Q and K deltas ("SageAttention v1/v2/v2++/v3 overview",
- * SageAttention v1 item (1): per-block or per-token quantisation of q, k). */
+ * SageAttention v1 item (1): per-block or per-token quantisation of q, k),
+ * and Q smoothing (same page, SageAttention2 bullet 2). */
 typedef enum {
-  SAGE_QK_PER_BLOCK = 0, /* one delta per 128-token block (and head)             */
-  SAGE_QK_PER_TOKEN = 1  /* one delta per token                                   */
+  SAGE_QK_PER_BLOCK = 0,         /* one delta per 128-token block (and head)     */
+  SAGE_QK_PER_TOKEN = 1,         /* one delta per token                           */
+  SAGE_QK_PER_BLOCK_SMOOTH_Q = 2 /* per block, each Q block minus its channel
+                                    mean before quantisation; the mean's part of
+                                    the logit, mean . k~_j, added back per key
+                                    (dense problems only)                         */
 } sage_qk_gran_t;
 
 /* Token count of one quantisation block and of one attention key/query tile. */
@@ -142,6 +147,12 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
  * dequantised as y = fp32(S_ij * deltaK_j), arg = fmaf(y, fp32(deltaQ_i *
  * sm_scale * log2 e), -m) (per block: c = fp32(fp32(deltaQ*deltaK) * kappa),
  * arg = fmaf(S, c, -m)).
+ * With SAGE_QK_PER_BLOCK_SMOOTH_Q the codes of query block I are those of
+ * fp32(q - qmean_I), qmean_I the exact channel mean of the block's rows (the
+ * K mean's definition), and the scaled logit is y = fmaf(S, c, b_Ij) with
+ * b_Ij = fp32(kappa * qmean_I . fp32(k_j - kmean)), the dot product summed in
+ * fp64 in channel order, then arg = y - m.
+ * Its workspace also holds qmean and b (B*H*NB*(D + NB*128) floats).
  *   ws : at least sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, qk_gran).
  * sage_attn_fwd(...) = sage_attn_fwd_ex(..., Hkv = H, ..., SAGE_QK_PER_BLOCK).
  */
@@ -256,6 +267,8 @@ sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
  * padding rows 0.  sage_attn_quantized_ex needs k_scale 16-byte aligned (the
  * kernel copies 128 deltas at a time).  ws: at least sage_scratch_bytes(B, H,
  * D), which covers every Hkv <= H (SAGE_ERR_WORKSPACE when too small).
+ * SAGE_QK_PER_BLOCK_SMOOTH_Q has its own two stages (sage_quantize_sq,
+ * sage_attn_quantized_sq); these two return SAGE_ERR_INVALID_ARG for it.
  */
 sage_status_t sage_quantize_ex(const void* q, const void* k, const void* v, int in_dt, int B,
                                int H, int Hkv, int N, int D, int pv_mode, int qk_gran,
@@ -268,6 +281,33 @@ sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale
                                      int v_dt, int out_dt, int B, int H, int Hkv, int N, int D,
                                      int causal, float sm_scale, int pv_mode, int qk_gran,
                                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The two stages with Q smoothing (SAGE_QK_PER_BLOCK_SMOOTH_Q, dense).
+ * sage_quantize_sq writes, besides the outputs of sage_quantize_ex with
+ * per-block deltas,
+ *   q_mean : fp32 [B, H, NB, D], the block means of Q;
+ *   q_bias : fp32 [B, H, NB, NP], q_bias[b,h,I,j] = fp32(kappa * q_mean[b,h,I]
+ *            . fp32(k_j - k_mean)) for key j of the key/value head of h, kappa
+ *            = fp32(sm_scale * log2 e); keys j >= N give 0; with causal != 0
+ *            the blocks I < j/128, which the mask hides, are not written.
+ *            16-byte aligned.
+ * sm_scale and causal are those the attention stage will use.
+ * sage_attn_quantized_sq takes the codes and deltas with q_bias.  ws: as
+ * sage_quantize_ex / sage_attn_quantized_ex.
+ */
+sage_status_t sage_quantize_sq(const void* q, const void* k, const void* v, int in_dt, int B,
+                               int H, int Hkv, int N, int D, int pv_mode, int causal,
+                               float sm_scale, int8_t* q_codes, float* q_scale, float* q_mean,
+                               int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
+                               float* v_scale, float* q_bias, void* ws, size_t ws_bytes,
+                               void* stream);
+sage_status_t sage_attn_quantized_sq(const int8_t* q_codes, const float* q_scale,
+                                     const int8_t* k_codes, const float* k_scale,
+                                     const float* q_bias, const void* v, const uint8_t* v_codes,
+                                     const float* v_scale, void* out, int v_dt, int out_dt, int B,
+                                     int H, int Hkv, int N, int D, int causal, float sm_scale,
+                                     int pv_mode, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Stage 1 for a packed varlen batch.  Layouts (TB = number of 128-token blocks

@@ -35,6 +35,10 @@ SIGNATURES = {
                           _P], _I),
     "sage_quantize_ex": ([_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
                           _P, _SZ, _P], _I),
+    "sage_quantize_sq": ([_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P,
+                          _P, _P, _P, _P, _SZ, _P], _I),
+    "sage_attn_quantized_sq": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                _I, _F, _I, _P, _SZ, _P], _I),
     "sage_attn_quantized_ex": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
                                 _F, _I, _I, _P, _SZ, _P], _I),
     "sage_attn_ref_rows": ([_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P], _I),

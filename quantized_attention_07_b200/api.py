@@ -137,7 +137,8 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
 
     k and v may have fewer heads than q ([B, Hkv, N, D], H a multiple of Hkv):
     grouped-query attention, query head h reading key/value head h // (H // Hkv).
-    qk_gran: "block" (one Q/K delta per 128 tokens) or "token" (one per token).
+    qk_gran: "block" (one Q/K delta per 128 tokens), "token" (one per token) or
+    "block_sq" (per block, with each Q block smoothed by its channel mean).
     """
     _need_cuda_contig(q, k, v)
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
@@ -263,7 +264,8 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     workspace: Optional[Workspace] = None, qk_gran: str = "block") -> torch.Tensor:
     """SageAttention forward over packed [T, H, D] tensors with int32 cu_seqlens.
     k, v may be [T, Hkv, D] with Hkv dividing H (grouped-query attention);
-    qk_gran: one Q/K delta per 128-token block ("block") or per token ("token")."""
+    qk_gran: one Q/K delta per 128-token block ("block") or per token ("token");
+    Q smoothing ("block_sq") is for dense inputs only."""
     _need_cuda_contig(q, k, v, cu_seqlens)
     if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
         raise ValueError("q must be [T, H, D] and k, v one [T, Hkv, D] shape")
@@ -282,6 +284,8 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     lib = _lib.load()
     scale = float(sm_scale) if sm_scale else 0.0
     gran = _gran(qk_gran)
+    if qk_gran == "block_sq":
+        raise ValueError("qk_gran 'block_sq' (Q smoothing) is implemented for dense inputs only")
     if gran:
         ws = _workspace(q.device, int(lib.sage_workspace_bytes_varlen_ex(T, batch, H, Hkv, D, mode,
                                                                          gran)), workspace)
@@ -310,7 +314,7 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
 
 # ---------------------------------------------------------------- stages --
 
-QK_GRANS = {"block": 0, "token": 1}
+QK_GRANS = {"block": 0, "token": 1, "block_sq": 2}
 
 
 def _gran(g: str) -> int:
@@ -323,7 +327,10 @@ def _gran(g: str) -> int:
 class Quantized:
     """Outputs of the smoothing + quantisation stage (all device tensors).
     Dense: q_codes [B, H, NP, D], k_codes [B, Hkv, NP, D]; deltas [.., NB]
-    per 128-token block or [.., NP] per token (qk_gran)."""
+    per 128-token block or [.., NP] per token (qk_gran).  Q smoothing
+    ("block_sq") adds the Q block means q_mean [B, H, NB, D] and the per-key
+    mean term q_bias [B, H, NB, NP], which depends on the attention call's
+    causal flag and sm_scale (recorded in sq_causal, sq_sm_scale)."""
     q_codes: torch.Tensor
     q_scale: torch.Tensor
     k_codes: torch.Tensor
@@ -333,14 +340,20 @@ class Quantized:
     v_scale: Optional[torch.Tensor]
     pv_mode: str
     qk_gran: str = "block"
+    q_mean: Optional[torch.Tensor] = None
+    q_bias: Optional[torch.Tensor] = None
+    sq_causal: bool = False
+    sq_sm_scale: float = 0.0
 
 
 def alloc_quantized(B: int, H: int, N: int, D: int, pv_mode: str, device,
                     Hkv: Optional[int] = None, qk_gran: str = "block") -> Quantized:
     NB = (N + BLOCK - 1) // BLOCK
-    NS = NB * BLOCK if _gran(qk_gran) else NB
+    _gran(qk_gran)
+    NS = NB * BLOCK if qk_gran == "token" else NB
     Hk = Hkv or H
     fp8 = pv_mode == "fp8"
+    sq = qk_gran == "block_sq"
     e = dict(device=device)
     return Quantized(
         torch.empty((B, H, NB * BLOCK, D), dtype=torch.int8, **e),
@@ -350,14 +363,19 @@ def alloc_quantized(B: int, H: int, N: int, D: int, pv_mode: str, device,
         torch.empty((B, Hk, D), dtype=torch.float32, **e),
         torch.empty((B, Hk, N, D), dtype=torch.uint8, **e) if fp8 else None,
         torch.empty((B, Hk, D), dtype=torch.float32, **e) if fp8 else None,
-        pv_mode, qk_gran)
+        pv_mode, qk_gran,
+        torch.empty((B, H, NB, D), dtype=torch.float32, **e) if sq else None,
+        torch.empty((B, H, NB, NB * BLOCK), dtype=torch.float32, **e) if sq else None)
 
 
 def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
              pv_mode: str = "fp16", qz: Optional[Quantized] = None,
-             workspace: Optional[Workspace] = None, qk_gran: str = "block") -> Quantized:
+             workspace: Optional[Workspace] = None, qk_gran: str = "block",
+             causal: bool = False, sm_scale: Optional[float] = None) -> Quantized:
     """Stage 1 (K smoothing, INT8 Q/K per block or per token, FP8 V) of a dense
-    problem; k, v may have fewer heads than q (grouped-query)."""
+    problem; k, v may have fewer heads than q (grouped-query).  With
+    qk_gran "block_sq" Q is smoothed too, and causal / sm_scale must be those
+    of the attention call (the per-key mean term is scaled and masked here)."""
     _need_cuda_contig(q, k)
     B, H, N, D = q.shape
     Hkv = k.shape[1]
@@ -369,6 +387,16 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
         _need_cuda_contig(v)
     qz = qz or alloc_quantized(B, H, N, D, pv_mode, q.device, Hkv, qk_gran)
     ws = _workspace(q.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
+    if qk_gran == "block_sq":
+        scale = float(sm_scale) if sm_scale else 0.0
+        _check(_lib.load().sage_quantize_sq(
+            _ptr(q), _ptr(k), _ptr(v) if mode == 1 else None, _dtype_code(q.dtype), B, H, Hkv, N,
+            D, mode, int(bool(causal)), scale, _ptr(qz.q_codes), _ptr(qz.q_scale),
+            _ptr(qz.q_mean), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(qz.k_mean),
+            _ptr(qz.v_codes), _ptr(qz.v_scale), _ptr(qz.q_bias), ws.ptr, ws.nbytes,
+            _stream(q.device)), "sage_quantize_sq")
+        qz.sq_causal, qz.sq_sm_scale = bool(causal), scale
+        return qz
     _check(_lib.load().sage_quantize_ex(
         _ptr(q), _ptr(k), _ptr(v) if mode == 1 else None, _dtype_code(q.dtype), B, H, Hkv, N, D,
         mode, gran, _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale),
@@ -390,6 +418,17 @@ def attn_quantized(qz: Quantized, v: torch.Tensor, causal: bool = False,
     if out is None:
         out = torch.empty((B, H, N, D), dtype=od, device=v.device)
     ws = _workspace(v.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
+    if qz.qk_gran == "block_sq":
+        scale = float(sm_scale) if sm_scale else 0.0
+        if bool(causal) != qz.sq_causal or scale != qz.sq_sm_scale:
+            raise ValueError("Q smoothing's mean term was built for another causal / sm_scale")
+        _check(_lib.load().sage_attn_quantized_sq(
+            _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale),
+            _ptr(qz.q_bias), _ptr(v), _ptr(qz.v_codes), _ptr(qz.v_scale), _ptr(out),
+            _dtype_code(v.dtype), _dtype_code(out.dtype, True), B, H, Hkv, N, D,
+            int(bool(causal)), scale, mode, ws.ptr, ws.nbytes, _stream(v.device)),
+            "sage_attn_quantized_sq")
+        return out
     _check(_lib.load().sage_attn_quantized_ex(
         _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(v),
         _ptr(qz.v_codes), _ptr(qz.v_scale), _ptr(out), _dtype_code(v.dtype),

@@ -18,6 +18,12 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                          uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
                          int per_token, cudaStream_t st);
+cudaError_t launch_quant_q_smooth(int BH, int N, int D, bool bf16, const void* q,
+                                  int8_t* q_codes, float* q_scale, float* q_mean,
+                                  uint32_t* status, cudaStream_t st);
+cudaError_t launch_q_smooth_bias(int B, int H, int Hkv, int N, int D, bool bf16, int causal,
+                                 float kappa, const void* k, const float* k_mean,
+                                 const float* q_mean, float* bias, cudaStream_t st);
 cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
                             const int32_t* tiles, int n, int32_t* out, uint32_t* status,
                             cudaStream_t st);
@@ -58,6 +64,7 @@ struct Layout {
   size_t k_sum, v_amax, sync, sync_q, blk_off, pair_off;  // scratch
   size_t q_codes, k_codes, q_scale, k_scale, k_mean;   // quantised operands
   size_t v_codes, v_scale;
+  size_t q_mean, q_bias;                              // Q smoothing (dense)
   size_t scratch_end, total;
 };
 
@@ -65,7 +72,10 @@ struct Layout {
 // without grouping).  sync: work counter + one completion counter per
 // key/value head for the launch that quantises K (and Q when Hkv = H);
 // sync_q: the work counter of the separate Q launch when Hkv < H.
-Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, bool per_token = false) {
+// gran: a sage_qk_gran_t (per-token deltas; Q smoothing adds the block means
+// and the per-key mean term).
+Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, int gran = SAGE_QK_PER_BLOCK) {
+  const bool per_token = gran == SAGE_QK_PER_TOKEN;
   const size_t BH = (size_t)B * H, BK = (size_t)B * Hkv, NB = ((size_t)N + BLK - 1) / BLK,
                NP = NB * BLK, NS = per_token ? NP : NB;  // deltas per head
   Layout L{};
@@ -83,6 +93,10 @@ Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, bool per_toke
   if (fp8) {
     L.v_codes = o; o += al(BK * (size_t)N * D);
     L.v_scale = o; o += al(BK * D * 4);
+  }
+  if (gran == SAGE_QK_PER_BLOCK_SMOOTH_Q) {
+    L.q_mean = o; o += al(BH * NB * D * 4);
+    L.q_bias = o; o += al(BH * NB * NP * 4);
   }
   L.total = o;
   return L;
@@ -126,7 +140,12 @@ bool dense_args_ok(int B, int H, int N, int D, int pv_mode) {
 }
 
 bool gqa_heads_ok(int H, int Hkv) { return Hkv >= 1 && Hkv <= H && H % Hkv == 0; }
-bool gran_ok(int g) { return g == SAGE_QK_PER_BLOCK || g == SAGE_QK_PER_TOKEN; }
+bool gran_ok(int g) {
+  return g == SAGE_QK_PER_BLOCK || g == SAGE_QK_PER_TOKEN || g == SAGE_QK_PER_BLOCK_SMOOTH_Q;
+}
+bool gran_varlen_ok(int g) { return g == SAGE_QK_PER_BLOCK || g == SAGE_QK_PER_TOKEN; }
+// sage_quantize_ex / sage_attn_quantized_ex: Q smoothing has its own stages
+bool gran_split_ok(int g) { return g == SAGE_QK_PER_BLOCK || g == SAGE_QK_PER_TOKEN; }
 
 bool varlen_args_ok(int T, int batch, int max_seqlen, int H, int D, int pv_mode) {
   return T >= 0 && batch >= 1 && max_seqlen >= 0 && max_seqlen <= kMaxN && H >= 1 &&
@@ -186,16 +205,48 @@ sage_status_t quantize_dense(const void* q, const void* k, const void* v, int in
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
 
+// Dense stage 1 with Q smoothing: K (and V) as for per-block deltas over the
+// key/value heads, then the smoothed Q blocks and the per-key mean term.
+sage_status_t quantize_dense_sq(const void* q, const void* k, const void* v, int in_dt, int B,
+                                int H, int N, int D, int pv_mode, int causal, float sm_scale,
+                                int8_t* q_codes, float* q_scale, float* q_mean, int8_t* k_codes,
+                                float* k_scale, float* k_mean, uint8_t* v_codes, float* v_scale,
+                                float* q_bias, void* ws, const Layout& L, cudaStream_t st,
+                                int Hkv) {
+  const bool fp8 = pv_mode == SAGE_PV_FP8, bf16 = in_dt == SAGE_BF16;
+  sage_status_t r = clear_scratch(ws, L, fp8, st);
+  if (r != SAGE_OK) return r;
+  SeqLayout S{};
+  S.varlen = 0;
+  S.N = N;
+  S.H = Hkv;
+  const unsigned NB = (unsigned)((N + BLK - 1) / BLK);
+  cudaError_t e = launch_quant(S, dim3(NB, (unsigned)(B * Hkv)), D, bf16, fp8, q, k, v, q_codes,
+                               q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
+                               at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
+                               at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync), QUANT_KV, 0, st);
+  if (e == cudaSuccess)
+    e = launch_quant_q_smooth(B * H, N, D, bf16, q, q_codes, q_scale, q_mean, at<uint32_t>(ws, 0),
+                              st);
+  if (e == cudaSuccess)
+    e = launch_q_smooth_bias(B, H, Hkv, N, D, bf16, causal ? 1 : 0, kappa_of(sm_scale, D), k,
+                             k_mean, q_mean, q_bias, st);
+  if (e == cudaErrorNotSupported) return SAGE_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
+}
+
 sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
                          const float* k_scale, const void* v, const uint8_t* v_codes,
                          const float* v_scale, void* out, int v_dt, int out_dt, int B, int H,
                          int N, int D, int causal, float sm_scale, int pv_mode, void* ws,
-                         cudaStream_t st, int Hkv, int per_token = 0) {
+                         cudaStream_t st, int Hkv, int per_token = 0,
+                         const float* q_bias = nullptr) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   AttnLaunch A{};
   A.p.H = H;
   A.p.Hkv = Hkv;
   A.p.per_token = per_token;
+  A.p.q_bias = q_bias;
   A.p.N = N;
   A.p.BH = B * H;
   A.p.NB = (N + BLK - 1) / BLK;
@@ -289,7 +340,7 @@ sage_status_t sage_quantize_ex(const void* q, const void* k, const void* v, int 
                                int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
                                float* k_mean, uint8_t* v_codes, float* v_scale, void* ws,
                                size_t ws_bytes, void* stream) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran) ||
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_split_ok(qk_gran) ||
       !in_dtype_ok(in_dt))
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
@@ -319,7 +370,7 @@ sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale
                                      int v_dt, int out_dt, int B, int H, int Hkv, int N, int D,
                                      int causal, float sm_scale, int pv_mode, int qk_gran,
                                      void* ws, size_t ws_bytes, void* stream) {
-  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran) ||
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_split_ok(qk_gran) ||
       !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
@@ -345,9 +396,51 @@ sage_status_t sage_attn_quantized(const int8_t* q_codes, const float* q_scale,
                                 SAGE_QK_PER_BLOCK, ws, ws_bytes, stream);
 }
 
+sage_status_t sage_quantize_sq(const void* q, const void* k, const void* v, int in_dt, int B,
+                               int H, int Hkv, int N, int D, int pv_mode, int causal,
+                               float sm_scale, int8_t* q_codes, float* q_scale, float* q_mean,
+                               int8_t* k_codes, float* k_scale, float* k_mean, uint8_t* v_codes,
+                               float* v_scale, float* q_bias, void* ws, size_t ws_bytes,
+                               void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !in_dtype_ok(in_dt) ||
+      !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes) ||
+      !q_scale || !aligned16(q_mean) || !k_scale || !aligned16(k_mean) || !aligned16(q_bias) ||
+      !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
+  const Layout L = dense_layout(B, H, N, D, fp8, Hkv);
+  if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
+  return quantize_dense_sq(q, k, v, in_dt, B, H, N, D, pv_mode, causal, sm_scale, q_codes,
+                           q_scale, q_mean, k_codes, k_scale, k_mean, v_codes, v_scale, q_bias,
+                           ws, L, as_stream(stream), Hkv);
+}
+
+sage_status_t sage_attn_quantized_sq(const int8_t* q_codes, const float* q_scale,
+                                     const int8_t* k_codes, const float* k_scale,
+                                     const float* q_bias, const void* v, const uint8_t* v_codes,
+                                     const float* v_scale, void* out, int v_dt, int out_dt, int B,
+                                     int H, int Hkv, int N, int D, int causal, float sm_scale,
+                                     int pv_mode, void* ws, size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !out_dtype_ok(out_dt) ||
+      !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !k_scale || !aligned16(q_bias) ||
+      !aligned16(out) || !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+    return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
+  return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
+                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), Hkv, 2, q_bias);
+}
+
 size_t sage_workspace_bytes_ex(int B, int H, int Hkv, int N, int D, int pv_mode, int qk_gran) {
   if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv) || !gran_ok(qk_gran)) return 0;
-  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv, qk_gran == SAGE_QK_PER_TOKEN).total;
+  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv, qk_gran).total;
 }
 
 sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int in_dt,
@@ -360,9 +453,23 @@ sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8, tok = qk_gran == SAGE_QK_PER_TOKEN;
-  const Layout L = dense_layout(B, H, N, D, fp8, Hkv, tok);
+  const Layout L = dense_layout(B, H, N, D, fp8, Hkv, qk_gran);
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
+  if (qk_gran == SAGE_QK_PER_BLOCK_SMOOTH_Q) {
+    sage_status_t r = quantize_dense_sq(
+        q, k, v, in_dt, B, H, N, D, pv_mode, causal, sm_scale, at<int8_t>(ws, L.q_codes),
+        at<float>(ws, L.q_scale), at<float>(ws, L.q_mean), at<int8_t>(ws, L.k_codes),
+        at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
+        fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr, fp8 ? at<float>(ws, L.v_scale) : nullptr,
+        at<float>(ws, L.q_bias), ws, L, st, Hkv);
+    if (r != SAGE_OK) return r;
+    return attn_dense(at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
+                      at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), v,
+                      fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
+                      fp8 ? at<float>(ws, L.v_scale) : nullptr, out, in_dt, out_dt, B, H, N, D,
+                      causal, sm_scale, pv_mode, ws, st, Hkv, 2, at<float>(ws, L.q_bias));
+  }
   sage_status_t r = quantize_dense(
       q, k, v, in_dt, B, H, N, D, pv_mode, at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
       at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
@@ -461,7 +568,7 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
                                        int Hkv, int D, int causal, float sm_scale, int pv_mode,
                                        int qk_gran, void* ws, size_t ws_bytes, void* stream) {
   if (!varlen_args_ok(total_tokens, batch, max_seqlen, H, D, pv_mode) || !gqa_heads_ok(H, Hkv) ||
-      !gran_ok(qk_gran) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
+      !gran_varlen_ok(qk_gran) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
       !std::isfinite(sm_scale))
     return SAGE_ERR_INVALID_ARG;
   const int tok = qk_gran == SAGE_QK_PER_TOKEN ? 1 : 0;
@@ -529,7 +636,7 @@ sage_status_t sage_attn_fwd_varlen(const void* q, const void* k, const void* v, 
 size_t sage_workspace_bytes_varlen_ex(int total_tokens, int batch, int H, int Hkv, int D,
                                       int pv_mode, int qk_gran) {
   if (!varlen_args_ok(total_tokens, batch, 0, H, D, pv_mode) || !gqa_heads_ok(H, Hkv) ||
-      !gran_ok(qk_gran))
+      !gran_varlen_ok(qk_gran))
     return 0;
   return varlen_layout(total_tokens, batch, H, D, pv_mode == SAGE_PV_FP8, Hkv,
                        qk_gran == SAGE_QK_PER_TOKEN).total;

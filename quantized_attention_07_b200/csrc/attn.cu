@@ -50,7 +50,7 @@ namespace {
 
 constexpr int SUB = 64;  // keys per softmax sub-tile
 
-template <int D, bool PV8, bool TOK>
+template <int D, bool PV8, int GR>
 struct Cfg {
   // warpgroups: 2 softmax, 1 control
   static constexpr int WGS = 3;
@@ -65,7 +65,9 @@ struct Cfg {
 
   static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
   static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
-  static constexpr int KS = TOK ? BLK * 4 : 0;          // per-token K deltas of a stage
+  // per stage, on the K barrier: the 128 per-token K deltas (GR 1), or the
+  // Q-smoothing term of both query tiles for the stage's keys (GR 2)
+  static constexpr int KS = GR == 1 ? BLK * 4 : GR == 2 ? 2 * BLK * 4 : 0;
   static constexpr int AUX = 1024;                      // barriers
   static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - AUX;
   static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT + KS);
@@ -243,11 +245,12 @@ __device__ __forceinline__ bool take_item(Bars* B, int r, uint32_t* status, bool
 
 // --------------------------------------------------------------- producer --
 
-template <int D, bool PV8, bool TOK>
+template <int D, bool PV8, int GR>
 __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                          const AttnParams& p, Bars* B, uint8_t* sQ, uint8_t* sK, uint8_t* sV,
                          float* sKs) {
-  using C = Cfg<D, PV8, TOK>;
+  using C = Cfg<D, PV8, GR>;
+  [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
   // The whole warp runs this loop (uniform control flow); one elected lane
   // issues each TMA instruction.  Stages form one ring across the CTA's work
   // items: G counts the stages loaded so far.
@@ -300,7 +303,19 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
         break;
       }
       if (ptx::elect_one()) {
-        ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);
+        if constexpr (SMQ) {
+          // Q smoothing: each present query tile's mean term for the stage's
+          // 128 keys, on the K barrier (a tile without keys has no bias row)
+          const int nt_q = w.nsub1 > 0 ? 2 : 1;
+          ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + nt_q * BLK * 4);
+          for (int tq = 0; tq < nt_q; ++tq)
+            ptx::bulk_load_plain(sKs + (s * 2 + tq) * BLK,
+                                 p.q_bias + ((long long)w.code_z * p.NB + 2 * w.pair + tq) *
+                                                (long long)p.NB * BLK + (long long)j * BLK,
+                                 BLK * 4, &B->k_full[s]);
+        } else {
+          ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);
+        }
         ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
         if constexpr (TOK)  // the stage's 128 per-token K deltas, on the same barrier
           ptx::bulk_load_plain(sKs + s * BLK, p.k_scale + (w.ks_idx0 + j) * BLK, C::KS,
@@ -339,10 +354,11 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
 // Issue order per thread is execution order, so S_t(i+2) never overwrites
 // P_t(i) before P.V has read it.  A 128-key stage is released to the producer
 // when both tiles' warps have committed it (kv_empty counts two arrivals).
-template <int D, bool PV8, bool BF16V, bool TOK>
+template <int D, bool PV8, bool BF16V, int GR>
 __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const uint8_t* sQ,
                            const uint8_t* sK, const uint8_t* sV, int t) {
-  using C = Cfg<D, PV8, TOK>;
+  using C = Cfg<D, PV8, GR>;
+  [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
   constexpr uint32_t IDESC_QK = ptx::instr_desc(2, 1, 1, 0, 0, 128, SUB);
   constexpr uint32_t IDESC_PV =
       PV8 ? ptx::instr_desc(1, 0, 0, 0, 1, 128, D)
@@ -524,6 +540,30 @@ __device__ __forceinline__ float row_scale_max(uint32_t* v, const float* dk, int
   return fmaxf(m0, m1);
 }
 
+// Q smoothing: y = fma(S, c, bk_j) written back over S (fp32 bit patterns),
+// the mean term bk (kappa applied) joining before the maximum; returns max y
+// over the unmasked columns (-inf if none).
+template <int NC, bool MASKED>
+__device__ __forceinline__ float row_bias_max(uint32_t* v, const float* bk, float c, int first_key,
+                                              int limit) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < NC; j += 4) {
+    const float4 b = *reinterpret_cast<const float4*>(bk + j);
+    const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float y = __fmaf_rn((float)(int)v[j + e], c, bb[e]);
+      v[j + e] = __float_as_uint(y);
+      if (!MASKED || first_key + j + e < limit) {
+        if (e & 1) m1 = fmaxf(m1, y);
+        else m0 = fmaxf(m0, y);
+      }
+    }
+  }
+  return fmaxf(m0, m1);
+}
+
 // Share of the exponentials computed by the FMA-pipe polynomial: one pair in
 // POLY_EVERY (0 = none; every 2^x on the special-function unit).
 constexpr int POLY_EVERY = 0;
@@ -563,11 +603,12 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
   return s.x + s.y;
 }
 
-template <int D, bool PV8, bool BF16V, bool TOK>
+template <int D, bool PV8, bool BF16V, int GR>
 __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w, Bars* B,
                                              uint32_t tmem, int t, const float* sKs, int I0,
                                              int G0, volatile int* loop) {
-  using C = Cfg<D, PV8, TOK>;
+  using C = Cfg<D, PV8, GR>;
+  [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
   using In = In16<BF16V>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
@@ -614,6 +655,12 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
         const float ym = full_tile ? row_scale_max<SUB, false>(sv, dk, key0, limit)
                                    : row_scale_max<SUB, true>(sv, dk, key0, limit);
         m_blk = ym == -INFINITY ? -INFINITY : __fmul_rn(ym, c);
+      } else if constexpr (SMQ) {
+        const int g = G0 + i / 2;  // the mean term came with the K stage
+        if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, p.status, true)) return false;
+        const float* bk = sKs + ((g % C::NS) * 2 + t) * BLK + (i & 1) * SUB;
+        m_blk = full_tile ? row_bias_max<SUB, false>(sv, bk, c, key0, limit)
+                          : row_bias_max<SUB, true>(sv, bk, c, key0, limit);
       } else {
         const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
                                    : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
@@ -622,6 +669,9 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
       return true;
     };
 
+    // multiplier inside the exponent: c, or 1 once S holds the scaled logit
+    // (Q smoothing: arg = fp32(y - m))
+    const float ce = SMQ ? 1.0f : c;
     if constexpr (!PV8) {
       uint32_t sv[SUB];
 #pragma unroll
@@ -636,8 +686,8 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
 #pragma unroll
       for (int cc = 0; cc < SUB / 32; ++cc) {
         float pv[32];
-        rowsum += full_tile ? row_exp<false, 32, TOK>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv)
-                            : row_exp<true, 32, TOK>(sv + 32 * cc, c, -m_new, key0 + 32 * cc, limit, pv);
+        rowsum += full_tile ? row_exp<false, 32, TOK || SMQ>(sv + 32 * cc, ce, -m_new, key0 + 32 * cc, limit, pv)
+                            : row_exp<true, 32, TOK || SMQ>(sv + 32 * cc, ce, -m_new, key0 + 32 * cc, limit, pv);
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) packed[k] = In::pack(pv[2 * k], pv[2 * k + 1]);
@@ -678,8 +728,8 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
 #pragma unroll
       for (int cc = 0; cc < SUB / 16; ++cc) {
         float pv[16];
-        rowsum += full_tile ? row_exp<false, 16, TOK>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv)
-                            : row_exp<true, 16, TOK>(sv + 16 * cc, c, -m_new, key0 + 16 * cc, limit, pv);
+        rowsum += full_tile ? row_exp<false, 16, TOK || SMQ>(sv + 16 * cc, ce, -m_new, key0 + 16 * cc, limit, pv)
+                            : row_exp<true, 16, TOK || SMQ>(sv + 16 * cc, ce, -m_new, key0 + 16 * cc, limit, pv);
         uint32_t packed[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -771,7 +821,7 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
 // tile's sub-tiles so far, G0 the ring stages, loop[1] the items with keys
 // (o_done phase).  The item counts sit in a per-warp shared-memory slot
 // rather than in registers, which the per-sub-tile loop needs.
-template <int D, bool PV8, bool BF16V, bool TOK>
+template <int D, bool PV8, bool BF16V, int GR>
 __device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, const float* sKs) {
   volatile int* loop = B->sm_loop[threadIdx.x / 32];  // [0] items taken, [1] items with keys
   loop[0] = 0;
@@ -786,7 +836,7 @@ __device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, c
     if (!w.valid) continue;
     const int nsub = t == 0 ? w.nsub0 : w.nsub1;
     if (nsub > 0) {
-      if (!softmax_item<D, PV8, BF16V, TOK>(p, w, B, tmem, t, sKs, I0, G0, loop)) return;
+      if (!softmax_item<D, PV8, BF16V, GR>(p, w, B, tmem, t, sKs, I0, G0, loop)) return;
       loop[1] = loop[1] + 1;
     }
     I0 += nsub;
@@ -796,17 +846,18 @@ __device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, c
 
 // ---------------------------------------------------------------- kernel --
 
-template <int D, bool PV8, bool BF16V, bool TOK>
-__global__ void __launch_bounds__(Cfg<D, PV8, TOK>::THREADS, 1)
+template <int D, bool PV8, bool BF16V, int GR>
+__global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using C = Cfg<D, PV8, TOK>;
+  using C = Cfg<D, PV8, GR>;
+  [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + 2 * C::QT;
   uint8_t* sV = sK + C::NS * C::QT;
-  float* sKs = reinterpret_cast<float*>(sV + C::NS * C::VT);  // TOK: [NS][128] K deltas
+  float* sKs = reinterpret_cast<float*>(sV + C::NS * C::VT);  // GR 1: [NS][128] K deltas; GR 2: [NS][2][128] mean terms
   Bars* B = reinterpret_cast<Bars*>(sV + C::NS * (C::VT + C::KS));
   static_assert(sizeof(Bars) <= C::AUX, "aux layout");
 
@@ -851,13 +902,13 @@ __global__ void __launch_bounds__(Cfg<D, PV8, TOK>::THREADS, 1)
   if (wg == C::WG_CTRL) {
     ptx::setmaxnreg_dec<C::REG_CTRL>();
     if (warp == warp_tma) {
-      producer<D, PV8, TOK>(&tm_q, &tm_k, &tm_v, p, B, sQ, sK, sV, sKs);
+      producer<D, PV8, GR>(&tm_q, &tm_k, &tm_v, p, B, sQ, sK, sV, sKs);
     } else if (warp == warp_mma || warp == warp_mma + 1) {
-      mma_issuer<D, PV8, BF16V, TOK>(p, B, tmem, sQ, sK, sV, warp - warp_mma);
+      mma_issuer<D, PV8, BF16V, GR>(p, B, tmem, sQ, sK, sV, warp - warp_mma);
     }
   } else {
     ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
-    softmax_wg<D, PV8, BF16V, TOK>(p, B, tmem, wg, sKs);
+    softmax_wg<D, PV8, BF16V, GR>(p, B, tmem, wg, sKs);
   }
 
   ptx::tc_fence_before();
@@ -995,9 +1046,10 @@ static CUtensorMapSwizzle swz_for(int row_bytes) {
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 }
 
-template <int D, bool PV8, bool BF16V, bool TOK>
+template <int D, bool PV8, bool BF16V, int GR>
 static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
-  using C = Cfg<D, PV8, TOK>;
+  using C = Cfg<D, PV8, GR>;
+  [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle cs = swz_for(D);
   if (!make_map3(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.q_codes, D, L.code_rows, L.code_z, D,
@@ -1019,7 +1071,7 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
     okv = make_map3(&tv, vdt, esz, L.v, D, L.code_z_kv, L.T, (uint64_t)D * esz,
                     (uint64_t)D * esz * L.code_z_kv, vbox0, 1, BLK, vs);
   if (!okv) return cudaErrorInvalidValue;
-  auto kern = attn_fwd_kernel<D, PV8, BF16V, TOK>;
+  auto kern = attn_fwd_kernel<D, PV8, BF16V, GR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -1031,20 +1083,21 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool TOK>
+template <int GR>
 static cudaError_t launch_attn_g(const AttnLaunch& L, cudaStream_t st) {
   if (L.D == 64) {
-    if (L.pv8) return launch_attn_t<64, true, false, TOK>(L, st);
-    return L.bf16v ? launch_attn_t<64, false, true, TOK>(L, st)
-                   : launch_attn_t<64, false, false, TOK>(L, st);
+    if (L.pv8) return launch_attn_t<64, true, false, GR>(L, st);
+    return L.bf16v ? launch_attn_t<64, false, true, GR>(L, st)
+                   : launch_attn_t<64, false, false, GR>(L, st);
   }
-  if (L.pv8) return launch_attn_t<128, true, false, TOK>(L, st);
-  return L.bf16v ? launch_attn_t<128, false, true, TOK>(L, st)
-                 : launch_attn_t<128, false, false, TOK>(L, st);
+  if (L.pv8) return launch_attn_t<128, true, false, GR>(L, st);
+  return L.bf16v ? launch_attn_t<128, false, true, GR>(L, st)
+                 : launch_attn_t<128, false, false, GR>(L, st);
 }
 
 cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st) {
-  return L.p.per_token ? launch_attn_g<true>(L, st) : launch_attn_g<false>(L, st);
+  if (L.p.per_token == 2) return launch_attn_g<2>(L, st);
+  return L.p.per_token ? launch_attn_g<1>(L, st) : launch_attn_g<0>(L, st);
 }
 
 template <int D>

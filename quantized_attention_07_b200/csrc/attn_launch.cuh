@@ -11,7 +11,9 @@ struct AttnParams {
   int NB;                // dense: key blocks per head = ceil(N/128)
   int NPAIR;             // dense: query tile pairs per head = ceil(N/256)
   int causal;
-  int per_token;         // dense: one delta per token ([BH][NP] / [B*Hkv][NP]), not per block
+  int per_token;         // 1: one delta per token ([BH][NP] / [B*Hkv][NP]), not per block;
+                         // 2 (dense): per block, Q smoothed (q_bias holds the mean term)
+  const float* q_bias;   // per_token 2: [BH][NB][NB*128] fp32, kappa applied
   float kappa;           // fp32(sm_scale * log2 e)
   const float* q_scale;  // dense [BH][NB]; varlen [H][TBmax]
   const float* k_scale;

@@ -436,6 +436,164 @@ __global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
                             tok);
 }
 
+// ------------------------------------------------------------ Q smoothing --
+//
+// SageAttention2's smoothing of Q (dtcms.com page, v2 bullet 2): each
+// 128-token query block I is quantised after subtracting its own channel mean
+// qmean_I, and the part of the logit that the mean carries, qmean_I . k~_j,
+// is added back per key by the attention kernel.
+
+// One CTA per (query block, head): the exact block mean (the K mean's
+// fixed-point sum, over this block's rows), then per-block codes of
+// fp32(q - qmean_I) with one delta, as the K blocks are coded.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(THREADS) quant_q_smooth_kernel(
+    int N, const void* __restrict__ q, int8_t* __restrict__ q_codes,
+    float* __restrict__ q_scale, float* __restrict__ q_mean, uint32_t* __restrict__ status) {
+  using T = Tile<D>;
+  __shared__ float red[THREADS / 32];
+  __shared__ long long red64[THREADS / 32][D];
+  __shared__ float s_mean[D];
+  SeqLayout L{};
+  L.N = N;
+  BlockPos P;
+  dense_block_pos(L, blockIdx.y, blockIdx.x, P);
+  const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
+  const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
+
+  uint4 rq[T::NIT];
+  load_raw<D>(q, P, rq);
+  float x[T::NIT][8];
+  to_float<D, BF16>(rq, x);
+
+  // exact channel sums of rint(x * 2^24) (padding rows are zeros)
+  long long acc[8];
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0;
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float xv = x[i][e];
+      if (fabsf(xv) < 65536.0f) acc[e] += __float2ll_rn(__fmul_rn(xv, 16777216.0f));
+      else bad = true;  // non-finite or out of the exact-mean range
+    }
+  if (bad) set_status(status, ST_RANGE);
+#pragma unroll
+  for (int o = T::CPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  if (lane < T::CPR)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red64[w][8 * c + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    long long sum = 0;
+#pragma unroll
+    for (int i = 0; i < THREADS / 32; ++i) sum += red64[i][threadIdx.x];
+    const float mu = k_mean_value((unsigned long long)sum, P.rows);
+    s_mean[threadIdx.x] = mu;
+    q_mean[P.scale_idx * D + threadIdx.x] = mu;
+  }
+  __syncthreads();
+
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = s_mean[8 * c + e];
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < T::NIT; ++i) {
+    const bool valid = (r0 + i * T::RS) < P.rows;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      x[i][e] = valid ? __fsub_rn(x[i][e], m[e]) : 0.0f;
+      a = fmaxf(a, fabsf(x[i][e]));
+    }
+  }
+  const float amax = block_max(a, red);
+  store_codes<D>(x, amax, q_codes, P.code_row0);
+  if (threadIdx.x == 0) q_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+}
+
+// The per-key term: bias[bh][I][j] = fp32(kappa * sum_d qmean_I[d] k~_j[d]),
+// k~_j = fp32(k_j - kmean) of the key/value head that query head bh reads.
+// The sum is taken in fp64 in channel order (each product of two fp32 values
+// is exact in fp64), then multiplied by kappa and rounded once to fp32: the
+// value, and so every FP8 code of P that depends on it, does not hinge on a
+// summation order of this kernel's choosing.
+// One CTA per (128-key tile J, query head), one thread per key: the thread
+// keeps its k~ row in registers and runs over the query blocks, G at a time,
+// whose means the CTA first stages in shared memory as fp64 (every thread
+// then reads the same address: a broadcast).  With a causal mask, blocks
+// I < J never see the tile and are skipped.  Keys past N get 0.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128) q_smooth_bias_kernel(
+    int N, int H, int Hkv, int causal, float kappa, const void* __restrict__ k,
+    const float* __restrict__ k_mean, const float* __restrict__ q_mean,
+    float* __restrict__ bias) {
+  constexpr int G = 8;                 // query blocks per pass
+  __shared__ double s_qm[D][G];        // means of G blocks, channel-major
+  const int NB = (N + BLK - 1) / BLK;
+  const int J = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / H, h = bh - b * H;
+  const int bkv = b * Hkv + h / (H / Hkv);
+  const int j = J * BLK + threadIdx.x;
+  float kt[D];
+  if (j < N) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(k) +
+                                                      ((long long)bkv * N + j) * D);
+    const float2* km = reinterpret_cast<const float2*>(k_mean + (long long)bkv * D);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 u = __ldg(src + c);
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = In16<BF16>::to_float2(wv[e]);
+        const float2 mu = __ldg(km + 4 * c + e);
+        kt[8 * c + 2 * e] = __fsub_rn(f.x, mu.x);
+        kt[8 * c + 2 * e + 1] = __fsub_rn(f.y, mu.y);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; ++c) kt[c] = 0.0f;
+  }
+  const long long NP = (long long)NB * BLK;
+  const float* qm = q_mean + (long long)bh * NB * D;
+  float* out = bias + (long long)bh * NB * NP + j;
+  const double kap = (double)kappa;
+  for (int I0 = causal ? J : 0; I0 < NB; I0 += G) {
+    __syncthreads();  // the previous group's means are no longer read
+    for (int x = threadIdx.x; x < G * D; x += 128) {
+      const int g = x / D, d = x - g * D;
+      s_qm[d][g] = I0 + g < NB ? (double)__ldg(qm + (long long)(I0 + g) * D + d) : 0.0;
+    }
+    __syncthreads();
+    double acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.0;
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      // converted where used (volatile: not hoisted out of the block loop,
+      // which would hold D doubles in registers)
+      double kd;
+      asm volatile("cvt.f64.f32 %0, %1;" : "=d"(kd) : "f"(kt[d]));
+      const double2* m2 = reinterpret_cast<const double2*>(&s_qm[d][0]);
+#pragma unroll
+      for (int g2 = 0; g2 < G / 2; ++g2) {
+        const double2 m = m2[g2];
+        acc[2 * g2] = __fma_rn(m.x, kd, acc[2 * g2]);
+        acc[2 * g2 + 1] = __fma_rn(m.y, kd, acc[2 * g2 + 1]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      if (I0 + g < NB) out[(long long)(I0 + g) * NP] = __double2float_rn(__dmul_rn(acc[g], kap));
+  }
+}
+
 // ---------------------------------------------------------- streamed, dense --
 //
 // Dense inputs: one persistent CTA per SM.  Warp 8 claims work items from a
@@ -1101,6 +1259,40 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
     else { if (fp8) SAGE_Q(128, false, true); else SAGE_Q(128, false, false); }
   }
 #undef SAGE_Q
+}
+
+// Q smoothing, dense [B*H, N, D] query heads: block means, codes and deltas
+// of the smoothed Q (grid: blocks x heads).
+cudaError_t launch_quant_q_smooth(int BH, int N, int D, bool bf16, const void* q,
+                                  int8_t* q_codes, float* q_scale, float* q_mean,
+                                  uint32_t* status, cudaStream_t st) {
+  const dim3 grid((N + BLK - 1) / BLK, BH);
+  if (D == 64) {
+    if (bf16) quant_q_smooth_kernel<64, true><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
+    else quant_q_smooth_kernel<64, false><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
+  } else {
+    if (bf16) quant_q_smooth_kernel<128, true><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
+    else quant_q_smooth_kernel<128, false><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
+  }
+  return cudaGetLastError();
+}
+
+// The per-key term of Q smoothing into bias [B*H][NB][NB*128] (fp32, kappa
+// applied); k is [B*Hkv, N, D], k_mean [B*Hkv, D], q_mean [B*H, NB, D].
+cudaError_t launch_q_smooth_bias(int B, int H, int Hkv, int N, int D, bool bf16, int causal,
+                                 float kappa, const void* k, const float* k_mean,
+                                 const float* q_mean, float* bias, cudaStream_t st) {
+  const dim3 grid((N + BLK - 1) / BLK, B * H);
+#define SAGE_B(DD, BB)                                                                     \
+  q_smooth_bias_kernel<DD, BB><<<grid, 128, 0, st>>>(N, H, Hkv, causal, kappa, k, k_mean, \
+                                                     q_mean, bias)
+  if (D == 64) {
+    if (bf16) SAGE_B(64, true); else SAGE_B(64, false);
+  } else {
+    if (bf16) SAGE_B(128, true); else SAGE_B(128, false);
+  }
+#undef SAGE_B
+  return cudaGetLastError();
 }
 
 }  // namespace sage

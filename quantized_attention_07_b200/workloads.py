@@ -18,6 +18,9 @@ Recipe (per workload):
     channel offset that K smoothing removes.
   * optional outliers: an independent Bernoulli(p) draw per Q and per K entry
     picks entries that are multiplied by a factor (after the bias is added).
+  * optional Q channel offset (the offset Q smoothing removes): q[d] += c[d],
+    c[d] ~ N(0, sigma_q^2) per (sequence, head, channel), drawn last so the
+    other draws do not depend on it.
   * varlen: sequence lengths are drawn uniformly (inclusive) from a range, and
     ``cu_seqlens`` is their prefix sum; the packed layout is [T, H, D].
   * grouped-query attention (Hkv < H): Q, K, V are drawn for H heads as above
@@ -53,7 +56,9 @@ class Workload:
     len_hi: int = 0
     seed: int = 0
     Hkv: int = 0                # key/value heads (grouped-query attention); 0: = H
-    qk_gran: str = "block"      # Q/K deltas per 128-token block or per token
+    qk_gran: str = "block"      # Q/K deltas per 128-token block, per token, or per block
+                                # with Q smoothing ("block_sq")
+    q_bias_sigma: float = 0.0   # Q channel offset (see the recipe)
 
     @property
     def kv_heads(self) -> int:
@@ -89,6 +94,12 @@ WORKLOADS = {
     "dit_8k_fp8_tok": Workload("dit_8k_fp8_tok", B=1, H=24, N=8192, D=64, dtype="fp16",
                                causal=False, pv_mode="fp8", bias_sigma=3.0, outlier_p=0.01,
                                outlier_scale=20.0, seed=20260003, qk_gran="token"),
+    # the video-DiT shape with Q smoothing (SageAttention2), on a Q that carries
+    # a channel offset like K
+    "dit_8k_fp8_sq": Workload("dit_8k_fp8_sq", B=1, H=24, N=8192, D=64, dtype="fp16",
+                              causal=False, pv_mode="fp8", bias_sigma=3.0, outlier_p=0.01,
+                              outlier_scale=20.0, seed=20260003, qk_gran="block_sq",
+                              q_bias_sigma=3.0),
 }
 
 
@@ -118,7 +129,8 @@ def _outliers(x: torch.Tensor, g: torch.Generator, p: float, scale: float) -> to
 
 def make_dense(B: int, H: int, N: int, D: int, dtype: str = "fp16", bias_sigma: float = 3.0,
                outlier_p: float = 0.0, outlier_scale: float = 1.0, seed: int = 0,
-               k_const_over_tokens: bool = False) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+               k_const_over_tokens: bool = False,
+               q_bias_sigma: float = 0.0) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Dense [B,H,N,D] q, k, v drawn by the recipe in the module docstring."""
     g = torch.Generator().manual_seed(seed)
     q = torch.randn((B, H, N, D), generator=g)
@@ -130,6 +142,8 @@ def make_dense(B: int, H: int, N: int, D: int, dtype: str = "fp16", bias_sigma: 
     k = k + bias
     q = _outliers(q, g, outlier_p, outlier_scale)
     k = _outliers(k, g, outlier_p, outlier_scale)
+    if q_bias_sigma > 0.0:
+        q = q + torch.randn((B, H, 1, D), generator=g) * q_bias_sigma
     t = DTYPES[dtype]
     return q.to(t), k.to(t), v.to(t)
 
@@ -163,7 +177,7 @@ def make_inputs(wl: Workload) -> Inputs:
         q, k, v, cu = make_varlen(lens, wl.H, wl.D, wl.dtype, wl.bias_sigma, seed=wl.seed + 1)
         return Inputs(q, k, v, cu, wl)
     q, k, v = make_dense(wl.B, wl.H, wl.N, wl.D, wl.dtype, wl.bias_sigma, wl.outlier_p,
-                         wl.outlier_scale, seed=wl.seed)
+                         wl.outlier_scale, seed=wl.seed, q_bias_sigma=wl.q_bias_sigma)
     if wl.kv_heads != wl.H:
         k, v = k[:, :wl.kv_heads].contiguous(), v[:, :wl.kv_heads].contiguous()
     return Inputs(q, k, v, None, wl)

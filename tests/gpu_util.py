@@ -21,10 +21,10 @@ def half_ulp(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
     return 0.5 * np.exp2(e - mant)
 
 
-def gpu_quantize_dense(q, k, v, pv_mode, qk_gran="block"):
+def gpu_quantize_dense(q, k, v, pv_mode, qk_gran="block", causal=False, sm_scale=None):
     dev = torch.device("cuda")
     qz = sage.quantize(q.to(dev), k.to(dev), v.to(dev) if v is not None else None, pv_mode,
-                       qk_gran=qk_gran)
+                       qk_gran=qk_gran, causal=causal, sm_scale=sm_scale)
     torch.cuda.synchronize()
     sage.sync_status()
     return qz
@@ -122,7 +122,8 @@ def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
             g = q.shape[1] // k.shape[1]
             k, v = heads.repeat_kv_packed(k, g), heads.repeat_kv_packed(v, g)
     qz = heads.quantize(q, k, v, cu, pv_mode, gran=qk_gran)
-    emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran)
+    emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran,
+                             k=k if qk_gran == "block_sq" else None)
     ref = heads.reference_rows(q, k, v, cu, picks, causal, sm_scale)
     E = np.stack([emu[p] for p in picks])
     R = np.stack([ref[p] for p in picks])
