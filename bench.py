@@ -354,6 +354,15 @@ def run_ours(args, rank, world, local):
         "clocks": clocks,
         "gpu_launches": launches_per_step * K,
     }
+    qb = quant_algorithmic_bytes(wl)
+    if qb and not grouped and not wl.varlen:
+        # stage 1 (K smoothing + quantisation) against the copy bandwidth
+        qms = statistics.mean(quant_ms)
+        gbs = qb / (qms * 1e-3) / 1e9
+        line["quantisation"] = {"bound": "hbm", "ms": round(qms, 4), "algorithmic_bytes": qb,
+                                "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                "frac": round(gbs / pk["hbm_gbs"], 4),
+                                "launches_per_step": launches_per_step - 1}
     if e2e:
         line["e2e"] = e2e
     if cpu:
@@ -362,6 +371,25 @@ def run_ours(args, rank, world, local):
 
 
 # -------------------------------------------------------------- oracle arm --
+
+def quant_algorithmic_bytes(wl) -> int:
+    """Bytes stage 1 must move for a dense workload: Q and K read (2 B per
+    element) and their int8 codes written (1 B), FP8 P.V: V read and its e4m3
+    codes written (3 B); per-token deltas 4 B per row of Q and K; Q smoothing:
+    the fp32 per-key mean term written (4 B per query block and key).  The
+    second pass over K (its mean first) is overhead, not counted."""
+    if wl.varlen:
+        return 0
+    NB = (wl.N + 127) // 128
+    q_el = wl.B * wl.H * wl.N * wl.D
+    kv_el = wl.B * wl.kv_heads * wl.N * wl.D
+    b = 3 * q_el + 3 * kv_el + (3 * kv_el if wl.pv_mode == "fp8" else 0)
+    if wl.qk_gran == "token":
+        b += 4 * wl.N * (wl.B * wl.H + wl.B * wl.kv_heads)
+    if wl.qk_gran == "block_sq":
+        b += 4 * wl.B * wl.H * NB * NB * 128
+    return b
+
 
 def cpu_oracle_throughput(wl, inp, budget_rows: int, quant_heads: int, seed: int = 7) -> dict:
     """Time the CPU oracle (quantisation + emulated attention rows) on a bounded

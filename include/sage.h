@@ -150,8 +150,8 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
  * With SAGE_QK_PER_BLOCK_SMOOTH_Q the codes of query block I are those of
  * fp32(q - qmean_I), qmean_I the exact channel mean of the block's rows (the
  * K mean's definition), and the scaled logit is y = fmaf(S, c, b_Ij) with
- * b_Ij = fp32(kappa * qmean_I . fp32(k_j - kmean)), the dot product summed in
- * fp64 in channel order, then arg = y - m.
+ * b_Ij = fp32(kappa * qmean_I . fp32(k_j - kmean)), the dot product as fp32
+ * fused multiply-adds in channel order, then arg = y - m.
  * Its workspace also holds qmean and b (B*H*NB*(D + NB*128) floats).
  *   ws : at least sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, qk_gran).
  * sage_attn_fwd(...) = sage_attn_fwd_ex(..., Hkv = H, ..., SAGE_QK_PER_BLOCK).
@@ -288,7 +288,8 @@ sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale
  * per-block deltas,
  *   q_mean : fp32 [B, H, NB, D], the block means of Q;
  *   q_bias : fp32 [B, H, NB, NP], q_bias[b,h,I,j] = fp32(kappa * q_mean[b,h,I]
- *            . fp32(k_j - k_mean)) for key j of the key/value head of h, kappa
+ *            . fp32(k_j - k_mean)) (fp32 FMAs in channel order) for key j of the
+ *            key/value head of h, kappa
  *            = fp32(sm_scale * log2 e); keys j >= N give 0; with causal != 0
  *            the blocks I < j/128, which the mask hides, are not written.
  *            16-byte aligned.

@@ -181,7 +181,8 @@ def attn_ref_rows(q, k, v, sm_scale: float, causal: bool, rows) -> np.ndarray:
 def q_smooth_bias(qmean: np.ndarray, k: np.ndarray, kmean: np.ndarray, sm_scale: float,
                   ldo: Optional[int] = None) -> np.ndarray:
     """Per-key term of Q smoothing for one head: [nb, ldo] fp32 with
-    out[I, j] = fp32(kappa * qmean[I] . (k[j] - kmean)) for j < n (0 beyond).
+    out[I, j] = fp32(kappa * qmean[I] . (k[j] - kmean)) for j < n (0 beyond),
+    the dot product as fp32 fused multiply-adds in channel order.
     qmean: [nb, D] block means of Q; k: [n, D]; kmean: [D]."""
     qmean, k, kmean = _f32(qmean), _f32(k), _f32(kmean)
     nb, D = qmean.shape

@@ -497,7 +497,12 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
  * smoothing; the term here uses the smoothed k~ = fp32(k - kmean) that the K
  * codes come from.)
  *
- *   out[I*ldo + j] = fp32( kappa * sum_d qmean[I][d] * k~_j[d] )   (fp64 sum)
+ *   acc    = 0;  acc = fmaf(qmean[I][d], k~_j[d], acc)  for d = 0 .. D-1
+ *   out[I*ldo + j] = fp32(acc * kappa)
+ *
+ * The pages fix no precision for this dot product; it is the kernel's: fp32
+ * fused multiply-adds in channel order, so that the term, and every FP8 code
+ * of P that depends on it, agrees bit for bit.
  *
  * qmean: [nb][D]; k: row j at k + j*ld; kmean: [D]; out: [nb][ldo], columns
  * j < n written.
@@ -507,12 +512,12 @@ void oracle_q_smooth_bias(const float* qmean, long nb, const float* k, long n, i
 {
     for (long I = 0; I < nb; ++I) {
         for (long j = 0; j < n; ++j) {
-            double acc = 0.0;
+            float acc = 0.0f;
             for (int d = 0; d < D; ++d) {
                 const float ks = k[j * ld + d] - kmean[d];
-                acc += (double)qmean[I * D + d] * (double)ks;
+                acc = fmaf(qmean[I * D + d], ks, acc);
             }
-            out[I * ldo + j] = (float)(acc * (double)kappa);
+            out[I * ldo + j] = acc * kappa;
         }
     }
 }

@@ -516,24 +516,24 @@ __global__ void __launch_bounds__(THREADS) quant_q_smooth_kernel(
   if (threadIdx.x == 0) q_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
 }
 
-// The per-key term: bias[bh][I][j] = fp32(kappa * sum_d qmean_I[d] k~_j[d]),
-// k~_j = fp32(k_j - kmean) of the key/value head that query head bh reads.
-// The sum is taken in fp64 in channel order (each product of two fp32 values
-// is exact in fp64), then multiplied by kappa and rounded once to fp32: the
-// value, and so every FP8 code of P that depends on it, does not hinge on a
-// summation order of this kernel's choosing.
+// The per-key term: bias[bh][I][j] = fp32(acc * kappa), acc the fp32 fused
+// multiply-adds of qmean_I[d] and k~_j[d] = fp32(k_j[d] - kmean[d]) in
+// channel order, for the key/value head that query head bh reads.  The fixed
+// order makes the value (and every FP8 code of P that depends on it) the
+// oracle's, bit for bit.
 // One CTA per (128-key tile J, query head), one thread per key: the thread
-// keeps its k~ row in registers and runs over the query blocks, G at a time,
-// whose means the CTA first stages in shared memory as fp64 (every thread
-// then reads the same address: a broadcast).  With a causal mask, blocks
-// I < J never see the tile and are skipped.  Keys past N get 0.
+// keeps its k~ row in registers and runs over the query blocks, G at a time
+// (G independent accumulators, paired into packed FMAs), whose means the CTA
+// first stages in shared memory channel-major (every thread then reads the
+// same address: a broadcast).  With a causal mask, blocks I < J never see the
+// tile and are skipped.  Keys past N get 0.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
     int N, int H, int Hkv, int causal, float kappa, const void* __restrict__ k,
     const float* __restrict__ k_mean, const float* __restrict__ q_mean,
     float* __restrict__ bias) {
   constexpr int G = 8;                 // query blocks per pass
-  __shared__ double s_qm[D][G];        // means of G blocks, channel-major
+  __shared__ __align__(16) float s_qm[D][G];  // means of G blocks, channel-major
   const int NB = (N + BLK - 1) / BLK;
   const int J = blockIdx.x, bh = blockIdx.y;
   const int b = bh / H, h = bh - b * H;
@@ -563,34 +563,33 @@ __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
   const long long NP = (long long)NB * BLK;
   const float* qm = q_mean + (long long)bh * NB * D;
   float* out = bias + (long long)bh * NB * NP + j;
-  const double kap = (double)kappa;
   for (int I0 = causal ? J : 0; I0 < NB; I0 += G) {
     __syncthreads();  // the previous group's means are no longer read
     for (int x = threadIdx.x; x < G * D; x += 128) {
       const int g = x / D, d = x - g * D;
-      s_qm[d][g] = I0 + g < NB ? (double)__ldg(qm + (long long)(I0 + g) * D + d) : 0.0;
+      s_qm[d][g] = I0 + g < NB ? __ldg(qm + (long long)(I0 + g) * D + d) : 0.0f;
     }
     __syncthreads();
-    double acc[G];
+    float2 acc[G / 2];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.0;
+    for (int g2 = 0; g2 < G / 2; ++g2) acc[g2] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int d = 0; d < D; ++d) {
-      // converted where used (volatile: not hoisted out of the block loop,
-      // which would hold D doubles in registers)
-      double kd;
-      asm volatile("cvt.f64.f32 %0, %1;" : "=d"(kd) : "f"(kt[d]));
-      const double2* m2 = reinterpret_cast<const double2*>(&s_qm[d][0]);
+      const float2 kd = make_float2(kt[d], kt[d]);
+      const float4* m4 = reinterpret_cast<const float4*>(&s_qm[d][0]);
 #pragma unroll
-      for (int g2 = 0; g2 < G / 2; ++g2) {
-        const double2 m = m2[g2];
-        acc[2 * g2] = __fma_rn(m.x, kd, acc[2 * g2]);
-        acc[2 * g2 + 1] = __fma_rn(m.y, kd, acc[2 * g2 + 1]);
+      for (int g4 = 0; g4 < G / 4; ++g4) {
+        const float4 m = m4[g4];
+        acc[2 * g4] = __ffma2_rn(make_float2(m.x, m.y), kd, acc[2 * g4]);
+        acc[2 * g4 + 1] = __ffma2_rn(make_float2(m.z, m.w), kd, acc[2 * g4 + 1]);
       }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-      if (I0 + g < NB) out[(long long)(I0 + g) * NP] = __double2float_rn(__dmul_rn(acc[g], kap));
+    for (int g2 = 0; g2 < G / 2; ++g2) {
+      if (I0 + 2 * g2 < NB) out[(long long)(I0 + 2 * g2) * NP] = __fmul_rn(acc[g2].x, kappa);
+      if (I0 + 2 * g2 + 1 < NB)
+        out[(long long)(I0 + 2 * g2 + 1) * NP] = __fmul_rn(acc[g2].y, kappa);
+    }
   }
 }
 
