@@ -86,15 +86,34 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
     """gran "block": one delta per 128-token block (deltas [B,H,NB] dense,
     [H, TB] varlen); "token": one delta per token, the quantiser applied to
     one-row blocks, stored like the code rows (deltas [B,H,NP] dense,
-    [H, TB*128] varlen; padding rows 0); "block_sq" (dense only): per-block
-    deltas of Q smoothed by its block mean (SageAttention2's smoothing of Q),
-    the means in q_mean [B,H,NB,D]."""
+    [H, TB*128] varlen; padding rows 0); "block_sq": per-block deltas of Q
+    smoothed by its block mean (SageAttention2's smoothing of Q), the means in
+    q_mean ([B,H,NB,D] dense, [H,TB,D] varlen)."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     status = 0
     tok = gran == "token"
+    if gran == "block_sq" and cu is not None:
+        # per sequence: Q blocks smoothed by their own means (q_mean [H, TB, D],
+        # indexed like the deltas); K and V as for "block"
+        qz = quantize(q, k, v, cu_seqlens, pv_mode, "block")
+        T, H, D = q.shape
+        S = len(cu) - 1
+        nblk = [(cu[s + 1] - cu[s] + BLK - 1) // BLK for s in range(S)]
+        boff = np.concatenate([[0], np.cumsum(nblk)]).astype(np.int64)
+        TB = int(boff[-1])
+        qc = np.zeros((H, TB * BLK, D), np.int8)
+        qd = np.zeros((H, TB), np.float32)
+        qm = np.zeros((H, TB, D), np.float32)
+        for s, h, x in _heads(q, cu):
+            for I in range(nblk[s]):
+                xb = np.ascontiguousarray(x[I * BLK:(I + 1) * BLK])
+                g = int(boff[s]) + I
+                _, qm[h, g], st = k_mean(xb)
+                status |= st
+                qc[h, g * BLK:g * BLK + xb.shape[0]], qd[h, g] = quant_block(xb, qm[h, g])
+        return Quantized(qc, qd, qz.k_codes, qz.k_delta, qz.k_sum, qz.k_mean, qz.v_codes,
+                         qz.v_delta, status | qz.status, qm)
     if gran == "block_sq":
-        if cu is not None:
-            raise ValueError("Q smoothing is defined here for dense inputs")
         qz = quantize(q, k, v, None, pv_mode, "block")  # K and V as for "block"
         B, H, N, D = q.shape
         NB = (N + BLK - 1) // BLK
@@ -203,8 +222,8 @@ def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, caus
                  seqlens: Optional[list[int]] = None, gran: str = "block",
                  k: Optional[torch.Tensor] = None) -> dict:
     """E for the listed (seq, head, row) picks -> {pick: fp32 [D]}.  gran
-    "block_sq" needs k (dense, [B,H,N,D], one head per query head) for the
-    per-key term of Q smoothing."""
+    "block_sq" needs k (one head per query head; dense [B,H,N,D] or packed
+    [T,H,D]) for the per-key term of Q smoothing."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     sm_scale = default_sm_scale(D) if sm_scale is None else sm_scale
     p16 = "bf16" if v.dtype == torch.bfloat16 else "fp16"
@@ -217,8 +236,14 @@ def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, caus
         if pv_mode == "fp16":
             vv = vf[s, h] if cu is None else np.ascontiguousarray(vf[cu[s]:cu[s + 1], h])
         bias = None
-        if gran == "block_sq":
+        if gran == "block_sq" and cu is None:
             bias = q_smooth_bias(qz.q_mean[s, h], k[s, h].float().numpy(), qz.k_mean[s, h],
+                                 sm_scale)
+        elif gran == "block_sq":
+            b0 = sum((cu[i + 1] - cu[i] + BLK - 1) // BLK for i in range(s))
+            nb = (n + BLK - 1) // BLK
+            bias = q_smooth_bias(qz.q_mean[h, b0:b0 + nb],
+                                 k[cu[s]:cu[s + 1], h].float().numpy(), qz.k_mean[s, h],
                                  sm_scale)
         o = attn_emul_rows(qc, qd, kc, kd, n, D, sm_scale, causal, pv_mode, rows, v=vv, p16=p16,
                            vc=vc, vdelta=vd, per_token=gran == "token", bias=bias)

@@ -12,7 +12,8 @@ scaled logit.  The pins below fix it from outside the oracle:
   mis-signed mean term, a mean taken over the wrong block, or codes of the
   unsmoothed q all miss by orders of magnitude;
 - zero block means: smoothing is then the identity, and the emulation must be
-  bit-identical to the plain per-block one.
+  bit-identical to the plain per-block one;
+- a packed batch of one sequence is the dense problem: bit-identical.
 """
 from __future__ import annotations
 
@@ -90,8 +91,9 @@ def test_exact_inputs_reach_fp64_attention(N, D, causal):
 
 
 def test_bias_is_per_block_and_per_key():
-    """q_smooth_bias against its definition on dyadic values, where the fp64 sum
-    is exact: out[I, j] = fp32(kappa * qmean_I . (k_j - kmean))."""
+    """q_smooth_bias against its definition on dyadic values, where every fp32
+    partial sum is exact (so the fp64 matrix product gives the same sum):
+    out[I, j] = fp32(kappa * qmean_I . (k_j - kmean))."""
     rng = np.random.default_rng(5)
     nb, n, D = 3, 70, 64
     qm = (rng.integers(-64, 65, size=(nb, D)) * 2.0 ** -4).astype(np.float32)
@@ -146,3 +148,34 @@ def test_smoothing_helps_on_biased_queries():
     e_sq = np.mean([np.abs(sq[p] - ref[r]).mean() for r, p in enumerate(picks)])
     e_pb = np.mean([np.abs(pb[p] - ref[r]).mean() for r, p in enumerate(picks)])
     assert e_sq < 0.7 * e_pb, (e_sq, e_pb)
+
+
+def test_packed_single_sequence_equals_dense():
+    """A packed batch of one sequence is the dense problem with B = 1: the
+    smoothed codes, means and emulated rows agree bit for bit, and a second
+    sequence after it does not change the first one's rows."""
+    g = torch.Generator().manual_seed(31)
+    n, H, D = 300, 2, 64
+    qd_, kd_, vd_ = (torch.randn(1, H, n, D, generator=g).half() for _ in range(3))
+    qd_ = (qd_.float() + 3.0 * torch.randn(1, H, 1, D, generator=g)).half()
+    dense = heads.quantize(qd_, kd_, vd_, gran="block_sq")
+    pk = lambda t: t[0].transpose(0, 1).contiguous()              # [n, H, D]
+    extra = lambda t: torch.randn(200, H, D, generator=g).half()
+    qp = torch.cat([pk(qd_), extra(qd_)]); kp = torch.cat([pk(kd_), extra(kd_)])
+    vp = torch.cat([pk(vd_), extra(vd_)])
+    cu = torch.tensor([0, n, n + 200], dtype=torch.int32)
+    packed = heads.quantize(qp, kp, vp, cu, gran="block_sq")
+    nb = (n + BLK - 1) // BLK
+    for h in range(H):
+        np.testing.assert_array_equal(packed.q_mean[h, :nb], dense.q_mean[0, h])
+        np.testing.assert_array_equal(packed.q_codes[h, :nb * BLK], dense.q_codes[0, h])
+        np.testing.assert_array_equal(packed.q_delta[h, :nb], dense.q_delta[0, h])
+    rows = [0, 1, 127, 128, 299]
+    for causal in (False, True):
+        a = heads.emulate_rows(dense, vd_, None, [(0, h, i) for h in range(H) for i in rows], D,
+                               causal, "fp16", gran="block_sq", k=kd_)
+        b = heads.emulate_rows(packed, vp, cu, [(0, h, i) for h in range(H) for i in rows], D,
+                               causal, "fp16", gran="block_sq", k=kp)
+        for h in range(H):
+            for i in rows:
+                np.testing.assert_array_equal(a[(0, h, i)], b[(0, h, i)])
