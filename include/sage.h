@@ -82,8 +82,7 @@ typedef enum {
   SAGE_QK_PER_TOKEN = 1,         /* one delta per token                           */
   SAGE_QK_PER_BLOCK_SMOOTH_Q = 2 /* per block, each Q block minus its channel
                                     mean before quantisation; the mean's part of
-                                    the logit, mean . k~_j, added back per key
-                                    (dense problems only)                         */
+                                    the logit, mean . k~_j, added back per key    */
 } sage_qk_gran_t;
 
 /* Token count of one quantisation block and of one attention key/query tile. */
@@ -215,11 +214,19 @@ sage_status_t sage_attn_fwd_varlen_gqa(const void* q, const void* k, const void*
 /*
  * General variable-length forward pass: grouped-query heads (as
  * sage_attn_fwd_varlen_gqa) and the Q/K delta granularity qk_gran (as
- * sage_attn_fwd_ex; per token, every packed token has its own Q and K delta).
- *   ws : at least sage_workspace_bytes_varlen_ex(...).
+ * sage_attn_fwd_ex; per token, every packed token has its own Q and K delta;
+ * with Q smoothing every sequence's Q blocks take their own means and the
+ * mean term covers that sequence's keys).
+ *   ws : at least sage_workspace_bytes_varlen_ex(...), or for
+ *        SAGE_QK_PER_BLOCK_SMOOTH_Q sage_workspace_bytes_varlen_sq(...), whose
+ *        size depends on max_seqlen (the mean terms take at most
+ *        4 * H * ceil(max_seqlen/128) * (total_tokens + 128*batch) bytes).
+ * sage_workspace_bytes_varlen_ex returns 0 for SAGE_QK_PER_BLOCK_SMOOTH_Q.
  */
 size_t sage_workspace_bytes_varlen_ex(int total_tokens, int batch, int H, int Hkv, int D,
                                       int pv_mode, int qk_gran);
+size_t sage_workspace_bytes_varlen_sq(int total_tokens, int batch, int max_seqlen, int H,
+                                      int Hkv, int D, int pv_mode);
 sage_status_t sage_attn_fwd_varlen_ex(const void* q, const void* k, const void* v, void* out,
                                       int in_dt, int out_dt, const int32_t* cu_seqlens, int batch,
                                       int max_seqlen, int total_tokens, int H, int Hkv, int D,

@@ -264,8 +264,8 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     workspace: Optional[Workspace] = None, qk_gran: str = "block") -> torch.Tensor:
     """SageAttention forward over packed [T, H, D] tensors with int32 cu_seqlens.
     k, v may be [T, Hkv, D] with Hkv dividing H (grouped-query attention);
-    qk_gran: one Q/K delta per 128-token block ("block") or per token ("token");
-    Q smoothing ("block_sq") is for dense inputs only."""
+    qk_gran: one Q/K delta per 128-token block ("block"), per token ("token"),
+    or per block with Q smoothing ("block_sq")."""
     _need_cuda_contig(q, k, v, cu_seqlens)
     if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
         raise ValueError("q must be [T, H, D] and k, v one [T, Hkv, D] shape")
@@ -284,11 +284,12 @@ def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
     lib = _lib.load()
     scale = float(sm_scale) if sm_scale else 0.0
     gran = _gran(qk_gran)
-    if qk_gran == "block_sq":
-        raise ValueError("qk_gran 'block_sq' (Q smoothing) is implemented for dense inputs only")
     if gran:
-        ws = _workspace(q.device, int(lib.sage_workspace_bytes_varlen_ex(T, batch, H, Hkv, D, mode,
-                                                                         gran)), workspace)
+        if qk_gran == "block_sq":  # its workspace depends on max_seqlen
+            nb = int(lib.sage_workspace_bytes_varlen_sq(T, batch, int(max_seqlen), H, Hkv, D, mode))
+        else:
+            nb = int(lib.sage_workspace_bytes_varlen_ex(T, batch, H, Hkv, D, mode, gran))
+        ws = _workspace(q.device, nb, workspace)
         _check(lib.sage_attn_fwd_varlen_ex(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
             _dtype_code(out.dtype, True), _ptr(cu_seqlens), batch, int(max_seqlen), T, H, Hkv, D,

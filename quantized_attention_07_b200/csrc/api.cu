@@ -11,19 +11,20 @@ namespace sage {
 
 cudaError_t launch_varlen_prep(const int32_t* cu, int batch, int max_seqlen, int total_tokens,
                                int32_t* blk_off, int32_t* pair_off, uint32_t* status,
-                               cudaStream_t st);
+                               cudaStream_t st, long long* sq_off = nullptr);
 cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool fp8,
                          const void* q, const void* k, const void* v, int8_t* q_codes,
                          float* q_scale, int8_t* k_codes, float* k_scale, float* k_mean,
                          uint8_t* v_codes, float* v_scale, unsigned long long* k_sum,
                          uint32_t* v_amax, uint32_t* status, unsigned int* sync, int parts,
                          int per_token, cudaStream_t st);
-cudaError_t launch_quant_q_smooth(int BH, int N, int D, bool bf16, const void* q,
-                                  int8_t* q_codes, float* q_scale, float* q_mean,
+cudaError_t launch_quant_q_smooth(const SeqLayout& L, dim3 grid, int D, bool bf16,
+                                  const void* q, int8_t* q_codes, float* q_scale, float* q_mean,
                                   uint32_t* status, cudaStream_t st);
-cudaError_t launch_q_smooth_bias(int B, int H, int Hkv, int N, int D, bool bf16, int causal,
-                                 float kappa, const void* k, const float* k_mean,
-                                 const float* q_mean, float* bias, cudaStream_t st);
+cudaError_t launch_q_smooth_bias(const SeqLayout& L, dim3 grid, int H, int Hkv, int D, bool bf16,
+                                 int causal, float kappa, const void* k, const float* k_mean,
+                                 const float* q_mean, float* bias, long long head_stride,
+                                 const long long* sq_off, cudaStream_t st);
 cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
                             const int32_t* tiles, int n, int32_t* out, uint32_t* status,
                             cudaStream_t st);
@@ -64,7 +65,8 @@ struct Layout {
   size_t k_sum, v_amax, sync, sync_q, blk_off, pair_off;  // scratch
   size_t q_codes, k_codes, q_scale, k_scale, k_mean;   // quantised operands
   size_t v_codes, v_scale;
-  size_t q_mean, q_bias;                              // Q smoothing (dense)
+  size_t q_mean, q_bias, sq_off;                      // Q smoothing
+  long long bias_head_stride;                         // varlen Q smoothing: floats per head
   size_t scratch_end, total;
 };
 
@@ -108,9 +110,12 @@ long long pair_max(long long T, long long batch) { return (T + (2 * BLK - 1) * b
 
 // Varlen layout for H query heads and Hkv key/value heads (Hkv = H without
 // grouping): Q codes / deltas over H heads, everything of K and V over Hkv.
+// gran: a sage_qk_gran_t; Q smoothing needs max_seqlen, which bounds the
+// per-head size of the mean term: sum_s nb_s^2 <= ceil(max_seqlen/128) * TB.
 Layout varlen_layout(int T, int batch, int H, int D, bool fp8, int Hkv = 0,
-                     bool per_token = false) {
+                     int gran = SAGE_QK_PER_BLOCK, int max_seqlen = 0) {
   if (Hkv <= 0) Hkv = H;
+  const bool per_token = gran == SAGE_QK_PER_TOKEN, sq = gran == SAGE_QK_PER_BLOCK_SMOOTH_Q;
   const size_t SH = (size_t)batch * Hkv, TB = (size_t)tb_max(T, batch);
   const size_t NS = per_token ? TB * BLK : TB;  // deltas per head
   Layout L{};
@@ -120,6 +125,7 @@ Layout varlen_layout(int T, int batch, int H, int D, bool fp8, int Hkv = 0,
   L.sync = o; o += al(4);
   L.blk_off = o; o += al(((size_t)batch + 1) * 4);
   L.pair_off = o; o += al(((size_t)batch + 1) * 4);
+  if (sq) { L.sq_off = o; o += al(((size_t)batch + 1) * 8); }
   L.scratch_end = o;
   L.q_codes = o; o += al((size_t)H * TB * BLK * D);
   L.k_codes = o; o += al((size_t)Hkv * TB * BLK * D);
@@ -129,6 +135,12 @@ Layout varlen_layout(int T, int batch, int H, int D, bool fp8, int Hkv = 0,
   if (fp8) {
     L.v_codes = o; o += al((size_t)T * Hkv * D);
     L.v_scale = o; o += al(SH * D * 4);
+  }
+  if (sq) {
+    const size_t MB = ((size_t)max_seqlen + BLK - 1) / BLK;
+    L.bias_head_stride = (long long)(MB * TB * BLK);
+    L.q_mean = o; o += al((size_t)H * TB * D * 4);
+    L.q_bias = o; o += al((size_t)H * MB * TB * BLK * 4);
   }
   L.total = o;
   return L;
@@ -225,12 +237,13 @@ sage_status_t quantize_dense_sq(const void* q, const void* k, const void* v, int
                                q_scale, k_codes, k_scale, k_mean, v_codes, v_scale,
                                at<unsigned long long>(ws, L.k_sum), at<uint32_t>(ws, L.v_amax),
                                at<uint32_t>(ws, 0), at<unsigned int>(ws, L.sync), QUANT_KV, 0, st);
+  S.H = H;
   if (e == cudaSuccess)
-    e = launch_quant_q_smooth(B * H, N, D, bf16, q, q_codes, q_scale, q_mean, at<uint32_t>(ws, 0),
-                              st);
+    e = launch_quant_q_smooth(S, dim3(NB, (unsigned)(B * H)), D, bf16, q, q_codes, q_scale,
+                              q_mean, at<uint32_t>(ws, 0), st);
   if (e == cudaSuccess)
-    e = launch_q_smooth_bias(B, H, Hkv, N, D, bf16, causal ? 1 : 0, kappa_of(sm_scale, D), k,
-                             k_mean, q_mean, q_bias, st);
+    e = launch_q_smooth_bias(S, dim3(NB, (unsigned)(B * H)), H, Hkv, D, bf16, causal ? 1 : 0,
+                             kappa_of(sm_scale, D), k, k_mean, q_mean, q_bias, 0, nullptr, st);
   if (e == cudaErrorNotSupported) return SAGE_ERR_UNSUPPORTED;
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
@@ -506,13 +519,16 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
                                    int D, int pv_mode, int8_t* q_codes, float* q_scale,
                                    int8_t* k_codes, float* k_scale, float* k_mean,
                                    uint8_t* v_codes, float* v_scale, void* ws, const Layout& L,
-                                   cudaStream_t st, int Hkv = 0, int per_token = 0) {
+                                   cudaStream_t st, int Hkv = 0, int per_token = 0,
+                                   int causal = 0, float sm_scale = 0.0f) {
   if (Hkv <= 0) Hkv = H;
-  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  const bool fp8 = pv_mode == SAGE_PV_FP8, bf16 = in_dt == SAGE_BF16;
+  const bool sq = per_token == 2;  // Q smoothing
   sage_status_t r = clear_scratch(ws, L, fp8, st);
   if (r != SAGE_OK) return r;
   cudaError_t e = launch_varlen_prep(cu, batch, max_seqlen, T, at<int32_t>(ws, L.blk_off),
-                                     at<int32_t>(ws, L.pair_off), at<uint32_t>(ws, 0), st);
+                                     at<int32_t>(ws, L.pair_off), at<uint32_t>(ws, 0), st,
+                                     sq ? at<long long>(ws, L.sq_off) : nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "varlen preparation launch");
   const long long TB = tb_max(T, batch);
   if (TB == 0) return SAGE_OK;
@@ -523,6 +539,23 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
   S.blk_off = at<int32_t>(ws, L.blk_off);
   S.batch = batch;
   S.TBmax = (int)TB;
+  if (sq) {
+    // K (, V) per block over the key/value heads; the smoothed Q blocks and
+    // the per-key mean term over the query heads
+    e = launch_quant(S, dim3((unsigned)TB, Hkv), D, bf16, fp8, q, k, v, q_codes, q_scale, k_codes,
+                     k_scale, k_mean, v_codes, v_scale, at<unsigned long long>(ws, L.k_sum),
+                     at<uint32_t>(ws, L.v_amax), at<uint32_t>(ws, 0), nullptr, QUANT_KV, 0, st);
+    S.H = H;
+    if (e == cudaSuccess)
+      e = launch_quant_q_smooth(S, dim3((unsigned)TB, H), D, bf16, q, q_codes, q_scale,
+                                at<float>(ws, L.q_mean), at<uint32_t>(ws, 0), st);
+    if (e == cudaSuccess)
+      e = launch_q_smooth_bias(S, dim3((unsigned)TB, H), H, Hkv, D, bf16, causal ? 1 : 0,
+                               kappa_of(sm_scale, D), k, k_mean, at<float>(ws, L.q_mean),
+                               at<float>(ws, L.q_bias), L.bias_head_stride,
+                               at<long long>(ws, L.sq_off), st);
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
+  }
   // grouped-query: K (, V) over the Hkv key/value heads, then Q over the H
   // query heads; otherwise both in one pair of launches
   const bool grouped = Hkv != H;
@@ -568,15 +601,16 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
                                        int Hkv, int D, int causal, float sm_scale, int pv_mode,
                                        int qk_gran, void* ws, size_t ws_bytes, void* stream) {
   if (!varlen_args_ok(total_tokens, batch, max_seqlen, H, D, pv_mode) || !gqa_heads_ok(H, Hkv) ||
-      !gran_varlen_ok(qk_gran) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
+      !gran_ok(qk_gran) || !in_dtype_ok(in_dt) || !out_dtype_ok(out_dt) ||
       !std::isfinite(sm_scale))
     return SAGE_ERR_INVALID_ARG;
-  const int tok = qk_gran == SAGE_QK_PER_TOKEN ? 1 : 0;
+  // 0 per block, 1 per token, 2 per block with Q smoothing
+  const int tok = qk_gran == SAGE_QK_PER_TOKEN ? 1 : qk_gran == SAGE_QK_PER_BLOCK_SMOOTH_Q ? 2 : 0;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws) ||
       !cu_seqlens)
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8;
-  const Layout L = varlen_layout(total_tokens, batch, H, D, fp8, Hkv, tok != 0);
+  const Layout L = varlen_layout(total_tokens, batch, H, D, fp8, Hkv, qk_gran, max_seqlen);
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   if (total_tokens == 0) return SAGE_OK;
   cudaStream_t st = as_stream(stream);
@@ -584,7 +618,7 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
       q, k, v, in_dt, cu_seqlens, batch, max_seqlen, total_tokens, H, D, pv_mode,
       at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale), at<int8_t>(ws, L.k_codes),
       at<float>(ws, L.k_scale), at<float>(ws, L.k_mean), fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
-      fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L, st, Hkv, tok);
+      fp8 ? at<float>(ws, L.v_scale) : nullptr, ws, L, st, Hkv, tok, causal, sm_scale);
   if (r != SAGE_OK) return r;
   const long long TB = tb_max(total_tokens, batch), PM = pair_max(total_tokens, batch);
   if (PM == 0) return SAGE_OK;
@@ -607,6 +641,11 @@ static sage_status_t attn_fwd_varlen_g(const void* q, const void* k, const void*
   A.p.TBmax = (int)TB;
   A.p.status = at<uint32_t>(ws, 0);
   A.p.sched = at<unsigned int>(ws, kSchedOff);
+  if (tok == 2) {
+    A.p.q_bias = at<float>(ws, L.q_bias);
+    A.p.sq_off = at<long long>(ws, L.sq_off);
+    A.p.bias_head_stride = L.bias_head_stride;
+  }
   A.D = D;
   A.pv8 = fp8;
   A.bf16v = in_dt == SAGE_BF16;
@@ -638,8 +677,15 @@ size_t sage_workspace_bytes_varlen_ex(int total_tokens, int batch, int H, int Hk
   if (!varlen_args_ok(total_tokens, batch, 0, H, D, pv_mode) || !gqa_heads_ok(H, Hkv) ||
       !gran_varlen_ok(qk_gran))
     return 0;
+  return varlen_layout(total_tokens, batch, H, D, pv_mode == SAGE_PV_FP8, Hkv, qk_gran).total;
+}
+
+size_t sage_workspace_bytes_varlen_sq(int total_tokens, int batch, int max_seqlen, int H,
+                                      int Hkv, int D, int pv_mode) {
+  if (!varlen_args_ok(total_tokens, batch, max_seqlen, H, D, pv_mode) || !gqa_heads_ok(H, Hkv))
+    return 0;
   return varlen_layout(total_tokens, batch, H, D, pv_mode == SAGE_PV_FP8, Hkv,
-                       qk_gran == SAGE_QK_PER_TOKEN).total;
+                       SAGE_QK_PER_BLOCK_SMOOTH_Q, max_seqlen).total;
 }
 
 sage_status_t sage_attn_fwd_varlen_ex(const void* q, const void* k, const void* v, void* out,

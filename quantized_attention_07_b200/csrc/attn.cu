@@ -146,6 +146,8 @@ struct Work {
   long long vs_idx;      // v_scale row index (FP8)
   int nsub0, nsub1;      // 64-key sub-tiles for query tile 0 / 1 (0 = tile absent)
   int nkv;               // 128-key stages to stream
+  long long bias_row0;   // Q smoothing: float index of query tile 0's mean-term row
+  long long bias_ld;     // floats between the rows of consecutive query blocks
 };
 
 // Work item idx of the launch (0 <= idx < p.items).  Dense: idx -> (head,
@@ -180,6 +182,8 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p, int idx) {
     w.out_row0 = (long long)bh * p.N;
     w.out_stride = 1;
     w.vs_idx = bkv;
+    w.bias_ld = (long long)p.NB * BLK;
+    w.bias_row0 = ((long long)bh * p.NB + 2 * pair) * w.bias_ld;
   } else {
     const int h = idx / p.PM;
     const int item = idx - h * p.PM;
@@ -204,6 +208,11 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p, int idx) {
     w.out_row0 = (long long)tok0 * p.H + h;
     w.out_stride = p.H;
     w.vs_idx = (long long)s * p.Hkv + hk;
+    if (p.per_token == 2) {  // the sequence's own [nb_s][nb_s*128] block of the term
+      w.bias_ld = (long long)((n + BLK - 1) / BLK) * BLK;
+      w.bias_row0 = (long long)h * p.bias_head_stride + __ldg(p.sq_off + s) * BLK +
+                    2LL * pair * w.bias_ld;
+    }
   }
   w.valid = 1;
   w.n = n;
@@ -310,8 +319,7 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
           ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + nt_q * BLK * 4);
           for (int tq = 0; tq < nt_q; ++tq)
             ptx::bulk_load_plain(sKs + (s * 2 + tq) * BLK,
-                                 p.q_bias + ((long long)w.code_z * p.NB + 2 * w.pair + tq) *
-                                                (long long)p.NB * BLK + (long long)j * BLK,
+                                 p.q_bias + w.bias_row0 + tq * w.bias_ld + (long long)j * BLK,
                                  BLK * 4, &B->k_full[s]);
         } else {
           ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);

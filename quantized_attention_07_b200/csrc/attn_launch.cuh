@@ -12,8 +12,11 @@ struct AttnParams {
   int NPAIR;             // dense: query tile pairs per head = ceil(N/256)
   int causal;
   int per_token;         // 1: one delta per token ([BH][NP] / [B*Hkv][NP]), not per block;
-                         // 2 (dense): per block, Q smoothed (q_bias holds the mean term)
-  const float* q_bias;   // per_token 2: [BH][NB][NB*128] fp32, kappa applied
+                         // 2: per block, Q smoothed (q_bias holds the mean term)
+  const float* q_bias;   // per_token 2: dense [BH][NB][NB*128] fp32, kappa applied;
+                         // varlen: sequence s, head h at h*bias_head_stride + sq_off[s]*128
+  const long long* sq_off;        // varlen per_token 2: [batch+1] prefix of ceil(n_s/128)^2
+  long long bias_head_stride;     // varlen per_token 2: floats per query head
   float kappa;           // fp32(sm_scale * log2 e)
   const float* q_scale;  // dense [BH][NB]; varlen [H][TBmax]
   const float* k_scale;

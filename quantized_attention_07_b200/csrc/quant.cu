@@ -446,18 +446,18 @@ __global__ void __launch_bounds__(THREADS) quant_pass2_kernel(
 // One CTA per (query block, head): the exact block mean (the K mean's
 // fixed-point sum, over this block's rows), then per-block codes of
 // fp32(q - qmean_I) with one delta, as the K blocks are coded.
+// Dense: grid (blocks, B*H), q_mean [B*H][NB][D]; varlen: grid (TBmax, H),
+// q_mean [H][TBmax][D] (indexed like the deltas).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(THREADS) quant_q_smooth_kernel(
-    int N, const void* __restrict__ q, int8_t* __restrict__ q_codes,
+    SeqLayout L, const void* __restrict__ q, int8_t* __restrict__ q_codes,
     float* __restrict__ q_scale, float* __restrict__ q_mean, uint32_t* __restrict__ status) {
   using T = Tile<D>;
   __shared__ float red[THREADS / 32];
   __shared__ long long red64[THREADS / 32][D];
   __shared__ float s_mean[D];
-  SeqLayout L{};
-  L.N = N;
   BlockPos P;
-  dense_block_pos(L, blockIdx.y, blockIdx.x, P);
+  if (!block_pos(L, P)) return;
   const int c = threadIdx.x % T::CPR, r0 = threadIdx.x / T::CPR;
   const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
 
@@ -516,9 +516,58 @@ __global__ void __launch_bounds__(THREADS) quant_q_smooth_kernel(
   if (threadIdx.x == 0) q_scale[P.scale_idx] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
 }
 
-// The per-key term: bias[bh][I][j] = fp32(acc * kappa), acc the fp32 fused
+// Where the mean term of one (key tile, query head) CTA lives.
+struct BiasPos {
+  int n;                 // sequence length
+  int nb;                // its query / key blocks
+  int J;                 // key tile within the sequence
+  const uint16_t* k0;    // key token 0 of the sequence, this key/value head
+  long long k_stride;    // elements between consecutive tokens of k
+  const float* kmean;    // [D] of the key/value head
+  const float* qm;       // [nb][D] block means of the query head
+  float* out;            // [nb][nb*128] term of the (sequence, query head)
+};
+
+// Dense: grid (NB, B*H); varlen: grid (TBmax, H) over the global key blocks.
+__device__ __forceinline__ bool bias_pos(const SeqLayout& L, int Hq, int Hkv, int D,
+                                         const void* k, const float* k_mean, const float* q_mean,
+                                         float* bias, long long head_stride,
+                                         const long long* sq_off, BiasPos& P) {
+  if (!L.varlen) {
+    const int NB = (L.N + BLK - 1) / BLK;
+    const int bh = blockIdx.y, b = bh / Hq, h = bh - b * Hq;
+    const int bkv = b * Hkv + h / (Hq / Hkv);
+    P.n = L.N;
+    P.nb = NB;
+    P.J = blockIdx.x;
+    P.k0 = static_cast<const uint16_t*>(k) + (long long)bkv * L.N * D;
+    P.k_stride = D;
+    P.kmean = k_mean + (long long)bkv * D;
+    P.qm = q_mean + (long long)bh * NB * D;
+    P.out = bias + (long long)bh * NB * NB * BLK;
+    return true;
+  }
+  const int gb = blockIdx.x, h = blockIdx.y;
+  const int total = __ldg(L.blk_off + L.batch);
+  if (gb >= total) return false;
+  const int s = find_segment(L.blk_off, L.batch + 1, gb);
+  const int b0 = __ldg(L.blk_off + s);
+  const int t0 = __ldg(L.cu + s);
+  const int hk = h / (Hq / Hkv);
+  P.n = __ldg(L.cu + s + 1) - t0;
+  P.nb = (P.n + BLK - 1) / BLK;
+  P.J = gb - b0;
+  P.k0 = static_cast<const uint16_t*>(k) + ((long long)t0 * Hkv + hk) * D;
+  P.k_stride = (long long)Hkv * D;
+  P.kmean = k_mean + ((long long)s * Hkv + hk) * D;
+  P.qm = q_mean + ((long long)h * L.TBmax + b0) * D;
+  P.out = bias + (long long)h * head_stride + __ldg(sq_off + s) * BLK;
+  return true;
+}
+
+// The per-key term: bias[I][j] = fp32(acc * kappa), acc the fp32 fused
 // multiply-adds of qmean_I[d] and k~_j[d] = fp32(k_j[d] - kmean[d]) in
-// channel order, for the key/value head that query head bh reads.  The fixed
+// channel order, for the key/value head that the query head reads.  The fixed
 // order makes the value (and every FP8 code of P that depends on it) the
 // oracle's, bit for bit.
 // One CTA per (128-key tile J, query head), one thread per key: the thread
@@ -526,24 +575,21 @@ __global__ void __launch_bounds__(THREADS) quant_q_smooth_kernel(
 // (G independent accumulators, paired into packed FMAs), whose means the CTA
 // first stages in shared memory channel-major (every thread then reads the
 // same address: a broadcast).  With a causal mask, blocks I < J never see the
-// tile and are skipped.  Keys past N get 0.
+// tile and are skipped.  Keys past n get 0.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
-    int N, int H, int Hkv, int causal, float kappa, const void* __restrict__ k,
+    SeqLayout L, int H, int Hkv, int causal, float kappa, const void* __restrict__ k,
     const float* __restrict__ k_mean, const float* __restrict__ q_mean,
-    float* __restrict__ bias) {
+    float* __restrict__ bias, long long head_stride, const long long* __restrict__ sq_off) {
   constexpr int G = 8;                 // query blocks per pass
   __shared__ __align__(16) float s_qm[D][G];  // means of G blocks, channel-major
-  const int NB = (N + BLK - 1) / BLK;
-  const int J = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / H, h = bh - b * H;
-  const int bkv = b * Hkv + h / (H / Hkv);
-  const int j = J * BLK + threadIdx.x;
+  BiasPos P;
+  if (!bias_pos(L, H, Hkv, D, k, k_mean, q_mean, bias, head_stride, sq_off, P)) return;
+  const int jl = P.J * BLK + threadIdx.x;  // key within the sequence
   float kt[D];
-  if (j < N) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(k) +
-                                                      ((long long)bkv * N + j) * D);
-    const float2* km = reinterpret_cast<const float2*>(k_mean + (long long)bkv * D);
+  if (jl < P.n) {
+    const uint4* src = reinterpret_cast<const uint4*>(P.k0 + (long long)jl * P.k_stride);
+    const float2* km = reinterpret_cast<const float2*>(P.kmean);
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
       const uint4 u = __ldg(src + c);
@@ -560,14 +606,13 @@ __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
 #pragma unroll
     for (int c = 0; c < D; ++c) kt[c] = 0.0f;
   }
-  const long long NP = (long long)NB * BLK;
-  const float* qm = q_mean + (long long)bh * NB * D;
-  float* out = bias + (long long)bh * NB * NP + j;
-  for (int I0 = causal ? J : 0; I0 < NB; I0 += G) {
+  const long long NP = (long long)P.nb * BLK;
+  float* out = P.out + jl;
+  for (int I0 = causal ? P.J : 0; I0 < P.nb; I0 += G) {
     __syncthreads();  // the previous group's means are no longer read
     for (int x = threadIdx.x; x < G * D; x += 128) {
       const int g = x / D, d = x - g * D;
-      s_qm[d][g] = I0 + g < NB ? __ldg(qm + (long long)(I0 + g) * D + d) : 0.0f;
+      s_qm[d][g] = I0 + g < P.nb ? __ldg(P.qm + (long long)(I0 + g) * D + d) : 0.0f;
     }
     __syncthreads();
     float2 acc[G / 2];
@@ -586,8 +631,8 @@ __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
     }
 #pragma unroll
     for (int g2 = 0; g2 < G / 2; ++g2) {
-      if (I0 + 2 * g2 < NB) out[(long long)(I0 + 2 * g2) * NP] = __fmul_rn(acc[g2].x, kappa);
-      if (I0 + 2 * g2 + 1 < NB)
+      if (I0 + 2 * g2 < P.nb) out[(long long)(I0 + 2 * g2) * NP] = __fmul_rn(acc[g2].x, kappa);
+      if (I0 + 2 * g2 + 1 < P.nb)
         out[(long long)(I0 + 2 * g2 + 1) * NP] = __fmul_rn(acc[g2].y, kappa);
     }
   }
@@ -1149,25 +1194,35 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
 // One thread: validates cu_seqlens and writes the block and pair prefix sums.
 // On any inconsistency all prefixes are written as 0, so every later kernel of
 // the call finds no work, and the status word records SAGE_ERR_BAD_SEQLENS.
+// sq_off (Q smoothing, may be null): prefix sums of ceil(n_s/128)^2, the
+// per-sequence offsets of the mean term in units of 128 floats.
 __global__ void varlen_prep_kernel(const int32_t* __restrict__ cu, int batch, int max_seqlen,
                                    int total_tokens, int32_t* blk_off, int32_t* pair_off,
-                                   uint32_t* status) {
+                                   long long* sq_off, uint32_t* status) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   bool ok = __ldg(cu) == 0 && __ldg(cu + batch) == total_tokens;
   int b = 0, p = 0;
+  long long q2 = 0;
   for (int s = 0; s < batch && ok; ++s) {
     const int n = __ldg(cu + s + 1) - __ldg(cu + s);
     if (n < 0 || n > max_seqlen) { ok = false; break; }
     blk_off[s] = b;
     pair_off[s] = p;
-    b += (n + BLK - 1) / BLK;
+    if (sq_off) sq_off[s] = q2;
+    const int nb = (n + BLK - 1) / BLK;
+    b += nb;
     p += (n + 2 * BLK - 1) / (2 * BLK);
+    q2 += (long long)nb * nb;
   }
   if (ok) {
     blk_off[batch] = b;
     pair_off[batch] = p;
+    if (sq_off) sq_off[batch] = q2;
   } else {
-    for (int s = 0; s <= batch; ++s) blk_off[s] = pair_off[s] = 0;
+    for (int s = 0; s <= batch; ++s) {
+      blk_off[s] = pair_off[s] = 0;
+      if (sq_off) sq_off[s] = 0;
+    }
     set_status(status, ST_BAD_SEQLENS);
   }
 }
@@ -1178,9 +1233,9 @@ __global__ void varlen_prep_kernel(const int32_t* __restrict__ cu, int batch, in
 
 cudaError_t launch_varlen_prep(const int32_t* cu, int batch, int max_seqlen, int total_tokens,
                                int32_t* blk_off, int32_t* pair_off, uint32_t* status,
-                               cudaStream_t st) {
+                               cudaStream_t st, long long* sq_off) {
   varlen_prep_kernel<<<1, 32, 0, st>>>(cu, batch, max_seqlen, total_tokens, blk_off, pair_off,
-                                       status);
+                                       sq_off, status);
   return cudaGetLastError();
 }
 
@@ -1260,31 +1315,33 @@ cudaError_t launch_quant(const SeqLayout& L, dim3 grid, int D, bool bf16, bool f
 #undef SAGE_Q
 }
 
-// Q smoothing, dense [B*H, N, D] query heads: block means, codes and deltas
-// of the smoothed Q (grid: blocks x heads).
-cudaError_t launch_quant_q_smooth(int BH, int N, int D, bool bf16, const void* q,
-                                  int8_t* q_codes, float* q_scale, float* q_mean,
+// Q smoothing: block means, codes and deltas of the smoothed Q over the
+// layout L (dense: grid (blocks, B*H); varlen: grid (TBmax, H)).
+cudaError_t launch_quant_q_smooth(const SeqLayout& L, dim3 grid, int D, bool bf16,
+                                  const void* q, int8_t* q_codes, float* q_scale, float* q_mean,
                                   uint32_t* status, cudaStream_t st) {
-  const dim3 grid((N + BLK - 1) / BLK, BH);
   if (D == 64) {
-    if (bf16) quant_q_smooth_kernel<64, true><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
-    else quant_q_smooth_kernel<64, false><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
+    if (bf16) quant_q_smooth_kernel<64, true><<<grid, THREADS, 0, st>>>(L, q, q_codes, q_scale, q_mean, status);
+    else quant_q_smooth_kernel<64, false><<<grid, THREADS, 0, st>>>(L, q, q_codes, q_scale, q_mean, status);
   } else {
-    if (bf16) quant_q_smooth_kernel<128, true><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
-    else quant_q_smooth_kernel<128, false><<<grid, THREADS, 0, st>>>(N, q, q_codes, q_scale, q_mean, status);
+    if (bf16) quant_q_smooth_kernel<128, true><<<grid, THREADS, 0, st>>>(L, q, q_codes, q_scale, q_mean, status);
+    else quant_q_smooth_kernel<128, false><<<grid, THREADS, 0, st>>>(L, q, q_codes, q_scale, q_mean, status);
   }
   return cudaGetLastError();
 }
 
-// The per-key term of Q smoothing into bias [B*H][NB][NB*128] (fp32, kappa
-// applied); k is [B*Hkv, N, D], k_mean [B*Hkv, D], q_mean [B*H, NB, D].
-cudaError_t launch_q_smooth_bias(int B, int H, int Hkv, int N, int D, bool bf16, int causal,
-                                 float kappa, const void* k, const float* k_mean,
-                                 const float* q_mean, float* bias, cudaStream_t st) {
-  const dim3 grid((N + BLK - 1) / BLK, B * H);
-#define SAGE_B(DD, BB)                                                                     \
-  q_smooth_bias_kernel<DD, BB><<<grid, 128, 0, st>>>(N, H, Hkv, causal, kappa, k, k_mean, \
-                                                     q_mean, bias)
+// The per-key term of Q smoothing (fp32, kappa applied).  Dense: grid (NB,
+// B*H), k [B*Hkv, N, D], k_mean [B*Hkv, D], q_mean [B*H, NB, D], bias
+// [B*H][NB][NB*128].  Varlen: grid (TBmax, H), k [T, Hkv, D], k_mean
+// [batch, Hkv, D], q_mean [H, TBmax, D], bias of sequence s and head h at
+// h*head_stride + sq_off[s]*128, [nb_s][nb_s*128].
+cudaError_t launch_q_smooth_bias(const SeqLayout& L, dim3 grid, int H, int Hkv, int D, bool bf16,
+                                 int causal, float kappa, const void* k, const float* k_mean,
+                                 const float* q_mean, float* bias, long long head_stride,
+                                 const long long* sq_off, cudaStream_t st) {
+#define SAGE_B(DD, BB)                                                                        \
+  q_smooth_bias_kernel<DD, BB><<<grid, 128, 0, st>>>(L, H, Hkv, causal, kappa, k, k_mean,    \
+                                                     q_mean, bias, head_stride, sq_off)
   if (D == 64) {
     if (bf16) SAGE_B(64, true); else SAGE_B(64, false);
   } else {

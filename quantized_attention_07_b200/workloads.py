@@ -149,7 +149,8 @@ def make_dense(B: int, H: int, N: int, D: int, dtype: str = "fp16", bias_sigma: 
 
 
 def make_varlen(seqlens: list[int], H: int, D: int, dtype: str = "bf16", bias_sigma: float = 3.0,
-                seed: int = 0) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+                seed: int = 0, q_bias_sigma: float = 0.0
+                ) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
     """Packed [T,H,D] q, k, v plus int32 cu_seqlens for the given lengths."""
     g = torch.Generator().manual_seed(seed)
     T = int(sum(seqlens))
@@ -162,6 +163,9 @@ def make_varlen(seqlens: list[int], H: int, D: int, dtype: str = "bf16", bias_si
     for s, n in enumerate(seqlens):
         b = torch.randn((1, H, D), generator=g) * bias_sigma
         k[cu[s]:cu[s + 1]] += b
+    if q_bias_sigma > 0.0:  # drawn last: the other draws do not depend on it
+        for s, n in enumerate(seqlens):
+            q[cu[s]:cu[s + 1]] += torch.randn((1, H, D), generator=g) * q_bias_sigma
     t = DTYPES[dtype]
     return q.to(t), k.to(t), v.to(t), torch.tensor(cu, dtype=torch.int32)
 

@@ -142,8 +142,19 @@ def test_smoothing_helps_with_a_query_offset():
     assert cos["block_sq"] > cos["block"] and cos["block_sq"] > 0.99
 
 
-def test_varlen_rejects_smoothing():
-    q = torch.zeros((256, 2, 64), dtype=torch.float16, device="cuda")
-    cu = torch.tensor([0, 256], dtype=torch.int32, device="cuda")
-    with pytest.raises(ValueError):
-        sage.attn_fwd_varlen(q, q, q, cu, 256, qk_gran="block_sq")
+VARLEN = [
+    # (seqlens, H, Hkv, D, dtype, causal, pv_mode)
+    ([300, 1, 130, 700], 2, 2, 64, "fp16", True, "fp16"),
+    ([520, 257], 4, 2, 128, "bf16", False, "fp8"),
+    ([0, 200, 0, 129], 2, 1, 128, "fp16", True, "fp8"),
+]
+
+
+@pytest.mark.parametrize("seqlens,H,Hkv,D,dtype,causal,pv_mode", VARLEN)
+def test_smoothed_varlen_against_oracle(seqlens, H, Hkv, D, dtype, causal, pv_mode):
+    """Packed batches: every sequence's Q blocks take their own means and the
+    mean term covers that sequence's keys (empty sequences included)."""
+    q, k, v, cu = W.make_varlen(seqlens, H, D, dtype, seed=sum(seqlens) + D, q_bias_sigma=3.0)
+    k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
+    picks = [(si, h, i) for si, n in enumerate(seqlens) for h in range(H) for i in range(0, n, 3)]
+    U.check_against_oracle(q, k, v, cu, causal, pv_mode, picks, qk_gran="block_sq")
