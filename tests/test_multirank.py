@@ -55,3 +55,19 @@ def test_two_rank_timing_and_independent_problems():
 def test_single_process_defaults():
     assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
     assert bench.rank_workload(W.WORKLOADS["long_32k"], 0) is W.WORKLOADS["long_32k"]
+
+
+def test_stage1_algorithmic_bytes():
+    """Stage 1's roofline numerator: Q and K read at 2 B and coded at 1 B per
+    element (6 B per token-channel for the pair), FP8 adds V's 3 B, Q
+    smoothing the fp32 per-key mean term; packed batches report none."""
+    wl = W.WORKLOADS["long_32k"]
+    assert bench.quant_algorithmic_bytes(wl) == 6 * 32 * 32768 * 128
+    fp8 = W.WORKLOADS["dit_8k_fp8"]
+    el = 24 * 8192 * 64
+    assert bench.quant_algorithmic_bytes(fp8) == 9 * el
+    sq = W.WORKLOADS["dit_8k_fp8_sq"]
+    assert bench.quant_algorithmic_bytes(sq) == 9 * el + 4 * 24 * 64 * 8192
+    gqa = W.WORKLOADS["llm_gqa_8k"]
+    assert bench.quant_algorithmic_bytes(gqa) == 3 * 8192 * 128 * (32 + 8)
+    assert bench.quant_algorithmic_bytes(W.WORKLOADS["varlen_8seq"]) == 0
