@@ -84,11 +84,38 @@ def tensor_peak(pk: dict, pv_mode: str, sustained: bool = False) -> float:
     return 1.0 / (0.5 / i8 + 0.5 / b16)  # half the ops INT8, half 16-bit
 
 
+def _code_only(src: str) -> str:
+    """C++ source without comments and blank-line / trailing-space differences,
+    so that an edit of the comments does not count as a new kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif src[i] in "\"'":  # string or character literal, copied as is
+            q, j = src[i], i + 1
+            while j < n and src[j] != q:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_hash() -> str:
+    """Hash of the attention kernel's code (comments excluded): the key under
+    which ncu traffic counters are recorded."""
     h = hashlib.sha256()
     for name in ("attn.cu", "ptx.cuh", "common.cuh", "attn_launch.cuh"):
-        with open(os.path.join(ROOT, "quantized_attention_07_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "quantized_attention_07_b200", "csrc", name),
+                  encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

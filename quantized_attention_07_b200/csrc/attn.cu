@@ -1,8 +1,9 @@
 // Fused SageAttention forward kernel for sm_100a.
 //
-// One CTA handles two 128-row query tiles of one (sequence, head) and streams
-// that head's keys and values through shared memory in 128-key stages; the
-// online softmax works on 64-key sub-tiles.
+// A persistent kernel, one CTA per SM.  A work item is a pair of 128-row
+// query tiles of one (sequence, head); the CTA takes items from a counter in
+// the workspace and streams each item's keys and values through shared
+// memory in 128-key stages; the online softmax works on 64-key sub-tiles.
 //
 //   control warpgroup (warp 0 of it: TMA producer; warps 1 and 2: MMA
 //                issue for query tile 0 / 1, one elected lane each; warp 1
@@ -33,6 +34,10 @@
 // FlashAttention到SageAttention的工程实践", section 3.1), P.V in 16 bits
 // ("SageAttention" bullet 3) or FP8 with two-level accumulation
 // ("SageAttention v1/v2/v2++/v3 overview", SageAttention 2 bullets 1 and 3).
+// The template parameter GR picks the Q/K delta granularity (same overview,
+// SageAttention v1 item (1)): 0 per block, 1 per token, 2 per block with Q
+// smoothing (SageAttention 2 bullet 2), whose per-key mean term joins the
+// scaled score before the row maximum.
 //
 // Every mbarrier wait is bounded.  On a timeout the waiting role records
 // ST_TIMEOUT, raises a CTA-wide abort flag that the other roles' waits also
