@@ -310,6 +310,9 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
 /* E: the quantised method, step by step.                                    */
 /* ------------------------------------------------------------------------ */
 
+/* fp32(log2 448): the FP8 P scale, applied in the exponent */
+#define LOG2_448F 8.807354927062988f
+
 /*
  * Emulated output rows of one (sequence, head).
  *
@@ -348,15 +351,19 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *     P_ij  = p_ij rounded to V's 16-bit format
  *     Part  = fp32(sum_j P_ij v_jd)                   (products summed in fp64)
  *     O_d   = fp32(fp32(alpha * O_d) + Part_d)
- *   pv_mode 1 (FP8 P.V, two-level accumulation):
- *     P^_ij = e4m3(fp32(p_ij * 448))                  static P scale 1/448
+ *   pv_mode 1 (FP8 P.V, two-level accumulation): p is formed scaled by the
+ *   static P scale 448 in the exponent, arg_ij = fmaf(S_ij, c_IJ,
+ *   fp32(L - m_new)) with L = fp32(log2 448), so p_ij = 448 2^(t - m) and
+ *   l sums these scaled p:
+ *     P^_ij = e4m3(p_ij)
  *     Part  = fp32(sum_j dec(P^_ij) dec(v^_jd))       one key block's partial
  *     O_d   = fmaf(alpha, O_d, Part_d)                flushed into the fp32
  *                                                     accumulator every block
  *   m = m_new
  *
  * Finally out_d = fp32(O_d / l)   (pv_mode 0), or
- *           out_d = fp32(fp32(O_d * fp32(deltaV_d / 448)) / l)   (pv_mode 1).
+ *           out_d = fp32(fp32(O_d * deltaV_d) / l)   (pv_mode 1: the 448 of
+ *           P and the 448 of l cancel).
  *
  * Masked keys (j >= n, or j > i when causal) take no part in the maximum and
  * contribute p = 0.  (A tile is entered only if it holds at least one
@@ -448,10 +455,12 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
             }
             float m_new = mblk > m + tau ? mblk : m;
             float alpha = (float)exp2((double)(m - m_new));
+            /* FP8 P.V: p is formed already scaled by 448, as 2^(arg + log2 448) */
+            const float sub = pv_mode == 0 ? -m_new : LOG2_448F - m_new;
             double psum = 0.0;
             for (int jj = 0; jj < nj; ++jj) {
-                float arg = bk ? y[jj] - m_new
-                            : per_token ? fmaf(y[jj], c, -m_new) : fmaf((float)S[jj], c, -m_new);
+                float arg = bk ? y[jj] + sub
+                            : per_token ? fmaf(y[jj], c, sub) : fmaf((float)S[jj], c, sub);
                 p[jj] = (float)exp2((double)arg);
                 psum += (double)p[jj];
             }
@@ -466,7 +475,7 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
                 for (int d = 0; d < D; ++d) O[d] = alpha * O[d] + (float)part[d];
             } else {
                 for (int jj = 0; jj < nj; ++jj) {
-                    double P = oracle_e4m3_decode(oracle_e4m3_encode(p[jj] * 448.0f));
+                    double P = oracle_e4m3_decode(oracle_e4m3_encode(p[jj]));
                     const uint8_t* vr = vc + (j0 + jj) * D;
                     for (int d = 0; d < D; ++d) part[d] += P * oracle_e4m3_decode(vr[d]);
                 }
@@ -477,7 +486,7 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
         float* o = out + r * D;
         for (int d = 0; d < D; ++d) {
             if (pv_mode == 0) o[d] = O[d] / l;
-            else o[d] = (O[d] * (vdelta[d] / 448.0f)) / l;
+            else o[d] = (O[d] * vdelta[d]) / l;  /* the 448 of P and of l cancel */
         }
         free(O); free(part); free(S); free(p); free(y);
     }

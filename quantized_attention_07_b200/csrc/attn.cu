@@ -54,6 +54,8 @@ namespace sage {
 namespace {
 
 constexpr int SUB = 64;  // keys per softmax sub-tile
+// fp32(log2 448): FP8 P.V forms p = 448 * 2^(t - m) as 2^(arg + log2 448)
+constexpr float kLog2_448 = 8.807354927062988f;
 
 template <int D, bool PV8, int GR>
 struct Cfg {
@@ -737,19 +739,18 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
       if (!tile_max(sv, m_blk)) return false;
       m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
       alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
-      // P^ = e4m3(448 p), four per TMEM column, written over S
+      // P^ = e4m3(p), p formed already scaled by 448 in the exponent
+      // (2^(arg + log2 448): no multiply), four per TMEM column, written over S;
+      // the row sum l is of the scaled p, so the 448 cancels in the epilogue
+      const float sub = __fsub_rn(kLog2_448, m_new);
 #pragma unroll
       for (int cc = 0; cc < SUB / 16; ++cc) {
         float pv[16];
-        rowsum += full_tile ? row_exp<false, 16, TOK || SMQ>(sv + 16 * cc, ce, -m_new, key0 + 16 * cc, limit, pv)
-                            : row_exp<true, 16, TOK || SMQ>(sv + 16 * cc, ce, -m_new, key0 + 16 * cc, limit, pv);
+        rowsum += full_tile ? row_exp<false, 16, TOK || SMQ>(sv + 16 * cc, ce, sub, key0 + 16 * cc, limit, pv)
+                            : row_exp<true, 16, TOK || SMQ>(sv + 16 * cc, ce, sub, key0 + 16 * cc, limit, pv);
         uint32_t packed[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 a = __fmul2_rn(make_float2(pv[4 * k], pv[4 * k + 1]), make_float2(448.0f, 448.0f));
-          const float2 bb = __fmul2_rn(make_float2(pv[4 * k + 2], pv[4 * k + 3]), make_float2(448.0f, 448.0f));
-          packed[k] = pack_e4m3x4(a.x, a.y, bb.x, bb.y);
-        }
+        for (int k = 0; k < 4; ++k) packed[k] = pack_e4m3x4(pv[4 * k], pv[4 * k + 1], pv[4 * k + 2], pv[4 * k + 3]);
         ptx::tmem_st4(tS + 4 * cc, packed);
       }
       if (i > 0) {
@@ -800,7 +801,7 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
     for (int k = 0; k < 32; ++k) {
       if constexpr (PV8) {
         const float acc = __fmaf_rn(alpha_prev, o32[32 * cc + k], __uint_as_float(ov[k]));
-        const float vf = __fdiv_rn(__ldg(p.v_scale + w.vs_idx * D + 32 * cc + k), 448.0f);
+        const float vf = __ldg(p.v_scale + w.vs_idx * D + 32 * cc + k);
         o[k] = __fmul_rn(__fmul_rn(acc, vf), inv_l);
       } else {
         o[k] = __fmul_rn(__uint_as_float(ov[k]), inv_l);
