@@ -926,7 +926,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
       bool ok = true;
       for (int t = 0; t < nt && ok; ++t) {
         const int slot = fill % NS;
-        if (fill >= NS) {  // lane 0 waits; the verdict is the warp's
+        if (fill >= NS) {  // lane 0 waits; the outcome is the warp's
           if (lane == 0) ok = ptx::mbar_wait(&empty[slot], ((fill / NS) & 1) ^ 1);
           ok = __shfl_sync(0xffffffffu, ok, 0);
         }
