@@ -132,3 +132,37 @@ def test_grouped_varlen_sizes_and_validation(lib):
     f = lib.sage_attn_fwd_varlen_gqa
     assert f(FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 4, 100, 300, 8, 3, 64, 0, 0.0, 0, FAKE, 1 << 40,
              None) == 1
+
+
+def test_q_smoothing_sizes_and_validation(lib):
+    """Q smoothing's workspace adds the block means and the fp32 per-key mean
+    term; packed batches size the term from max_seqlen; the plain split-stage
+    entry points refuse the smoothing granularity."""
+    B, H, N, D = 1, 4, 1000, 64
+    NB = (N + 127) // 128
+    al = lambda x: (x + 255) // 256 * 256
+    plain = lib.sage_workspace_bytes_ex(B, H, H, N, D, 1, 0)
+    sq = lib.sage_workspace_bytes_ex(B, H, H, N, D, 1, 2)
+    assert sq == plain + al(B * H * NB * D * 4) + al(B * H * NB * NB * 128 * 4)
+    assert lib.sage_workspace_bytes_ex(B, H, H, N, D, 1, 3) == 0        # unknown granularity
+    # packed: 0 through the _ex query (no max_seqlen), sized by the _sq query
+    assert lib.sage_workspace_bytes_varlen_ex(5000, 4, 8, 8, 128, 1, 2) == 0
+    short = lib.sage_workspace_bytes_varlen_sq(5000, 4, 1000, 8, 8, 128, 1)
+    long_ = lib.sage_workspace_bytes_varlen_sq(5000, 4, 4000, 8, 8, 128, 1)
+    base = lib.sage_workspace_bytes_varlen_ex(5000, 4, 8, 8, 128, 1, 0)
+    assert base < short < long_
+    assert lib.sage_workspace_bytes_varlen_sq(5000, 4, -1, 8, 8, 128, 1) == 0
+    # the plain split stages refuse qk_gran 2 before touching anything
+    q = lib.sage_quantize_ex
+    assert q(FAKE, FAKE, FAKE, 0, B, H, H, N, D, 0, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+             FAKE, 1 << 40, None) == 1
+    a = lib.sage_attn_quantized_ex
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, B, H, H, N, D, 0, 0.0, 0, 2,
+             FAKE, 1 << 40, None) == 1
+    # the smoothing stages validate like the others (D = 96 rejected)
+    qs = lib.sage_quantize_sq
+    assert qs(FAKE, FAKE, FAKE, 0, B, H, H, N, 96, 0, 0, 0.0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+              FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == 1
+    aq = lib.sage_attn_quantized_sq
+    assert aq(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, B, H, H, N, 96, 0, 0.0,
+              0, FAKE, 1 << 40, None) == 1
