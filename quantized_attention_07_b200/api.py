@@ -598,5 +598,43 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, attn_mask=None,
     return attn_fwd(q, k, v, causal=is_causal, sm_scale=scale, pv_mode=pv_mode, qk_gran=qk_gran)
 
 
+# The entry-point names of the SageAttention guide's API list ("SageAttention
+# complete guide", advanced features: sageattn, sageattn_qk_int8_pv_fp8_cuda,
+# sageattn_varlen), for callers switching over.  Each is argument marshalling
+# around attn_fwd / attn_fwd_varlen; every step runs in this library's kernels.
+
+def sageattn_qk_int8_pv_fp16_cuda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  is_causal: bool = False, sm_scale: Optional[float] = None,
+                                  qk_gran: str = "block") -> torch.Tensor:
+    """INT8 QK^T, 16-bit P.V with fp32 accumulation, [B, H, N, D] inputs."""
+    q, k, v = (t if t.is_contiguous() else t.contiguous() for t in (q, k, v))
+    return attn_fwd(q, k, v, causal=is_causal, sm_scale=sm_scale, pv_mode="fp16", qk_gran=qk_gran)
+
+
+PV_ACCUM_DTYPES = ("fp32+fp32", "fp32")
+
+
+def sageattn_qk_int8_pv_fp8_cuda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                 is_causal: bool = False, sm_scale: Optional[float] = None,
+                                 qk_gran: str = "block",
+                                 pv_accum_dtype: str = "fp32+fp32") -> torch.Tensor:
+    """INT8 QK^T, FP8 P.V with two-level fp32 accumulation (each 64-key tile's
+    partial flushed into an fp32 accumulator).  pv_accum_dtype names that
+    accumulation ("fp32+fp32"; "fp32" is taken as the same); other
+    accumulation types are not implemented (SageError(SAGE_ERR_UNSUPPORTED))."""
+    if pv_accum_dtype not in PV_ACCUM_DTYPES:
+        raise SageError(2, f"pv_accum_dtype {pv_accum_dtype!r}")
+    q, k, v = (t if t.is_contiguous() else t.contiguous() for t in (q, k, v))
+    return attn_fwd(q, k, v, causal=is_causal, sm_scale=sm_scale, pv_mode="fp8", qk_gran=qk_gran)
+
+
+def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                    max_seqlen: int, is_causal: bool = False, sm_scale: Optional[float] = None,
+                    pv_mode: str = "fp16", qk_gran: str = "block") -> torch.Tensor:
+    """Packed [T, H, D] sequences with int32 cu_seqlens (see attn_fwd_varlen)."""
+    return attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=is_causal, sm_scale=sm_scale,
+                           pv_mode=pv_mode, qk_gran=qk_gran)
+
+
 def default_sm_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)

@@ -33,3 +33,21 @@ def test_host_pipeline_equals_device_call(B, H, Hkv, N, D, dtype, causal, pv_mod
         torch.cuda.synchronize()
         sage.sync_status()
         assert torch.equal(hout, want.cpu())
+
+
+def test_guide_entry_points_equal_the_core_calls():
+    """The guide's API names run the same kernels as attn_fwd / attn_fwd_varlen."""
+    dev = torch.device("cuda")
+    q, k, v = (t.to(dev) for t in W.make_dense(1, 4, 700, 128, "bf16", seed=8))
+    a = sage.sageattn_qk_int8_pv_fp16_cuda(q, k, v, is_causal=True)
+    b = sage.attn_fwd(q, k, v, causal=True, pv_mode="fp16")
+    assert torch.equal(a, b)
+    a = sage.sageattn_qk_int8_pv_fp8_cuda(q, k, v, pv_accum_dtype="fp32+fp32")
+    b = sage.attn_fwd(q, k, v, pv_mode="fp8")
+    assert torch.equal(a, b)
+    qp, kp, vp, cu = (t.to(dev) for t in W.make_varlen([300, 129], 4, 64, "fp16", seed=9))
+    a = sage.sageattn_varlen(qp, kp, vp, cu, 300, is_causal=True)
+    b = sage.attn_fwd_varlen(qp, kp, vp, cu, 300, causal=True)
+    torch.cuda.synchronize()
+    sage.sync_status()
+    assert torch.equal(a, b)

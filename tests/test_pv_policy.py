@@ -48,3 +48,12 @@ def test_reference_rows_validation_on_host():
     assert f(F, F, F, 2, 1, 8, 2, 64, 64, 0, 0.0, F, 4, F, None) == 1   # dtype
     assert f(F, F, F, 0, 1, 8, 2, 64, 64, 0, float("nan"), F, 4, F, None) == 1
     assert f(F, F, F, 0, 1, 8, 2, 64, 64, 0, 0.0, F, 0, F, None) == 0   # nothing to do
+
+
+def test_fp8_entry_point_refuses_other_accumulation_types():
+    import torch
+
+    import quantized_attention_07_b200 as sage
+    x = torch.zeros((1, 1, 128, 64), dtype=torch.float16)
+    with pytest.raises(sage.SageError):
+        sage.sageattn_qk_int8_pv_fp8_cuda(x, x, x, pv_accum_dtype="fp16")
