@@ -85,8 +85,9 @@ def tensor_peak(pk: dict, pv_mode: str, sustained: bool = False) -> float:
 
 
 def _code_only(src: str) -> str:
-    """C++ source without comments and blank-line / trailing-space differences,
-    so that an edit of the comments does not count as a new kernel."""
+    """C++ source without comments, blank lines and whitespace differences, so
+    that an edit of the comments or of the layout does not count as a new
+    kernel."""
     out, i, n = [], 0, len(src)
     while i < n:
         if src.startswith("//", i):
@@ -104,7 +105,7 @@ def _code_only(src: str) -> str:
         else:
             out.append(src[i])
             i += 1
-    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    lines = [" ".join(ln.split()) for ln in "".join(out).splitlines()]
     return "\n".join(ln for ln in lines if ln)
 
 

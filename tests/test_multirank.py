@@ -71,3 +71,14 @@ def test_stage1_algorithmic_bytes():
     gqa = W.WORKLOADS["llm_gqa_8k"]
     assert bench.quant_algorithmic_bytes(gqa) == 3 * 8192 * 128 * (32 + 8)
     assert bench.quant_algorithmic_bytes(W.WORKLOADS["varlen_8seq"]) == 0
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The traffic record is keyed by the attention source without comments:
+    a comment edit keeps the key, a code edit changes it."""
+    src = 'int f(int x) {  // scale\n  /* twice */ return 2 * x;  // "//" stays\n}\nconst char* s = "/*x*/";\n'
+    same = 'int f(int x) {\n\n  return 2 * x;   // doubled\n}\nconst char* s = "/*x*/";\n'
+    code = 'int f(int x) {  // scale\n  return 3 * x;\n}\nconst char* s = "/*x*/";\n'
+    assert bench._code_only(src) == bench._code_only(same)
+    assert bench._code_only(src) != bench._code_only(code)
+    assert '"/*x*/"' in bench._code_only(src)
