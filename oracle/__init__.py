@@ -28,14 +28,12 @@ _CFLAGS = ["-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
 ORACLE_OK = 0
 ORACLE_ERR_RANGE = 1
 
-# Key-tile length of the online softmax (and of the FP8 two-level flush).
-# FlashAttention's tiling has no fixed tile size on the pages; 64 keys is the
-# reading taken (the quantisation block stays 128 tokens).
-KV_TILE = 64
-
-# How far (base 2) a tile's maximum must exceed the maximum in use before p is
-# re-referenced to it; see sage_oracle.c.  16-bit P.V: 8; FP8 P.V: 0.
-TAU = {"fp16": 8.0, "fp8": 0.0}
+# The plain form of the method (see sage_oracle.c): the online softmax and
+# the FP8 two-level flush run over the 128-token key blocks of the quantised K,
+# with the plain running maximum.  Other evaluation orders (shorter key tiles,
+# a threshold on moving the maximum, the FP8 P scale applied in the exponent,
+# a fixed-order fp32 Q-smoothing term) are parameters of the calls below.
+BLOCK = 128
 
 
 def build(force: bool = False) -> str:
@@ -68,10 +66,11 @@ def lib():
         L.oracle_attn_ref_rows.argtypes = [P, P, P, i64, i32, i64, i64, i64, f64, i32, P, i64, P]
         L.oracle_attn_ref_rows.restype = None
         L.oracle_attn_emul_rows.argtypes = [P, P, P, P, P, i64, P, P, i64, i32, i32, i32, f32, f32,
-                                            i32, i32, i32, P, i64, P, i32, P, i64]
+                                            i32, i32, i32, P, i64, P, i32, P, i64, i32]
         L.oracle_attn_emul_rows.restype = None
-        L.oracle_q_smooth_bias.argtypes = [P, i64, P, i64, i32, i64, P, f32, P, i64]
-        L.oracle_q_smooth_bias.restype = None
+        for name in ("oracle_q_smooth_bias", "oracle_q_smooth_bias_fma"):
+            getattr(L, name).argtypes = [P, i64, P, i64, i32, i64, P, f32, P, i64]
+            getattr(L, name).restype = None
         _lib = L
     return _lib
 
@@ -179,30 +178,34 @@ def attn_ref_rows(q, k, v, sm_scale: float, causal: bool, rows) -> np.ndarray:
 
 
 def q_smooth_bias(qmean: np.ndarray, k: np.ndarray, kmean: np.ndarray, sm_scale: float,
-                  ldo: Optional[int] = None) -> np.ndarray:
+                  ldo: Optional[int] = None, order: str = "fp64") -> np.ndarray:
     """Per-key term of Q smoothing for one head: [nb, ldo] fp32 with
-    out[I, j] = fp32(kappa * qmean[I] . (k[j] - kmean)) for j < n (0 beyond),
-    the dot product as fp32 fused multiply-adds in channel order.
+    out[I, j] = kappa * qmean[I] . (k[j] - kmean) for j < n (0 beyond).
+    order "fp64": the dot product in fp64, rounded once (the plain form);
+    "fma": fp32 fused multiply-adds in channel order, then times kappa.
     qmean: [nb, D] block means of Q; k: [n, D]; kmean: [D]."""
     qmean, k, kmean = _f32(qmean), _f32(k), _f32(kmean)
     nb, D = qmean.shape
     n = k.shape[0]
     ldo = n if ldo is None else ldo
     out = np.zeros((nb, ldo), dtype=np.float32)
-    lib().oracle_q_smooth_bias(_p(qmean), nb, _p(k), n, D, D, _p(kmean), float(kappa(sm_scale)),
-                               _p(out), ldo)
+    fn = {"fp64": lib().oracle_q_smooth_bias, "fma": lib().oracle_q_smooth_bias_fma}[order]
+    fn(_p(qmean), nb, _p(k), n, D, D, _p(kmean), float(kappa(sm_scale)), _p(out), ldo)
     return out
 
 
 def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, causal: bool,
                    pv_mode: str, rows, v=None, p16: str = "fp16", vc=None, vdelta=None,
-                   blk: int = 128, kv: int = KV_TILE, tau=None,
+                   blk: int = BLOCK, kv: int = BLOCK, tau: float = 0.0, p8_exp: bool = False,
                    per_token: bool = False, bias: Optional[np.ndarray] = None) -> np.ndarray:
     """The quantised method's output rows (fp32) for one head; see sage_oracle.c.
-    blk: quantisation block (tokens); kv: key tile of the online softmax;
-    per_token: qdelta / kdelta hold one delta per token (blk is then unused);
-    bias: Q smoothing's per-key term [nb, >= n] (q_smooth_bias), per-block
-    deltas only."""
+    blk: quantisation block (tokens); per_token: qdelta / kdelta hold one delta
+    per token (blk is then unused); bias: Q smoothing's per-key term
+    [nb, >= n] (q_smooth_bias), per-block deltas only.
+    The defaults are the plain method.  Other evaluation orders: kv (key tile
+    of the online softmax and of the FP8 flush, a divisor of the block), tau
+    (threshold on moving the maximum) and p8_exp (FP8 P scale applied in the
+    exponent)."""
     if not per_token and blk % kv:
         raise ValueError("the key tile must divide the quantisation block")
     if bias is not None and per_token:
@@ -223,8 +226,8 @@ def attn_emul_rows(qc, qdelta, kc, kdelta, n: int, D: int, sm_scale: float, caus
         vc_p, vd_p, v_p, ldv, mode = _p(vc), _p(vdelta), None, D, 1
     lib().oracle_attn_emul_rows(_p(qc), _p(qdelta), _p(kc), _p(kdelta), v_p, ldv, vc_p, vd_p, n,
                                 D, blk, kv, float(kappa(sm_scale)),
-                                float(TAU[pv_mode] if tau is None else tau), int(causal), mode,
+                                float(tau), int(causal), mode,
                                 1 if p16 == "bf16" else 0, _p(rows), len(rows), _p(out),
                                 int(bool(per_token)), _p(bias),
-                                0 if bias is None else bias.shape[1])
+                                0 if bias is None else bias.shape[1], int(bool(p8_exp)))
     return out

@@ -220,10 +220,13 @@ def _group(picks):
 def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, causal: bool,
                  pv_mode: str, sm_scale: Optional[float] = None,
                  seqlens: Optional[list[int]] = None, gran: str = "block",
-                 k: Optional[torch.Tensor] = None) -> dict:
+                 k: Optional[torch.Tensor] = None, kv: int = BLK, tau: float = 0.0,
+                 p8_exp: bool = False, bias_order: str = "fp64") -> dict:
     """E for the listed (seq, head, row) picks -> {pick: fp32 [D]}.  gran
     "block_sq" needs k (one head per query head; dense [B,H,N,D] or packed
-    [T,H,D]) for the per-key term of Q smoothing."""
+    [T,H,D]) for the per-key term of Q smoothing.  The defaults give the plain
+    method; kv, tau, p8_exp and bias_order select another evaluation order
+    (see attn_emul_rows and q_smooth_bias)."""
     cu = None if cu_seqlens is None else [int(c) for c in cu_seqlens.tolist()]
     sm_scale = default_sm_scale(D) if sm_scale is None else sm_scale
     p16 = "bf16" if v.dtype == torch.bfloat16 else "fp16"
@@ -238,15 +241,16 @@ def emulate_rows(qz: Quantized, v: torch.Tensor, cu_seqlens, picks, D: int, caus
         bias = None
         if gran == "block_sq" and cu is None:
             bias = q_smooth_bias(qz.q_mean[s, h], k[s, h].float().numpy(), qz.k_mean[s, h],
-                                 sm_scale)
+                                 sm_scale, order=bias_order)
         elif gran == "block_sq":
             b0 = sum((cu[i + 1] - cu[i] + BLK - 1) // BLK for i in range(s))
             nb = (n + BLK - 1) // BLK
             bias = q_smooth_bias(qz.q_mean[h, b0:b0 + nb],
                                  k[cu[s]:cu[s + 1], h].float().numpy(), qz.k_mean[s, h],
-                                 sm_scale)
+                                 sm_scale, order=bias_order)
         o = attn_emul_rows(qc, qd, kc, kd, n, D, sm_scale, causal, pv_mode, rows, v=vv, p16=p16,
-                           vc=vc, vdelta=vd, per_token=gran == "token", bias=bias)
+                           vc=vc, vdelta=vd, per_token=gran == "token", bias=bias, kv=kv,
+                           tau=tau, p8_exp=p8_exp)
         for r, i in enumerate(rows):
             out[(s, h, i)] = o[r]
     return out

@@ -310,7 +310,7 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
 /* E: the quantised method, step by step.                                    */
 /* ------------------------------------------------------------------------ */
 
-/* fp32(log2 448): the FP8 P scale, applied in the exponent */
+/* fp32(log2 448): the FP8 P scale when it is applied in the exponent */
 #define LOG2_448F 8.807354927062988f
 
 /*
@@ -320,24 +320,22 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  * (smoothed K), and either the 16-bit V values (pv_mode 0) or V's E4M3 codes
  * and per-channel deltas (pv_mode 1).  `blk` is the quantisation block; `kv`
  * (a divisor of blk) is the key-tile length of the tiled online softmax and of
- * the FP8 two-level flush -- the pages give FlashAttention's tiling without a
- * tile size ("Attention机制优化", section 3.1); the reading taken is 64 keys.
- * kappa = fp32(sm_scale * log2(e)): the softmax runs in base 2.
- * tau >= 0: the maximum m used to compute p is moved only when the tile's
- * maximum exceeds it by more than tau (base-2 units); in real arithmetic the
- * rescale factors cancel in O / l, so any tau gives the same attention, and
- * tau = 0 is the plain running maximum.  Reading taken: tau = 8 for 16-bit
- * P.V (p then stays below 2^8, exactly representable in range of fp16/bf16),
- * tau = 0 for FP8 P.V (P^ = e4m3(448 p) needs p <= 1).
+ * the FP8 two-level flush.  kappa = fp32(sm_scale * log2(e)): the softmax
+ * runs in base 2.
  *
- * For each row i (query block I = i / blk) and key tile T = 0, 1, ... in
- * ascending order (tiles starting at or before i when causal), the tile's keys
- * lying in quantisation block J = T*kv / blk, with m = -inf, l = 0, O = 0:
+ * THE METHOD (the plain form; kv = blk = 128, tau = 0, p8_exp = 0).  The
+ * pages give FlashAttention's tiled online softmax ("Attention机制优化",
+ * section 3.1) over the key blocks of the quantised K, and flush the FP8
+ * partial sums into the fp32 accumulator once per block ("SageAttention
+ * v1/v2/v2++/v3" overview, SageAttention 2 bullet 3).  For each row i (query
+ * block I = i / blk) and key tile T = 0, 1, ... in ascending order (tiles
+ * starting at or before i when causal), the tile's keys lying in quantisation
+ * block J = T*kv / blk, with m = -inf, l = 0, O = 0:
  *
  *   S_ij   = sum_d q^_id k^_jd                       exact int32
  *   c_IJ   = fp32( fp32(deltaQ_I * deltaK_J) * kappa )   dequant x softmax scale
  *   mb     = fp32(max_j S_ij * c_IJ)                   the tile's scaled max
- *   m_new  = mb if mb > m + tau, else m
+ *   m_new  = max(m, mb)                                the running maximum
  *   arg_ij = fmaf(S_ij, c_IJ, -m_new)                 dequant, scale and max
  *                                                     subtraction in one fused
  *                                                     multiply-add (reading of
@@ -351,23 +349,37 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  *     P_ij  = p_ij rounded to V's 16-bit format
  *     Part  = fp32(sum_j P_ij v_jd)                   (products summed in fp64)
  *     O_d   = fp32(fp32(alpha * O_d) + Part_d)
- *   pv_mode 1 (FP8 P.V, two-level accumulation): p is formed scaled by the
- *   static P scale 448 in the exponent, arg_ij = fmaf(S_ij, c_IJ,
- *   fp32(L - m_new)) with L = fp32(log2 448), so p_ij = 448 2^(t - m) and
- *   l sums these scaled p:
- *     P^_ij = e4m3(p_ij)
- *     Part  = fp32(sum_j dec(P^_ij) dec(v^_jd))       one key block's partial
- *     O_d   = fmaf(alpha, O_d, Part_d)                flushed into the fp32
- *                                                     accumulator every block
+ *   pv_mode 1 (FP8 P.V, two-level accumulation; static P scale 448, since
+ *   p <= 1 at the running maximum):
+ *     P^_ij = e4m3(fp32(p_ij * 448))
+ *     Part  = fp32(sum_j dec(P^_ij) dec(v^_jd))       one key tile's partial
+ *     O_d   = fp32(fp32(alpha * O_d) + Part_d)        flushed into the fp32
+ *                                                     accumulator every tile
  *   m = m_new
  *
  * Finally out_d = fp32(O_d / l)   (pv_mode 0), or
- *           out_d = fp32(fp32(O_d * deltaV_d) / l)   (pv_mode 1: the 448 of
- *           P and the 448 of l cancel).
+ *           out_d = fp32(O_d * deltaV_d / (448 l))   (pv_mode 1; the exact
+ *           value of the expression, rounded once).
  *
  * Masked keys (j >= n, or j > i when causal) take no part in the maximum and
  * contribute p = 0.  (A tile is entered only if it holds at least one
  * unmasked key of the row.)
+ *
+ * OTHER EVALUATION ORDERS of the same method.  In exact arithmetic the
+ * rescale factors cancel in O / l, so the following change only roundings;
+ * they exist so that a faster evaluation order can also be checked step for
+ * step:
+ *   kv < blk   shorter key tiles (both parts of a block share its deltas);
+ *   tau > 0    the maximum in use moves only when the tile's maximum exceeds
+ *              it by more than tau (base 2): m_new = mb if mb > m + tau,
+ *              else m; p may then reach 2^tau (16-bit P.V only: FP8 needs
+ *              p <= 1);
+ *   p8_exp = 1 (FP8 P.V) the P scale is applied in the exponent: arg_ij =
+ *              fmaf(S_ij, c_IJ, fp32(L - m_new)), L = fp32(log2 448), so p_ij
+ *              = 448 2^(t - m) directly, P^_ij = e4m3(p_ij), l sums these
+ *              scaled p, the flush is O_d = fmaf(alpha, O_d, Part_d), and
+ *              out_d = fp32(fp32(O_d * deltaV_d) / l) (the 448 of P and of l
+ *              cancel).
  *
  * p16_format: 0 = fp16, 1 = bf16 (V's own format, used for P in pv_mode 0).
  * out: [nrows][D] fp32.
@@ -387,19 +399,20 @@ void oracle_attn_ref_rows(const float* q, const float* k, const float* v, long n
  * the postsniper.ru post's SageAttention2 bullet 1, which also normalise Q).
  * The Q codes are those of q~ = q - qmean_I (per-block channel mean of Q), and
  * the part of q.k~ that the mean carries is added back per key:
- * bk[I*ldb + j] = fp32(kappa * qmean_I . k~_j) (see oracle_q_smooth_bias).
+ * bk[I*ldb + j] = kappa * qmean_I . k~_j (see oracle_q_smooth_bias).
  * Per-block deltas only:
  *   c_IJ   = fp32( fp32(deltaQ_I * deltaK_J) * kappa )
  *   y_ij   = fmaf(S_ij, c_IJ, bk_Ij)                  scaled logit
  *   mb     = max_j y_ij
- *   arg_ij = fp32(y_ij - m_new)
+ *   arg_ij = fp32(y_ij - m_new)    (p8_exp: fp32(y_ij + fp32(L - m_new)))
  * everything else as above.
  */
 void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* kc,
                            const float* kdelta, const float* v, long ldv, const uint8_t* vc,
                            const float* vdelta, long n, int D, int blk, int kv, float kappa,
                            float tau, int causal, int pv_mode, int p16_format, const long* rows,
-                           long nrows, float* out, int per_token, const float* bk, long ldb)
+                           long nrows, float* out, int per_token, const float* bk, long ldb,
+                           int p8_exp)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (long r = 0; r < nrows; ++r) {
@@ -455,8 +468,9 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
             }
             float m_new = mblk > m + tau ? mblk : m;
             float alpha = (float)exp2((double)(m - m_new));
-            /* FP8 P.V: p is formed already scaled by 448, as 2^(arg + log2 448) */
-            const float sub = pv_mode == 0 ? -m_new : LOG2_448F - m_new;
+            /* p8_exp: p is formed already scaled by 448, as 2^(arg + log2 448) */
+            const int fold = pv_mode == 1 && p8_exp;
+            const float sub = fold ? LOG2_448F - m_new : -m_new;
             double psum = 0.0;
             for (int jj = 0; jj < nj; ++jj) {
                 float arg = bk ? y[jj] + sub
@@ -475,18 +489,21 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
                 for (int d = 0; d < D; ++d) O[d] = alpha * O[d] + (float)part[d];
             } else {
                 for (int jj = 0; jj < nj; ++jj) {
-                    double P = oracle_e4m3_decode(oracle_e4m3_encode(p[jj]));
+                    const float p448 = fold ? p[jj] : p[jj] * 448.0f;
+                    double P = oracle_e4m3_decode(oracle_e4m3_encode(p448));
                     const uint8_t* vr = vc + (j0 + jj) * D;
                     for (int d = 0; d < D; ++d) part[d] += P * oracle_e4m3_decode(vr[d]);
                 }
-                for (int d = 0; d < D; ++d) O[d] = fmaf(alpha, O[d], (float)part[d]);
+                for (int d = 0; d < D; ++d)
+                    O[d] = fold ? fmaf(alpha, O[d], (float)part[d]) : alpha * O[d] + (float)part[d];
             }
             m = m_new;
         }
         float* o = out + r * D;
         for (int d = 0; d < D; ++d) {
             if (pv_mode == 0) o[d] = O[d] / l;
-            else o[d] = (O[d] * vdelta[d]) / l;  /* the 448 of P and of l cancel */
+            else if (p8_exp) o[d] = (O[d] * vdelta[d]) / l;  /* the 448 of P and of l cancel */
+            else o[d] = (float)((double)O[d] * (double)vdelta[d] / (448.0 * (double)l));
         }
         free(O); free(part); free(S); free(p); free(y);
     }
@@ -506,18 +523,37 @@ void oracle_attn_emul_rows(const int8_t* qc, const float* qdelta, const int8_t* 
  * smoothing; the term here uses the smoothed k~ = fp32(k - kmean) that the K
  * codes come from.)
  *
- *   acc    = 0;  acc = fmaf(qmean[I][d], k~_j[d], acc)  for d = 0 .. D-1
- *   out[I*ldo + j] = fp32(acc * kappa)
- *
- * The pages fix no precision for this dot product; it is the kernel's: fp32
- * fused multiply-adds in channel order, so that the term, and every FP8 code
- * of P that depends on it, agrees bit for bit.
+ * The pages fix no precision for this dot product.  The plain form:
+ *   out[I*ldo + j] = fp32( kappa * sum_d qmean[I][d] * k~_j[d] )
+ * with the products and the sum in fp64 (exact products of fp32 values) and
+ * one rounding at the end.
  *
  * qmean: [nb][D]; k: row j at k + j*ld; kmean: [D]; out: [nb][ldo], columns
  * j < n written.
  */
 void oracle_q_smooth_bias(const float* qmean, long nb, const float* k, long n, int D, long ld,
                           const float* kmean, float kappa, float* out, long ldo)
+{
+    for (long I = 0; I < nb; ++I) {
+        for (long j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) {
+                const float ks = k[j * ld + d] - kmean[d];
+                acc += (double)qmean[I * D + d] * (double)ks;
+            }
+            out[I * ldo + j] = (float)((double)kappa * acc);
+        }
+    }
+}
+
+/*
+ * The same term in a fixed fp32 evaluation order (another evaluation order of
+ * the step above, used to check such an order step for step):
+ *   acc = 0;  acc = fmaf(qmean[I][d], k~_j[d], acc)  for d = 0 .. D-1
+ *   out[I*ldo + j] = fp32(acc * kappa)
+ */
+void oracle_q_smooth_bias_fma(const float* qmean, long nb, const float* k, long n, int D, long ld,
+                              const float* kmean, float kappa, float* out, long ldo)
 {
     for (long I = 0; I < nb; ++I) {
         for (long j = 0; j < n; ++j) {

@@ -552,3 +552,131 @@ def test_per_token_varlen_layout_matches_dense_per_sequence():
             assert np.array_equal(qz.k_codes[h, r0:r0 + n], dz.k_codes[0, h, :n])
             assert np.array_equal(qz.k_delta[h, r0:r0 + n], dz.k_delta[0, h, :n])
         r0 += ((n + 127) // 128) * 128
+
+
+# --------------------------------------------- E exact: powers-of-two inputs --
+
+def _kappa_one_scale() -> float:
+    """An fp32 sm_scale with kappa = fp32(sm_scale * log2 e) = 1 exactly, so the
+    base-2 logits are the dequantised scores themselves."""
+    sm = float(np.float32(math.log(2.0)))
+    assert float(oracle.kappa(sm)) == 1.0
+    return sm
+
+
+def _exact_inputs(n, D, seed, eq=(0, 1), ek=(-1, 0, -1), nz=(1, 2, 2), ev=(-8, -7, -6)):
+    """q, k, v for which every step of E is exact and every p is a power of two.
+
+    Codes: Q row r of block I has three entries +-1 in channels 2..D-1
+    (times 2^eq_I); K rows nz_J entries +-1 (+-2 in blocks with ek_J = -1) with
+    zero channel sums per block (times 2^ek_J; the first block's logits are
+    smaller, so the running maximum moves later); each Q block holds the code 127
+    in channel 0 and each K block 127 and -127 in channel 1, channels no other
+    operand touches, so the deltas are exactly 2^eq_I, 2^ek_J and the K mean is
+    0.  With kappa = 1 the base-2 logit t_ij = S_ij 2^(eq_I + ek_J) is an
+    integer in [-8, 8] (eq in {0, 1}, ek in {-1, 0}).
+    V: e4m3 values times 2^ev_d per channel, each channel holding +-448, so V's
+    FP8 codes and scales reproduce it exactly (and it is exact in fp16)."""
+    rng = np.random.default_rng(seed)
+    q = np.zeros((n, D), np.int64)
+    k = np.zeros((n, D), np.int64)
+    for i in range(n):
+        for d in rng.choice(np.arange(2, D), size=3, replace=False):
+            q[i, d] = rng.choice([-1, 1])
+    for b in range(0, n, 128):
+        rows = np.arange(b, min(n, b + 128))
+        half = len(rows) // 2
+        mag = 2 if ek[(b // 128) % len(ek)] == -1 else 1
+        for r in rows[:half]:  # pairs of opposite rows: zero channel sums
+            for d in rng.choice(np.arange(2, D), size=nz[(b // 128) % len(nz)], replace=False):
+                k[r, d] = mag * rng.choice([-1, 1])
+        k[rows[half:2 * half]] = -k[rows[:half]]
+        q[b, 0] = 127
+        k[b, 1], k[rows[-1] if len(rows) > 1 else b, 1] = 127, -127
+    qs = np.array([2.0 ** eq[(i // 128) % len(eq)] for i in range(n)])[:, None]
+    ks = np.array([2.0 ** ek[(i // 128) % len(ek)] for i in range(n)])[:, None]
+    codes = rng.integers(0, 126, size=(n, D))          # e4m3 magnitudes below 448
+    vmag = oracle.e4m3_decode(codes.astype(np.uint8)).reshape(n, D)
+    vmag[rng.integers(0, n, size=D), np.arange(D)] = 448.0
+    vsign = rng.choice([-1.0, 1.0], size=(n, D))
+    v = vmag * vsign * np.array([2.0 ** ev[d % len(ev)] for d in range(D)])[None, :]
+    return (q * qs).astype(np.float32), (k * ks).astype(np.float32), v.astype(np.float32)
+
+
+EXACT_VARIANTS = [
+    ("fp16", {}),
+    ("fp8", {}),
+    ("fp16", dict(kv=64, tau=8.0)),
+    ("fp8", dict(p8_exp=True)),
+]
+
+
+@pytest.mark.parametrize("pv_mode,opts", EXACT_VARIANTS)
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulation_exact_on_power_of_two_probabilities(pv_mode, opts, causal):
+    """Every p is 2^-a with a <= 15: P is exact in fp16, 448 p is exact in e4m3,
+    the rescale factors are powers of two, and the row sums are exact in fp32.
+    So E equals the fp64 reference up to the fp32 rounding of the partial sums
+    and of the final division (|E - R| <= 1e-5 max|v|), in either P.V mode and
+    in the other evaluation orders.  A rescale applied one block late or
+    never, a partial flushed twice or not at all, the delta of a wrong block,
+    a transposed operand or a mask slip each move rows by O(|v|)."""
+    n, D = 300, 16
+    q, k, v = _exact_inputs(n, D, seed=41 + causal)
+    sm = _kappa_one_scale()
+    qt, kt, vt = (torch.from_numpy(x)[None, None].half() for x in (q, k, v))
+    for a, b in ((qt, q), (kt, k), (vt, v)):
+        assert np.array_equal(a[0, 0].float().numpy(), b)
+    qz = heads.quantize(qt, kt, vt, None, pv_mode)
+    assert qz.q_delta[0, 0].tolist() == [1.0, 2.0, 1.0]
+    assert qz.k_delta[0, 0].tolist() == [0.5, 1.0, 0.5]
+    assert not qz.k_mean.any()
+    if pv_mode == "fp8":
+        dec = oracle.e4m3_decode(qz.v_codes[0, 0]).reshape(n, D) * qz.v_delta[0, 0][None, :]
+        assert np.array_equal(dec, v.astype(np.float64))
+    # preconditions: integer logits with a spread of at most 15 per row, and a
+    # running maximum that moves after the first block for many rows
+    t = (q.astype(np.float64) @ k.T.astype(np.float64))
+    assert np.array_equal(t, np.round(t))
+    mask = np.tril(np.ones((n, n), bool)) if causal else np.ones((n, n), bool)
+    tm = np.where(mask, t, np.nan)
+    assert (np.nanmax(tm, axis=1) - np.nanmin(tm, axis=1)).max() <= 15
+    first = np.nanmax(np.where(mask[:, :128], t[:, :128], np.nan), axis=1)
+    assert (first[128:] < np.nanmax(tm, axis=1)[128:]).mean() > 0.3
+    picks = [(0, 0, i) for i in range(n)]
+    out = heads.emulate_rows(qz, vt, None, picks, D, causal, pv_mode, sm, **opts)
+    E = np.stack([out[p] for p in picks])
+    R = oracle.attn_ref_rows(q, k, v, sm, causal, np.arange(n))
+    assert np.abs(E - R).max() <= 1e-5 * np.abs(v).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulation_fp8_within_the_rounding_of_p(causal):
+    """FP8 P.V on exactly quantisable Q, K (power-of-two block deltas, so the
+    running maximum moves between blocks) and exactly e4m3-representable V:
+    the only approximation left in E is P^ = e4m3(448 p), whose error is at most
+    2^-4 p (normal range) or 2^-10 / 448 (subnormal), so for every row i and
+    channel d
+        |E_id - R_id| <= sum_j max(2^-4 p_ij, 2^-10/448) |v_jd| / sum_j p_ij
+    with p_ij = exp(logit_ij - max_j logit_ij) from the fp64 reference."""
+    n, D = 300, 16
+    q, k, _ = _lossless_inputs(n, D, 18, q_exp=(0, -1, 1), k_exp=(-1, 0, 1))
+    _, _, v = _exact_inputs(n, D, seed=19)
+    sm = 1.0 / 12000.0
+    qt, kt, vt = (torch.from_numpy(x)[None, None].half() for x in (q, k, v))
+    qz = heads.quantize(qt, kt, vt, None, "fp8")
+    assert qz.q_delta[0, 0].tolist() == [1.0, 0.5, 2.0] and not qz.k_mean.any()
+    picks = [(0, 0, i) for i in range(n)]
+    out = heads.emulate_rows(qz, vt, None, picks, D, causal, "fp8", float(np.float32(sm)))
+    E = np.stack([out[p] for p in picks]).astype(np.float64)
+    R = oracle.attn_ref_rows(q, k, v, float(np.float32(sm)), causal, np.arange(n))
+    logit = q.astype(np.float64) @ k.T.astype(np.float64) * float(np.float32(sm))
+    if causal:
+        logit = np.where(np.tril(np.ones((n, n), bool)), logit, -np.inf)
+    p = np.exp(logit - logit.max(axis=1, keepdims=True))
+    perr = np.maximum(2.0 ** -4 * p, np.where(p > 0, 2.0 ** -10 / 448, 0.0))
+    bound = perr @ np.abs(v.astype(np.float64)) / p.sum(axis=1, keepdims=True)
+    slack = 1e-5 * np.abs(v).max()
+    assert np.all(np.abs(E - R) <= bound + slack)
+    # the bound is not vacuous: P^'s rounding shows, well inside it
+    assert 1e-4 * bound.max() < np.abs(E - R).max() < 0.5 * bound.max()
