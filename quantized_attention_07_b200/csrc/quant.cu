@@ -1253,16 +1253,15 @@ static cudaError_t launch_quant_t(const SeqLayout& L, dim3 grid, const void* q, 
   // (pass 1 alone for Q only; per-block deltas only).
   if (!L.varlen && items + 4096 < (1LL << 31)) {
     using S = Stream<D>;
-    static int sms = 0;  // per template instance
-    if (sms == 0) {
-      int dev = 0;
-      cudaGetDevice(&dev);
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      const cudaError_t e = cudaFuncSetAttribute(quant_stream_kernel<D, BF16, FP8>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)S::SMEM);
-      if (e != cudaSuccess) { sms = 0; return e; }
-    }
+    // Per call, on the current device: a function attribute is per device, so
+    // a value cached by the first caller would not hold on another device.
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(quant_stream_kernel<D, BF16, FP8>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+    if (e != cudaSuccess) return e;
     const long long cap = (long long)sms * S::CTAS_PER_SM;
     const int blocks = (int)(items < cap ? items : cap);
     // Items claimed but not yet finished: at most (ring slots + 1) per CTA.
