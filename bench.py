@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the side workloads timed next to the headline one")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (smaller cases for profiler captures; not a bench line)")
     return ap.parse_args()
@@ -201,27 +203,27 @@ class ClockSampler:
 
 # --------------------------------------------------------------- our arm --
 
-def run_ours(args, rank, world, local):
+def config_of(wl, inp, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    in_bytes = sum(t.numel() * t.element_size() for t in (inp.q, inp.k, inp.v))
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D,
+            "Hkv": wl.kv_heads, "qk_gran": wl.qk_gran,
+            "in_dtype": wl.dtype, "causal": wl.causal, "pv_mode": wl.pv_mode,
+            "seqlens": inp.seqlens if wl.varlen else None,
+            "l2": f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB of q,k,v > 126 MiB)"
+            if in_bytes > L2_BYTES else "inputs smaller than L2 (no flush)",
+            "parallelism": f"replicas x{world}"}
+
+
+def build_step(wl, inp, dev):
+    """The two stages of one step of the workload through the public API, on
+    device-resident inputs.  Returns (stage1, stage2, out, ws, launches per
+    step, grouped)."""
     import quantized_attention_07_b200 as sage
     from quantized_attention_07_b200 import api
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", device_id=dev,
-                                             timeout=datetime.timedelta(seconds=120))
-    wl = W.WORKLOADS[args.workload]
-    if args.heads:
-        wl = dataclasses.replace(wl, H=args.heads)
-    # each rank: its own seeded instance of the workload
-    inp = W.make_inputs(rank_workload(wl, rank))
-    ops = W.attention_ops(wl, inp.seqlens)
     q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
     cu = inp.cu_seqlens.to(dev) if inp.cu_seqlens is not None else None
-    stream = torch.cuda.current_stream(dev)
-    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
-
     grouped = not wl.varlen and wl.kv_heads != wl.H
     if grouped:
         # grouped-query attention: the whole public call per step (K, V
@@ -236,7 +238,7 @@ def run_ours(args, rank, world, local):
 
         def stage2():
             api.attn_fwd(q, k, v, causal=wl.causal, pv_mode=wl.pv_mode, out=out, workspace=ws)
-        launches_per_step = 3  # quant_stream_kernel (K, V), quant_stream_kernel (Q), attn_fwd
+        launches = 3  # quant_stream_kernel (K, V), quant_stream_kernel (Q), attn_fwd
     elif not wl.varlen:
         B, H, N, D = q.shape
         qz = api.alloc_quantized(B, H, N, D, wl.pv_mode, dev, qk_gran=wl.qk_gran)
@@ -251,7 +253,7 @@ def run_ours(args, rank, world, local):
             api.attn_quantized(qz, v, causal=wl.causal, out=out, workspace=ws)
         # quant_stream_kernel, attn_fwd_kernel; Q smoothing: Q in its own
         # kernel (quant_q_smooth_kernel) and the mean term (q_smooth_bias_kernel)
-        launches_per_step = 4 if wl.qk_gran == "block_sq" else 2
+        launches = 4 if wl.qk_gran == "block_sq" else 2
     else:
         T, H, D = q.shape
         out = torch.empty_like(q)
@@ -264,18 +266,21 @@ def run_ours(args, rank, world, local):
         def stage2():
             api.attn_fwd_varlen(q, k, v, cu, maxlen, causal=wl.causal, pv_mode=wl.pv_mode, out=out,
                                 workspace=ws)
-        launches_per_step = 4  # varlen_prep, quant_pass1, quant_pass2, attn_fwd
+        launches = 4  # varlen_prep, quant_pass1, quant_pass2, attn_fwd
+    return stage1, stage2, out, ws, launches, grouped
 
-    def step():
+
+def time_steps(stage1, stage2, ws, dev, K: int, warmup: int, local: int, world: int):
+    """W untimed steps, then K steps timed with CUDA events on the launching
+    stream (bracketed by a barrier and a synchronize), clocks sampled during
+    the timed region.  Returns (total ms, per-step stage-2 ms, per-step
+    stage-1 ms, clock summary)."""
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(warmup, 3)):
         stage1()
         stage2()
-
-    for _ in range(max(args.warmup, 3)):
-        step()
     torch.cuda.synchronize(dev)
     ws.sync_status()
-
-    K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     if world > 1:
         torch.distributed.barrier()
@@ -294,6 +299,73 @@ def run_ours(args, rank, world, local):
     total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
     attn_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
     quant_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    return total_ms, attn_ms, quant_ms, clk.summary()
+
+
+# Workloads timed next to the headline one in the same run (1 GPU): the FP8
+# P.V configurations (video-DiT D 64, packed causal D 128) and the causal
+# LLM block.
+SIDE_WORKLOADS = ("dit_8k_fp8", "varlen_8seq", "llm_causal_2k")
+SM_COUNT = 148
+
+
+def mufu_bound_ms(wl, seqlens, sm_mhz: float) -> float:
+    """Time of one 2^x per computed score on the special-function units
+    (16 per clock per SM): the attention kernel's non-tensor floor."""
+    scores = W.attention_ops(wl, seqlens) / (4.0 * wl.D)
+    return scores / (16.0 * SM_COUNT * sm_mhz * 1e6) * 1e3
+
+
+def side_config(name: str, dev, local: int, steps: int = 20) -> dict:
+    """One side workload: its step timed like the headline (whole step and the
+    attention stage alone), against the tensor peak and the MUFU floor."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl)
+    stage1, stage2, _, ws, _, _ = build_step(wl, inp, dev)
+    total_ms, attn_ms, _, clocks = time_steps(stage1, stage2, ws, dev, steps, 3, local, 1)
+    ops = W.attention_ops(wl, inp.seqlens)
+    pk = peaks()
+    peak = tensor_peak(pk, wl.pv_mode)
+    a_ms = statistics.mean(attn_ms)
+    achieved = ops / (a_ms * 1e-3) / 1e12
+    sm_max = clocks.get("sm_max_mhz") or 1965.0
+    mufu = mufu_bound_ms(wl, inp.seqlens, sm_max)
+    return {"workload": name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D, "causal": wl.causal,
+            "pv_mode": wl.pv_mode, "in_dtype": wl.dtype,
+            "seqlens": inp.seqlens if wl.varlen else None,
+            "value": round(job_throughput(ops, 1, steps, total_ms), 2),
+            "ms_per_step": round(total_ms / steps, 4),
+            "attn_ms": round(a_ms, 4), "attn_tops": round(achieved, 2),
+            "peak": round(peak, 1), "frac": round(achieved / peak, 4),
+            "frac_of_int8_peak": round(achieved / pk["int8"], 4),
+            "mufu_bound_ms": round(mufu, 4), "frac_of_mufu_bound": round(mufu / a_ms, 4),
+            "mufu_basis": f"one 2^x per computed score, 16/clk/SM x {SM_COUNT} SMs at "
+                          f"{sm_max:.0f} MHz",
+            "clocks": clocks, "steps": steps}
+
+
+def run_ours(args, rank, world, local):
+    import quantized_attention_07_b200 as sage
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev,
+                                             timeout=datetime.timedelta(seconds=120))
+    wl = W.WORKLOADS[args.workload]
+    if args.heads:
+        wl = dataclasses.replace(wl, H=args.heads)
+    # each rank: its own seeded instance of the workload
+    inp = W.make_inputs(rank_workload(wl, rank))
+    ops = W.attention_ops(wl, inp.seqlens)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (inp.q, inp.k, inp.v))
+    stage1, stage2, out, ws, launches_per_step, grouped = build_step(wl, inp, dev)
+
+    K = args.steps
+    total_ms, attn_ms, quant_ms, clocks = time_steps(stage1, stage2, ws, dev, K, args.warmup,
+                                                     local, world)
     total_ms = max_over_ranks(total_ms, dev)
 
     # end to end through the public call with host buffers: pinned H2D of the
@@ -338,6 +410,9 @@ def run_ours(args, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_throughput(wl, inp, budget_rows=8192, quant_heads=8)
+    side = None
+    if world == 1 and not args.no_per_config and not args.heads:
+        side = {n: side_config(n, dev, local) for n in SIDE_WORKLOADS if n != wl.name}
 
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -349,7 +424,6 @@ def run_ours(args, rank, world, local):
     achieved = ops / (attn_avg_ms * 1e-3) / 1e12
     peak = tensor_peak(pk, wl.pv_mode)
     value = job_throughput(ops, world, K, total_ms)
-    clocks = clk.summary()
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -363,13 +437,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "int8/fp8" if wl.pv_mode == "fp8" else "int8/fp16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D,
-                   "Hkv": wl.kv_heads, "qk_gran": wl.qk_gran,
-                   "in_dtype": wl.dtype, "causal": wl.causal, "pv_mode": wl.pv_mode,
-                   "seqlens": inp.seqlens if wl.varlen else None,
-                   "l2": f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB of q,k,v > 126 MiB)"
-                   if in_bytes > L2_BYTES else "inputs smaller than L2 (no flush)",
-                   "parallelism": f"replicas x{world}"},
+        "config": config_of(wl, inp, world),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(wl.name),
@@ -395,6 +463,8 @@ def run_ours(args, rank, world, local):
         line["e2e"] = e2e
     if cpu:
         line["cpu_baseline"] = cpu
+    if side:
+        line["per_config"] = side
     print(json.dumps(line), flush=True)
 
 
@@ -487,9 +557,7 @@ def run_reference(args, rank, world):
         "warmup": max(args.warmup, 3), "ms_per_step": round(1e3 * sum(t_steps) / K, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8/fp8" if wl.pv_mode == "fp8" else "int8/fp16", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D,
-                   "Hkv": wl.kv_heads, "qk_gran": wl.qk_gran,
-                   "in_dtype": wl.dtype, "causal": wl.causal, "pv_mode": wl.pv_mode},
+        "config": config_of(wl, inp, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": vals[0]["cores"],
                          "kind": "oracle",
                          "sample": "per step: " + vals[0]["sample"]},
