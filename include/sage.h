@@ -17,10 +17,16 @@
  *   - INT8 QK^T on the tensor cores, dequantised by deltaQ * deltaK
  *     (postsniper.ru page, step 3), fused with the softmax scale.
  *   - FlashAttention-style tiled online softmax ("Attention机制优化：从
- *     FlashAttention到SageAttention的工程实践", section 3.1).
+ *     FlashAttention到SageAttention的工程实践", section 3.1) over the 128-key
+ *     blocks of the quantised K.
  *   - P.V in 16 bits (postsniper.ru page, "SageAttention" bullet 3), or P and V
  *     in FP8 E4M3 with the FP8 partial product of every 128-key block flushed
  *     into an FP32 accumulator (dtcms.com page, SageAttention 2 bullets 1, 3).
+ *     With FP8 P.V, and with bf16 P in 16-bit P.V, p is formed against the
+ *     running maximum of whole 128-key blocks; with fp16 P the maximum is
+ *     taken per 64-key half-block and moves only when it rises by more than
+ *     8 (base 2), which changes only the rounding of P (the rescale factors
+ *     cancel in O / l).
  *   - The drop-in attention call shape q, k, v -> out over [B, H, N, D]
  *     ("sageattention in DeepSeek-VL2" (deepseek.csdn.net), step 2), plus a
  *     variable-length packed variant ("SageAttention complete guide"
@@ -71,7 +77,8 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1, SAGE_F32 = 2 /* outputs only */ } sa
 
 typedef enum {
   SAGE_PV_FP16 = 0, /* P.V with P rounded to V's 16-bit type, fp32 accumulate   */
-  SAGE_PV_FP8 = 1   /* P, V in FP8 E4M3, per-block fp32 two-level accumulation */
+  SAGE_PV_FP8 = 1   /* P, V in FP8 E4M3, fp32 two-level accumulation: the FP8
+                       partial of each 128-key block is flushed into fp32   */
 } sage_pv_mode_t;
 
 /* Granularity of the Q and K deltas ("SageAttention v1/v2/v2++/v3 overview",
@@ -150,7 +157,8 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
  * fp32(q - qmean_I), qmean_I the exact channel mean of the block's rows (the
  * K mean's definition), and the scaled logit is y = fmaf(S, c, b_Ij) with
  * b_Ij = fp32(kappa * qmean_I . fp32(k_j - kmean)), the dot product as fp32
- * fused multiply-adds in channel order, then arg = y - m.
+ * fused multiply-adds in channel order (within (D + 2) 2^-24 kappa
+ * sum_d |qmean_d k~_jd| of the exact value), then arg = y - m.
  * Its workspace also holds qmean and b (B*H*NB*(D + NB*128) floats).
  *   ws : at least sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, qk_gran).
  * sage_attn_fwd(...) = sage_attn_fwd_ex(..., Hkv = H, ..., SAGE_QK_PER_BLOCK).
@@ -234,6 +242,26 @@ sage_status_t sage_attn_fwd_varlen_ex(const void* q, const void* k, const void* 
                                       void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------ the two stages, separately -- */
+
+/*
+ * Smoothing and INT8 quantisation of Q and K alone (no V) for a dense
+ * [B, H, N, D] problem: K's per-channel mean over the N tokens of each head is
+ * subtracted ("SageAttention v1/v2/v2++/v3 overview" (dtcms.com),
+ * SageAttention v1 bullet 1), then every 128-token block of Q and of the
+ * smoothed K is quantised with delta = max|x| / 127, code = round(x / delta)
+ * ("SageAttention -- brand new attention" (postsniper.ru), quantisation intro
+ * steps 1-2).  This is the first stage of the qk_int8 entry points in the
+ * "SageAttention complete guide" API list.
+ *   q, k    : [B, H, N, D] 16-bit of type in_dt (SAGE_F16 or SAGE_BF16).
+ *   q_codes, k_codes, q_scale, k_scale, k_mean : as sage_quantize.
+ *   ws      : at least sage_scratch_bytes(B, H, D).
+ * Equal to sage_quantize with pv_mode SAGE_PV_FP16 (no V outputs); errors as
+ * sage_quantize (SAGE_ERR_RANGE through sage_sync_status for a K element
+ * outside the exact-mean range).
+ */
+sage_status_t sage_quant_qk(const void* q, const void* k, int in_dt, int B, int H, int N, int D,
+                            int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
+                            float* k_mean, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Stage 1 (smoothing + quantisation) of a dense problem into caller buffers:
@@ -348,8 +376,12 @@ sage_status_t sage_quantize_varlen(const void* q, const void* k, const void* v, 
  * device allocation, or a path that must not pay cudaMalloc's implicit
  * synchronisation).  It allocates nothing.
  *   status_out : optional DEVICE uint32; cleared by the call, then OR-ed with
- *                4 when a K element is non-finite or |k| >= 65536.  NULL:
- *                such errors are not reported.
+ *                4 when a K element is non-finite or |k| >= 65536, and with 1
+ *                when a bounded device-side wait gave up (the likeliest sign
+ *                of two calls racing on the shared array).  The outputs are
+ *                then unspecified.  NULL hides both errors: pass a word unless
+ *                the inputs and the call's exclusive use of the array are
+ *                known to be fine.
  * Limits and rules:
  *   - B*H*D <= SAGE_NOALLOC_MAX_BHD, else SAGE_ERR_WORKSPACE (nothing runs).
  *   - Every call shares the one array (per device) and it keeps the last
@@ -370,9 +402,32 @@ sage_status_t sage_quantize_noalloc(const void* q, const void* k, const void* v,
 /* ------------------------------------------------------------ diagnostics -- */
 
 /*
- * INT8 QK^T tiles through the same TMA + tcgen05 (kind::i8) path the attention
- * kernel uses: for each of n_tiles requests tiles[3*t .. 3*t+2] = (bh, I, J)
- * (host int32 array), writes S[r][c] = sum_d q_codes[bh][128 I + r][d] *
+ * The int32 QK^T scores of the attention kernel itself (postsniper.ru page,
+ * "SageAttention" bullet 1: QK^T in INT8).  Runs sage_attn_quantized (same
+ * arguments, same output `out`) with the fused attention kernel built to also
+ * store every 64-key sub-tile of S it computes, exactly as read from tensor
+ * memory before dequantisation, into
+ *   s_out : DEVICE int32 [B*H, NP, NP], NP = ceil(N/128)*128,
+ *           s_out[bh][i][j] = sum_d q_codes[bh][i][d] * k_codes[bh][j][d]
+ *           for query rows i < N and the keys j of every sub-tile the kernel
+ *           visits (non-causal: j < ceil(N/64)*64; causal: additionally
+ *           j < (i/128 + 1)*128).  Other entries are not written.
+ * Diagnostic: fp16 V (SAGE_PV_FP16 with v_dt SAGE_F16) or SAGE_PV_FP8 only,
+ * else SAGE_ERR_UNSUPPORTED.
+ */
+sage_status_t sage_attn_quantized_dump_s(const int8_t* q_codes, const float* q_scale,
+                                         const int8_t* k_codes, const float* k_scale,
+                                         const void* v, const uint8_t* v_codes,
+                                         const float* v_scale, void* out, int v_dt, int out_dt,
+                                         int B, int H, int N, int D, int causal, float sm_scale,
+                                         int pv_mode, int32_t* s_out, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+/*
+ * INT8 QK^T tiles by a separate one-tile kernel with the attention kernel's
+ * TMA loads and tcgen05 (kind::i8) instructions, as one M128 x N128 product:
+ * for each of n_tiles requests tiles[3*t .. 3*t+2] = (bh, I, J) (host int32
+ * array), writes S[r][c] = sum_d q_codes[bh][128 I + r][d] *
  * k_codes[bh][128 J + c][d] as int32 into s_out + t*128*128.  q_codes and
  * k_codes are the dense [B*H, NP, D] code arrays of sage_quantize.
  */
@@ -408,13 +463,24 @@ sage_status_t sage_selftest_wait_timeout(long long wait_cycles, void* ws, size_t
                                          void* stream);
 
 /*
- * Self-test of the software 2^x the attention kernel evaluates on the FMA
- * pipe for a share of the softmax exponentials (online softmax in base 2,
- * "Attention机制优化：从FlashAttention到SageAttention的工程实践", section 3.1):
- * y[i] = 2^x[i] for n DEVICE floats.  Valid for x >= -125 (smaller x are
- * clamped to -125); relative error below 2.2e-7.
+ * Self-test of the fused attention kernel's own failure path: runs
+ * sage_attn_quantized (same arguments) with every bounded wait limited to
+ * wait_cycles (1 .. 2^31) SM clock cycles, and with skip_k_stage = s > 0 every
+ * CTA leaves the K tile of its s-th pipeline stage unloaded, so the barrier
+ * of that stage never completes.  The waiting role gives up, records
+ * SAGE_ERR_TIMEOUT in the workspace's status word (returned by the next
+ * sage_sync_status), and every role of the CTA falls through to the teardown,
+ * which waits (bounded) for the CTA's own copies and MMAs and frees its tensor
+ * memory: the GPU and the workspace stay usable and `out` is unspecified.
+ * skip_k_stage = 0 runs the normal kernel with the shorter limit.
  */
-sage_status_t sage_selftest_exp2(const float* x, float* y, int n, void* stream);
+sage_status_t sage_selftest_attn_timeout(const int8_t* q_codes, const float* q_scale,
+                                         const int8_t* k_codes, const float* k_scale,
+                                         const void* v, const uint8_t* v_codes,
+                                         const float* v_scale, void* out, int v_dt, int out_dt,
+                                         int B, int H, int N, int D, int causal, float sm_scale,
+                                         int pv_mode, long long wait_cycles, int skip_k_stage,
+                                         void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

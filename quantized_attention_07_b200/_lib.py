@@ -53,8 +53,12 @@ SIGNATURES = {
     "sage_quantize_varlen": ([_P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                               _P, _P, _SZ, _P], _I),
     "sage_qk_int8_tiles": ([_P, _P, _I, _I, _I, _P, _I, _P, _P, _SZ, _P], _I),
+    "sage_quant_qk": ([_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "sage_attn_quantized_dump_s": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                    _F, _I, _P, _P, _SZ, _P], _I),
     "sage_selftest_wait_timeout": ([ctypes.c_longlong, _P, _SZ, _P], _I),
-    "sage_selftest_exp2": ([_P, _P, _I, _P], _I),
+    "sage_selftest_attn_timeout": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                    _F, _I, ctypes.c_longlong, _I, _P, _SZ, _P], _I),
     "sage_quantize_noalloc": ([_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
                                _P, _P], _I),
 }

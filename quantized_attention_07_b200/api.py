@@ -406,6 +406,43 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None,
     return qz
 
 
+def quant_qk(q: torch.Tensor, k: torch.Tensor,
+             workspace: Optional[Workspace] = None) -> Quantized:
+    """K smoothing and per-block INT8 quantisation of q and k alone (dense,
+    k with the heads of q), through sage_quant_qk."""
+    _need_cuda_contig(q, k)
+    B, H, N, D = q.shape
+    qz = alloc_quantized(B, H, N, D, "fp16", q.device)
+    ws = _workspace(q.device, int(_lib.load().sage_scratch_bytes(B, H, D)), workspace)
+    _check(_lib.load().sage_quant_qk(
+        _ptr(q), _ptr(k), _dtype_code(q.dtype), B, H, N, D, _ptr(qz.q_codes), _ptr(qz.q_scale),
+        _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(qz.k_mean), ws.ptr, ws.nbytes,
+        _stream(q.device)), "sage_quant_qk")
+    return qz
+
+
+def attn_quantized_dump_s(qz: Quantized, v: torch.Tensor, causal: bool = False,
+                          sm_scale: Optional[float] = None,
+                          fill: int = -2 ** 31) -> tuple[torch.Tensor, torch.Tensor]:
+    """Stage 2 of a dense problem (per-block deltas; fp16 V or FP8 P.V) with
+    the attention kernel's own int32 QK^T scores stored as it computes them.
+    Returns (out fp32 [B, H, N, D], S int32 [B*H, NP, NP]); entries of S the
+    kernel does not visit keep `fill`."""
+    _need_cuda_contig(v)
+    B, H, NP, D = qz.q_codes.shape
+    N = v.shape[2]
+    out = torch.empty((B, H, N, D), dtype=torch.float32, device=v.device)
+    s = torch.full((B * H, NP, NP), fill, dtype=torch.int32, device=v.device)
+    ws = _workspace(v.device, int(_lib.load().sage_scratch_bytes(B, H, D)), None)
+    _check(_lib.load().sage_attn_quantized_dump_s(
+        _ptr(qz.q_codes), _ptr(qz.q_scale), _ptr(qz.k_codes), _ptr(qz.k_scale), _ptr(v),
+        _ptr(qz.v_codes), _ptr(qz.v_scale), _ptr(out), _dtype_code(v.dtype),
+        _dtype_code(out.dtype, True), B, H, N, D, int(bool(causal)),
+        float(sm_scale) if sm_scale else 0.0, _pv(qz.pv_mode), _ptr(s), ws.ptr, ws.nbytes,
+        _stream(v.device)), "sage_attn_quantized_dump_s")
+    return out, s
+
+
 def attn_quantized(qz: Quantized, v: torch.Tensor, causal: bool = False,
                    sm_scale: Optional[float] = None, out_dtype: Optional[torch.dtype] = None,
                    out: Optional[torch.Tensor] = None,

@@ -253,7 +253,8 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
                          const float* v_scale, void* out, int v_dt, int out_dt, int B, int H,
                          int N, int D, int causal, float sm_scale, int pv_mode, void* ws,
                          cudaStream_t st, int Hkv, int per_token = 0,
-                         const float* q_bias = nullptr) {
+                         const float* q_bias = nullptr, int32_t* s_dump = nullptr,
+                         long long wait_limit = 0, int fault_skip_k = 0) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   AttnLaunch A{};
   A.p.H = H;
@@ -285,7 +286,12 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
   A.code_z_kv = B * Hkv;
   A.T = 0;
   A.p.items = B * H * A.p.NPAIR;
+  A.p.s_dump = s_dump;
+  A.p.s_dump_ld = (long long)A.p.NB * BLK;
+  A.p.wait_limit = wait_limit;
+  A.p.fault_skip_k = fault_skip_k;
   cudaError_t e = launch_attn(A, st);
+  if (e == cudaErrorNotSupported) return SAGE_ERR_UNSUPPORTED;
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "attention launch");
 }
 
@@ -377,6 +383,14 @@ sage_status_t sage_quantize(const void* q, const void* k, const void* v, int in_
                           stream);
 }
 
+sage_status_t sage_quant_qk(const void* q, const void* k, int in_dt, int B, int H, int N, int D,
+                            int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
+                            float* k_mean, void* ws, size_t ws_bytes, void* stream) {
+  return sage_quantize_ex(q, k, nullptr, in_dt, B, H, H, N, D, SAGE_PV_FP16, SAGE_QK_PER_BLOCK,
+                          q_codes, q_scale, k_codes, k_scale, k_mean, nullptr, nullptr, ws,
+                          ws_bytes, stream);
+}
+
 sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale,
                                      const int8_t* k_codes, const float* k_scale, const void* v,
                                      const uint8_t* v_codes, const float* v_scale, void* out,
@@ -449,6 +463,50 @@ sage_status_t sage_attn_quantized_sq(const int8_t* q_codes, const float* q_scale
   if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
   return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
                     H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), Hkv, 2, q_bias);
+}
+
+sage_status_t sage_attn_quantized_dump_s(const int8_t* q_codes, const float* q_scale,
+                                         const int8_t* k_codes, const float* k_scale,
+                                         const void* v, const uint8_t* v_codes,
+                                         const float* v_scale, void* out, int v_dt, int out_dt,
+                                         int B, int H, int N, int D, int causal, float sm_scale,
+                                         int pv_mode, int32_t* s_out, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !out_dtype_ok(out_dt) || !std::isfinite(sm_scale))
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !aligned16(k_scale) ||
+      !aligned16(out) || !aligned16(ws) || !aligned16(s_out))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+    return SAGE_ERR_INVALID_ARG;
+  if (!fp8 && v_dt != SAGE_F16) return SAGE_ERR_UNSUPPORTED;
+  if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
+  return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
+                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), H, 0, nullptr,
+                    s_out);
+}
+
+sage_status_t sage_selftest_attn_timeout(const int8_t* q_codes, const float* q_scale,
+                                         const int8_t* k_codes, const float* k_scale,
+                                         const void* v, const uint8_t* v_codes,
+                                         const float* v_scale, void* out, int v_dt, int out_dt,
+                                         int B, int H, int N, int D, int causal, float sm_scale,
+                                         int pv_mode, long long wait_cycles, int skip_k_stage,
+                                         void* ws, size_t ws_bytes, void* stream) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !out_dtype_ok(out_dt) || !std::isfinite(sm_scale) ||
+      wait_cycles < 1 || wait_cycles > (1LL << 31) || skip_k_stage < 0)
+    return SAGE_ERR_INVALID_ARG;
+  const bool fp8 = pv_mode == SAGE_PV_FP8;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !aligned16(k_scale) ||
+      !aligned16(out) || !aligned16(ws))
+    return SAGE_ERR_INVALID_ARG;
+  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+    return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
+  return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
+                    H, N, D, causal, sm_scale, pv_mode, ws, as_stream(stream), H, 0, nullptr,
+                    nullptr, wait_cycles, skip_k_stage);
 }
 
 size_t sage_workspace_bytes_ex(int B, int H, int Hkv, int N, int D, int pv_mode, int qk_gran) {

@@ -16,14 +16,16 @@
 //                read S from TMEM, dequantise with deltaQ*deltaK*sm_scale*log2 e,
 //                mask, online softmax in base 2, write P (fp16/bf16 or e4m3)
 //                back over S; 16-bit P.V: rescale O in TMEM when the maximum
-//                in use moves; FP8: fold the previous sub-tile's partial into
-//                an fp32 register accumulator (two-level accumulation).
+//                in use moves; FP8: fold the previous 128-key block's partial
+//                into an fp32 register accumulator (two-level accumulation).
 //
 // Each query tile owns two 64-column S buffers, so QK^T of sub-tile i+1 runs
 // on the tensor core while the softmax works on sub-tile i, and the two query
-// tiles keep both softmax warpgroups busy.  The maximum used for P moves only
-// when a row's tile maximum exceeds it by more than TAU (8 for 16-bit P.V,
-// so O rescales are rare; 0 for FP8 P.V, whose rescale is free in the flush).
+// tiles keep both softmax warpgroups busy.  With FP8 P.V or bf16 P the maximum
+// used for p is the plain running maximum over whole 128-key blocks: the first
+// half of a block waits for the second half's S as well and takes the maximum
+// over both.  With fp16 P it is taken per 64-key sub-tile and moves only when
+// a row's sub-tile maximum exceeds it by more than 8, so O rescales are rare.
 //
 // TMEM columns (512): S_0[0] [0,64) S_0[1] [64,128) S_1[0] [128,192)
 // S_1[1] [192,256) O_0 [256,256+D) O_1 [256+D,256+2D).
@@ -46,7 +48,6 @@
 #include <algorithm>
 
 #include "attn_launch.cuh"
-#include "exp2.cuh"
 #include "ptx.cuh"
 
 namespace sage {
@@ -68,7 +69,14 @@ struct Cfg {
   static constexpr int REG_CTRL = 56;
   static_assert(256 * REG_SOFTMAX + 128 * REG_CTRL <= 384 * 168,
                 "register split exceeds the launch allocation");
-  static constexpr float TAU = PV8 ? 0.0f : 8.0f;  // threshold for moving the maximum
+  // The maximum used for p: with FP8 P.V or bf16 P (a short format whose
+  // rounding of p must not depend on where a block is split) it is the plain
+  // running maximum over whole 128-key blocks (both 64-key halves of a block
+  // share it); with fp16 P it is taken per 64-key sub-tile and moves only when
+  // the sub-tile's maximum exceeds it by more than 8 (base 2: p < 2^8, exact
+  // in fp16's range), which makes the rescale of O rare.
+  static constexpr bool block_max(bool bf16v) { return PV8 || bf16v; }
+  static constexpr float tau(bool bf16v) { return block_max(bf16v) ? 0.0f : 8.0f; }
 
   static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
   static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
@@ -112,6 +120,7 @@ struct Bars {
   uint64_t k_full[8], v_full[8], kv_empty[8];
   uint32_t tmem_base;
   volatile int abort;
+  long long wait_limit;    // cycles before a bounded wait gives up
 };
 
 // Warp-uniform bounded wait: true when the phase completed, false (and the
@@ -124,7 +133,7 @@ __device__ __forceinline__ bool wait_bar(Bars* B, uint64_t* bar, uint32_t parity
     while (true) {
       if (ptx::mbar_try_wait(bar, parity)) { ok = true; break; }
       if (B->abort) break;
-      if (clock64() - t0 > SAGE_WAIT_LIMIT_CYCLES) {
+      if (clock64() - t0 > B->wait_limit) {
         set_status(status, ST_TIMEOUT);
         B->abort = 1;
         break;
@@ -331,7 +340,10 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
         } else {
           ptx::mbar_arrive_expect_tx(&B->k_full[s], C::QT + C::KS);
         }
-        ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
+        // (the timeout self-test leaves one K tile unloaded: its barrier then
+        // waits for bytes that never come)
+        if (p.fault_skip_k == 0 || G != p.fault_skip_k - 1)
+          ptx::tma_load_3d(sK + s * C::QT, tm_k, &B->k_full[s], 0, w.k_y0 + j * BLK, w.k_z);
         if constexpr (TOK)  // the stage's 128 per-token K deltas, on the same barrier
           ptx::bulk_load_plain(sKs + s * BLK, p.k_scale + (w.ks_idx0 + j) * BLK, C::KS,
                                &B->k_full[s]);
@@ -355,10 +367,10 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
   for (int jj = max(0, G - C::NS); jj < G; ++jj) {
     const int s = jj % C::NS;
     const uint32_t ph = (jj / C::NS) & 1;
-    ptx::mbar_wait(&B->k_full[s], ph);
-    ptx::mbar_wait(&B->v_full[s], ph);
+    ptx::mbar_wait(&B->k_full[s], ph, B->wait_limit);
+    ptx::mbar_wait(&B->v_full[s], ph, B->wait_limit);
   }
-  if (n > 0) ptx::mbar_wait(&B->q_full, (n - 1) & 1);
+  if (n > 0) ptx::mbar_wait(&B->q_full, (n - 1) & 1, B->wait_limit);
 }
 
 // ------------------------------------------------------------ MMA issuer --
@@ -419,7 +431,9 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
     const int I = I0 + i, g = G0 + i / 2;
     const uint32_t vb = ptx::smem_u32(sV + (g % C::NS) * C::VT + (i & 1) * C::V_SUB_BYTES);
     const uint32_t tP = tmem + 128 * t + SUB * (I & 1);
-    const uint32_t acc0 = PV8 ? 0u : (i > 0 ? 1u : 0u);  // an item's first P.V starts O
+    // an item's first P.V starts O; FP8: each block's first half starts a
+    // fresh partial, its second half accumulates into it
+    const uint32_t acc0 = PV8 ? ((i & 1) ? 1u : 0u) : (i > 0 ? 1u : 0u);
     if (ptx::elect_one()) {
       const uint64_t b0 = ptx::smem_desc(vb, C::V_LBO, C::V_SBO, C::V_SWZ);
 #pragma unroll
@@ -494,7 +508,7 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
   // Drain: every MMA this warp issued completes before TMEM is released.
   if (ptx::elect_one()) ptx::mma_commit(&B->done[t]);
   __syncwarp();
-  ptx::mbar_wait(&B->done[t], 0);
+  ptx::mbar_wait(&B->done[t], 0, B->wait_limit);
 }
 
 // --------------------------------------------------------------- softmax --
@@ -579,10 +593,6 @@ __device__ __forceinline__ float row_bias_max(uint32_t* v, const float* bk, floa
   return fmaxf(m0, m1);
 }
 
-// Share of the exponentials computed by the FMA-pipe polynomial: one pair in
-// POLY_EVERY (0 = none; every 2^x on the special-function unit).
-constexpr int POLY_EVERY = 0;
-
 // p for NC columns: p = 2^fma(S, c, -m) (masked columns give 0); returns the
 // sum of p.  Results are written to p[].
 template <bool MASKED, int NC, bool FIN = false>
@@ -596,15 +606,7 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
     const float2 x = FIN ? make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1]))
                          : s32x2_to_f32x2(v[i], v[i + 1]);
     const float2 a = __ffma2_rn(x, c2, n2);
-    float p0, p1;
-    if (POLY_EVERY > 0 && (i / 2) % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1) {
-      const float2 e = exp2_poly2(a);  // FMA-pipe 2^x for a share of the pairs
-      p0 = e.x;
-      p1 = e.y;
-    } else {
-      p0 = ptx::ex2(a.x);
-      p1 = ptx::ex2(a.y);
-    }
+    float p0 = ptx::ex2(a.x), p1 = ptx::ex2(a.y);
     if (MASKED) {
       if (first_key + i >= limit) p0 = 0.0f;
       if (first_key + i + 1 >= limit) p1 = 0.0f;
@@ -618,12 +620,18 @@ __device__ __forceinline__ float row_exp(const uint32_t* v, float c, float neg_m
   return s.x + s.y;
 }
 
-template <int D, bool PV8, bool BF16V, int GR>
+template <int D, bool PV8, bool BF16V, int GR, bool DUMP>
 __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w, Bars* B,
                                              uint32_t tmem, int t, const float* sKs, int I0,
                                              int G0, volatile int* loop) {
   using C = Cfg<D, PV8, GR>;
   [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
+  constexpr bool BM = C::block_max(BF16V);
+  constexpr float TAU = C::tau(BF16V);
+  // block maximum with 16-bit P: the even half's S stays in registers while
+  // the odd half's maximum is taken (FP8 P.V: the fp32 accumulator needs those
+  // registers, so S is loaded again)
+  constexpr bool KEEP = BM && !PV8;
   using In = In16<BF16V>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
@@ -646,6 +654,52 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
   }
   const int limit = p.causal ? min(w.n, row + 1) : w.n;  // keys >= limit are masked
 
+  // sub-tile ii: are all its keys unmasked for every row of the tile?
+  auto full_of = [&](int ii) -> bool {
+    const int k0 = ii * SUB;
+    return (k0 + SUB <= w.n) && (!p.causal || k0 + SUB - 1 <= qt * BLK);
+  };
+  // wait for QK^T of sub-tile ii and load its 64 columns of S
+  auto wait_s = [&](int ii) -> bool {
+    const int Ii = I0 + ii;
+    if (!wait_bar(B, &B->s_full[t][Ii & 1], (Ii / 2) & 1, p.status, true)) return false;
+    ptx::tc_fence_after();
+    return true;
+  };
+  auto load_s = [&](int ii, uint32_t (&sv)[SUB]) {
+    const uint32_t tS = tS0 + SUB * ((I0 + ii) & 1);
+#pragma unroll
+    for (int cc = 0; cc < SUB / 32; ++cc)
+      ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
+    ptx::tmem_wait_ld();
+  };
+  // The scaled maximum of sub-tile ii (-inf when no key of it is unmasked for
+  // this row).  Per token, S is first turned into y = fp32(S deltaK_j) in
+  // place (with Q smoothing into y = fma(S, c, b_j)); the K deltas or the mean
+  // term came with the K tile (wait on its barrier).
+  auto tile_max = [&](uint32_t (&sv)[SUB], int ii, float& m_blk) -> bool {
+    const int k0 = ii * SUB;
+    const bool full = full_of(ii);
+    if constexpr (TOK) {
+      const int g = G0 + ii / 2;  // ring stage of the sub-tile
+      if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, p.status, true)) return false;
+      const float* dk = sKs + (g % C::NS) * BLK + (ii & 1) * SUB;
+      const float ym = full ? row_scale_max<SUB, false>(sv, dk, k0, limit)
+                            : row_scale_max<SUB, true>(sv, dk, k0, limit);
+      m_blk = ym == -INFINITY ? -INFINITY : __fmul_rn(ym, c);
+    } else if constexpr (SMQ) {
+      const int g = G0 + ii / 2;
+      if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, p.status, true)) return false;
+      const float* bk = sKs + ((g % C::NS) * 2 + t) * BLK + (ii & 1) * SUB;
+      m_blk = full ? row_bias_max<SUB, false>(sv, bk, c, k0, limit)
+                   : row_bias_max<SUB, true>(sv, bk, c, k0, limit);
+    } else {
+      const int smax = full ? row_max<SUB>(sv, INT_MIN) : row_max_masked<SUB>(sv, INT_MIN, k0, limit);
+      m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+    }
+    return true;
+  };
+
   for (int i = 0; i < nsub; ++i) {
     const int I = I0 + i;                        // sub-tile count of this tile over the items
     const int b = I & 1;
@@ -654,50 +708,58 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
       const float kd = __ldg(p.k_scale + w.ks_idx0 + i / 2);
       c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
     }
-    if (!wait_bar(B, &B->s_full[t][b], (I / 2) & 1, p.status, true)) return false;
-    ptx::tc_fence_after();
+    if (!wait_s(i)) return false;
     const int key0 = i * SUB;
-    const bool full_tile = (key0 + SUB <= w.n) && (!p.causal || key0 + SUB - 1 <= qt * BLK);
-    float alpha, rowsum = 0.0f, m_new;
-    // The sub-tile's scaled maximum (-inf when no key of it is unmasked for
-    // this row).  Per token, S is first turned into y = fp32(S deltaK_j) in
-    // place; the K deltas came with the K tile (wait on its barrier).
-    auto tile_max = [&](uint32_t (&sv)[SUB], float& m_blk) -> bool {
-      if constexpr (TOK) {
-        const int g = G0 + i / 2;  // ring stage of the sub-tile
-        if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, p.status, true)) return false;
-        const float* dk = sKs + (g % C::NS) * BLK + (i & 1) * SUB;
-        const float ym = full_tile ? row_scale_max<SUB, false>(sv, dk, key0, limit)
-                                   : row_scale_max<SUB, true>(sv, dk, key0, limit);
-        m_blk = ym == -INFINITY ? -INFINITY : __fmul_rn(ym, c);
-      } else if constexpr (SMQ) {
-        const int g = G0 + i / 2;  // the mean term came with the K stage
-        if (!wait_bar(B, &B->k_full[g % C::NS], (g / C::NS) & 1, p.status, true)) return false;
-        const float* bk = sKs + ((g % C::NS) * 2 + t) * BLK + (i & 1) * SUB;
-        m_blk = full_tile ? row_bias_max<SUB, false>(sv, bk, c, key0, limit)
-                          : row_bias_max<SUB, true>(sv, bk, c, key0, limit);
-      } else {
-        const int smax = full_tile ? row_max<SUB>(sv, INT_MIN)
-                                   : row_max_masked<SUB>(sv, INT_MIN, key0, limit);
-        m_blk = smax == INT_MIN ? -INFINITY : __fmul_rn((float)smax, c);
+    const bool full_tile = full_of(i);
+    // `lead`: this sub-tile sets the maximum used for its p -- every sub-tile,
+    // or with the block maximum the first half of each 128-key block, whose
+    // maximum then covers the second half as well
+    const bool lead = !BM || (i & 1) == 0;
+    float alpha = 1.0f, rowsum = 0.0f, m_new = m;
+    uint32_t sv[SUB];
+    load_s(i, sv);
+    if constexpr (DUMP) {  // the raw int32 S of this row and sub-tile, as computed
+      if (row < w.n) {
+        int4* dst = reinterpret_cast<int4*>(
+            p.s_dump + ((long long)w.code_z * p.s_dump_ld + row) * p.s_dump_ld + key0);
+#pragma unroll
+        for (int k = 0; k < SUB / 4; ++k)
+          dst[k] = make_int4((int)sv[4 * k], (int)sv[4 * k + 1], (int)sv[4 * k + 2], (int)sv[4 * k + 3]);
       }
-      return true;
-    };
+    }
+    if (lead) {
+      float m_blk;
+      if (!tile_max(sv, i, m_blk)) return false;
+      if (BM && i + 1 < nsub) {
+        float m2;
+        if (!wait_s(i + 1)) return false;
+        if constexpr (KEEP) {
+          uint32_t sx[SUB];
+          load_s(i + 1, sx);
+          if (!tile_max(sx, i + 1, m2)) return false;
+        } else {
+          load_s(i + 1, sv);
+          if (!tile_max(sv, i + 1, m2)) return false;
+          load_s(i, sv);
+          if constexpr (TOK || SMQ) {
+            float unused;
+            if (!tile_max(sv, i, unused)) return false;
+          }
+        }
+        m_blk = fmaxf(m_blk, m2);
+      }
+      // a sub-tile (block) with no unmasked key for this row leaves the maximum unchanged
+      m_new = m_blk > __fadd_rn(m, TAU) ? m_blk : m;
+      alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
+    } else if constexpr (TOK || SMQ) {
+      float unused;  // second half of a block: S to scaled logits in place
+      if (!tile_max(sv, i, unused)) return false;
+    }
 
     // multiplier inside the exponent: c, or 1 once S holds the scaled logit
     // (Q smoothing: arg = fp32(y - m))
     const float ce = SMQ ? 1.0f : c;
     if constexpr (!PV8) {
-      uint32_t sv[SUB];
-#pragma unroll
-      for (int cc = 0; cc < SUB / 32; ++cc)
-        ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
-      ptx::tmem_wait_ld();
-      // a sub-tile with no unmasked key for this row leaves the maximum unchanged
-      float m_blk;
-      if (!tile_max(sv, m_blk)) return false;
-      m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
-      alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
 #pragma unroll
       for (int cc = 0; cc < SUB / 32; ++cc) {
         float pv[32];
@@ -708,9 +770,9 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
         for (int k = 0; k < 16; ++k) packed[k] = In::pack(pv[2 * k], pv[2 * k + 1]);
         ptx::tmem_st16(tS + 16 * cc, packed);
       }
-      // O <- alpha * O before this sub-tile's P.V accumulates into it (rare:
-      // only when some row's maximum moved by more than TAU)
-      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+      // O <- alpha * O before this sub-tile's P.V accumulates into it (only
+      // when some row's maximum moved by more than TAU)
+      if (lead && i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         if (!wait_bar(B, &B->o_full[t], (I - 1) & 1, p.status, true)) return false;
         ptx::tc_fence_after();
         const float2 a2 = make_float2(alpha, alpha);
@@ -729,16 +791,6 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
         }
       }
     } else {
-      // S of the sub-tile in one TMEM round trip
-      uint32_t sv[SUB];
-#pragma unroll
-      for (int cc = 0; cc < SUB / 32; ++cc)
-        ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
-      ptx::tmem_wait_ld();
-      float m_blk;
-      if (!tile_max(sv, m_blk)) return false;
-      m_new = m_blk > __fadd_rn(m, C::TAU) ? m_blk : m;
-      alpha = m_new == m ? 1.0f : ptx::ex2(__fsub_rn(m, m_new));
       // P^ = e4m3(p), p formed already scaled by 448 in the exponent
       // (2^(arg + log2 448): no multiply), four per TMEM column, written over S;
       // the row sum l is of the scaled p, so the 448 cancels in the epilogue
@@ -753,9 +805,11 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
         for (int k = 0; k < 4; ++k) packed[k] = pack_e4m3x4(pv[4 * k], pv[4 * k + 1], pv[4 * k + 2], pv[4 * k + 3]);
         ptx::tmem_st4(tS + 4 * cc, packed);
       }
-      if (i > 0) {
-        // two-level accumulation: O32 <- alpha_{i-1} O32 + Part_{i-1}, 64
-        // columns of the partial per TMEM round trip
+      if (lead && i > 0) {
+        // two-level accumulation, once per 128-key block: O32 <- alpha_{b-1}
+        // O32 + Part_{b-1}, the partial of both halves of the previous block
+        // (its P.V completed before this block's QK^T landed), 64 columns of
+        // the partial per TMEM round trip
         if (!wait_bar(B, &B->o_full[t], (I - 1) & 1, p.status, true)) return false;
         ptx::tc_fence_after();
         const float2 a2 = make_float2(alpha_prev, alpha_prev);
@@ -780,7 +834,7 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
     ptx::tc_fence_before();
     ptx::mbar_arrive(&B->p_full[t][b]);
     m = m_new;
-    alpha_prev = alpha;
+    if (lead) alpha_prev = alpha;
   }
 
   // ------------------------------------------------------------ epilogue --
@@ -835,7 +889,7 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
 // tile's sub-tiles so far, G0 the ring stages, loop[1] the items with keys
 // (o_done phase).  The item counts sit in a per-warp shared-memory slot
 // rather than in registers, which the per-sub-tile loop needs.
-template <int D, bool PV8, bool BF16V, int GR>
+template <int D, bool PV8, bool BF16V, int GR, bool DUMP>
 __device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, const float* sKs) {
   volatile int* loop = B->sm_loop[threadIdx.x / 32];  // [0] items taken, [1] items with keys
   loop[0] = 0;
@@ -850,7 +904,7 @@ __device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, c
     if (!w.valid) continue;
     const int nsub = t == 0 ? w.nsub0 : w.nsub1;
     if (nsub > 0) {
-      if (!softmax_item<D, PV8, BF16V, GR>(p, w, B, tmem, t, sKs, I0, G0, loop)) return;
+      if (!softmax_item<D, PV8, BF16V, GR, DUMP>(p, w, B, tmem, t, sKs, I0, G0, loop)) return;
       loop[1] = loop[1] + 1;
     }
     I0 += nsub;
@@ -860,7 +914,7 @@ __device__ void softmax_wg(const AttnParams& p, Bars* B, uint32_t tmem, int t, c
 
 // ---------------------------------------------------------------- kernel --
 
-template <int D, bool PV8, bool BF16V, int GR>
+template <int D, bool PV8, bool BF16V, int GR, bool DUMP>
 __global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -902,6 +956,7 @@ __global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
       ptx::mbar_init(&B->kv_empty[s], 2);  // one commit per query tile
     }
     B->abort = 0;
+    B->wait_limit = p.wait_limit > 0 ? p.wait_limit : SAGE_WAIT_LIMIT_CYCLES;
     ptx::fence_barrier_init();
   }
   if (warp == warp_mma) {
@@ -922,7 +977,7 @@ __global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
     }
   } else {
     ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
-    softmax_wg<D, PV8, BF16V, GR>(p, B, tmem, wg, sKs);
+    softmax_wg<D, PV8, BF16V, GR, DUMP>(p, B, tmem, wg, sKs);
   }
 
   ptx::tc_fence_before();
@@ -1060,7 +1115,7 @@ static CUtensorMapSwizzle swz_for(int row_bytes) {
   return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 }
 
-template <int D, bool PV8, bool BF16V, int GR>
+template <int D, bool PV8, bool BF16V, int GR, bool DUMP = false>
 static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
   using C = Cfg<D, PV8, GR>;
   [[maybe_unused]] constexpr bool TOK = GR == 1, SMQ = GR == 2;
@@ -1085,7 +1140,7 @@ static cudaError_t launch_attn_t(const AttnLaunch& L, cudaStream_t st) {
     okv = make_map3(&tv, vdt, esz, L.v, D, L.code_z_kv, L.T, (uint64_t)D * esz,
                     (uint64_t)D * esz * L.code_z_kv, vbox0, 1, BLK, vs);
   if (!okv) return cudaErrorInvalidValue;
-  auto kern = attn_fwd_kernel<D, PV8, BF16V, GR>;
+  auto kern = attn_fwd_kernel<D, PV8, BF16V, GR, DUMP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -1110,6 +1165,14 @@ static cudaError_t launch_attn_g(const AttnLaunch& L, cudaStream_t st) {
 }
 
 cudaError_t launch_attn(const AttnLaunch& L, cudaStream_t st) {
+  if (L.p.s_dump) {  // diagnostic instances: dense, per-block deltas, fp16 V or FP8 P.V
+    if (L.p.varlen || L.p.per_token || (!L.pv8 && L.bf16v)) return cudaErrorNotSupported;
+    if (L.D == 64)
+      return L.pv8 ? launch_attn_t<64, true, false, 0, true>(L, st)
+                   : launch_attn_t<64, false, false, 0, true>(L, st);
+    return L.pv8 ? launch_attn_t<128, true, false, 0, true>(L, st)
+                 : launch_attn_t<128, false, false, 0, true>(L, st);
+  }
   if (L.p.per_token == 2) return launch_attn_g<2>(L, st);
   return L.p.per_token ? launch_attn_g<1>(L, st) : launch_attn_g<0>(L, st);
 }

@@ -34,6 +34,16 @@ struct AttnParams {
   int items;             // work items of the launch: dense BH*NPAIR, varlen H*PM
   unsigned int* sched;   // [2] in the workspace header: next item, CTAs finished (zero between launches)
   uint32_t* status;
+  // diagnostic: when set (dense, per-block deltas, fp16 V or FP8 P.V only),
+  // every int32 S sub-tile the kernel computes is also stored here, row-major
+  // [BH][s_dump_ld][s_dump_ld] (query row, key), before its dequantisation
+  int32_t* s_dump;
+  long long s_dump_ld;   // NB * 128
+  // bounded waits: cycles before a wait gives up (0: SAGE_WAIT_LIMIT_CYCLES)
+  long long wait_limit;
+  // self-test of the timeout path: s > 0 leaves the K tile of every CTA's
+  // s-th pipeline stage unloaded, so that stage's barrier never completes
+  int fault_skip_k;
 };
 
 struct AttnLaunch {

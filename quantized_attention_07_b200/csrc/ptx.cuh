@@ -88,13 +88,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the barrier phase with the given parity has completed.  Returns
-// false if it did not complete within the cycle budget.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// false if it did not complete within limit_cycles SM clock cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit_cycles = SAGE_WAIT_LIMIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > SAGE_WAIT_LIMIT_CYCLES) return false;
+    if (clock64() - t0 > limit_cycles) return false;
   }
 }
 

@@ -3,7 +3,6 @@
 // records a timeout in the status word -- exactly what the attention kernel's
 // waits do when a pipeline partner never signals.  No fault, no trap.
 #include "common.cuh"
-#include "exp2.cuh"
 #include "ptx.cuh"
 
 namespace sage {
@@ -21,17 +20,6 @@ __global__ void wait_timeout_kernel(long long limit_cycles, uint32_t* status) {
     const long long t0 = clock64();
     while (!ok && clock64() - t0 <= limit_cycles) ok = ptx::mbar_try_wait(&bar, 0);
     if (!ok) set_status(status, ST_TIMEOUT);
-  }
-}
-
-__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
-    y[i] = r.x;
-    y[i + 1] = r.y;
-  } else if (i < n) {
-    y[i] = exp2_poly2(make_float2(x[i], 0.0f)).x;
   }
 }
 
@@ -53,13 +41,4 @@ extern "C" sage_status_t sage_selftest_wait_timeout(long long wait_cycles, void*
   cudaError_t e = sage::launch_wait_timeout(wait_cycles, static_cast<uint32_t*>(ws),
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
-}
-
-extern "C" sage_status_t sage_selftest_exp2(const float* x, float* y, int n, void* stream) {
-  if (n < 0 || (n > 0 && (!x || !y))) return SAGE_ERR_INVALID_ARG;
-  if (n == 0) return SAGE_OK;
-  const int threads = 256, pairs = (n + 1) / 2;
-  sage::exp2_poly_kernel<<<(pairs + threads - 1) / threads, threads, 0,
-                           static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

@@ -8,8 +8,45 @@ import torch
 import quantized_attention_07_b200 as sage
 from oracle import heads
 
-# Tolerances on the fp32 output against the oracle's emulation (max abs).
+# Tolerances on the fp32 output against the oracle's emulation of the plain
+# method (max abs): the contract.
 TOL = {"fp16": 2e-3, "fp8": 8e-3}
+
+# Agreement of the fp32 output with the oracle's emulation in the library's
+# own evaluation order (see `schedule`).  There the two sides take every
+# integer decision alike and round every p to P from the same maximum; what
+# is left is the special-function unit's 2^x (a few fp32 ulps), the order of
+# the sums inside one MMA and of the row sum l, and the reciprocal of l in the
+# epilogue, all ~1e-6 relative -- except where a p lies within those few ulps
+# of a rounding boundary of its 16- or 8-bit format and the two sides round
+# it apart: one such p moves its whole row by up to 2^-8 (bf16) or 2^-4 (e4m3)
+# of that p's share of the row, ~1e-3 on short rows.  Such rows are rare
+# (measured between two emulations: < 0.5 % of rows above 1e-5).  So the
+# check is on the bulk, with room for those rows:
+#   median |GPU - E_sched| <= 1e-6, 99th percentile <= 2e-5, and at most 2 % of
+#   the rows with a deviation above 1e-4.
+# A wrong scale, sub-tile, rescale or flush moves the bulk and fails it.
+TIGHT = dict(median=1e-6, q99=2e-5, row=1e-4, row_frac=0.02)
+
+
+def schedule(pv_mode: str, v_dtype: torch.dtype, qk_gran: str = "block") -> dict:
+    """The evaluation order of the CUDA kernels, as oracle emulation options.
+
+    FP8 P.V: the plain running maximum over 128-key blocks, the P scale 448
+    applied in the exponent (p = 2^(arg + log2 448)), l summing those scaled p.
+    16-bit P.V with bf16 P: the plain method.  16-bit P.V with fp16 P: the
+    maximum taken per 64-key sub-tile and moved only when it rises by more
+    than 8 (base 2).  Q smoothing: the mean term as fp32 fused multiply-adds
+    in channel order."""
+    if pv_mode == "fp8":
+        opt = dict(kv=128, tau=0.0, p8_exp=True)
+    elif v_dtype == torch.bfloat16:
+        opt = dict(kv=128, tau=0.0)
+    else:
+        opt = dict(kv=64, tau=8.0)
+    if qk_gran == "block_sq":
+        opt["bias_order"] = "fma"
+    return opt
 
 
 def half_ulp(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
@@ -103,9 +140,12 @@ def cosine(a: np.ndarray, b: np.ndarray) -> float:
 
 
 def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
-                         ref_cos_bar=0.999, qk_gran="block"):
-    """GPU fp32 output vs the oracle's emulation (max-abs tolerance) and the fp64
-    reference (cosine).  Also checks a 16-bit output run.  Returns a stats dict.
+                         ref_cos_bar=0.999, qk_gran="block", tight=TIGHT):
+    """GPU fp32 output vs the oracle's emulation of the plain method (max-abs
+    tolerance TOL, the contract), vs the emulation in the library's evaluation
+    order (the bulk statistics of `tight`), and vs the fp64 reference
+    (cosine).  Also checks a
+    16-bit output run against the plain emulation.  Returns a stats dict.
     Dense k, v with fewer heads than q run grouped-query attention on the GPU;
     the oracle sees them repeated (its repeat_kv)."""
     D = q.shape[-1]
@@ -122,21 +162,34 @@ def check_against_oracle(q, k, v, cu, causal, pv_mode, picks, sm_scale=None,
             g = q.shape[1] // k.shape[1]
             k, v = heads.repeat_kv_packed(k, g), heads.repeat_kv_packed(v, g)
     qz = heads.quantize(q, k, v, cu, pv_mode, gran=qk_gran)
-    emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran,
-                             k=k if qk_gran == "block_sq" else None)
+    kk = k if qk_gran == "block_sq" else None
+    emu = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran, k=kk)
+    sched = schedule(pv_mode, v.dtype, qk_gran)
+    emu_s = heads.emulate_rows(qz, v, cu, picks, D, causal, pv_mode, sm_scale, gran=qk_gran, k=kk,
+                               **sched)
     ref = heads.reference_rows(q, k, v, cu, picks, causal, sm_scale)
     E = np.stack([emu[p] for p in picks])
+    Es = np.stack([emu_s[p] for p in picks])
     R = np.stack([ref[p] for p in picks])
     G = gather(out32, picks, cu)
     G16 = gather(out16, picks, cu)
     tol = TOL[pv_mode]
     err = np.abs(G - E)
+    err_s = np.abs(G - Es)
     err16 = np.abs(G16 - E) - half_ulp(E, q.dtype)
+    row_s = err_s.max(axis=1)
     stats = dict(max_abs=float(err.max()), max_abs16=float(err16.max()),
+                 sched_median=float(np.median(err_s)), sched_q99=float(np.quantile(err_s, 0.99)),
+                 sched_rows_over=float((row_s > tight["row"]).mean()),
+                 max_abs_sched=float(err_s.max()), plain_vs_sched=float(np.abs(E - Es).max()),
                  cos_gpu_ref=cosine(G, R), cos_emu_ref=cosine(E, R))
     assert np.isfinite(G).all()
     assert err.max() <= tol, stats
     assert err16.max() <= tol, stats
+    assert err_s.max() <= tol, stats
+    assert stats["sched_median"] <= tight["median"], stats
+    assert stats["sched_q99"] <= tight["q99"], stats
+    assert stats["sched_rows_over"] <= tight["row_frac"], stats
     bar = min(ref_cos_bar, stats["cos_emu_ref"] - 1e-4)
     assert stats["cos_gpu_ref"] >= bar, stats
     return stats

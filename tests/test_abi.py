@@ -31,10 +31,48 @@ def declared_functions() -> list[str]:
 
 
 def test_header_declares_the_boundary():
+    """The entry points of the hot path's C ABI: smoothing + quantisation of Q
+    and K (sage_quant_qk), the whole forward pass over [B, H, N, D]
+    (sage_attn_fwd: q, k, v, out, B, H, N, D, causal, sm_scale, pv_mode) and
+    its variable-length variant taking cu_seqlens; plus the split stages, the
+    status word and the kernel's own int32 QK^T dump."""
     names = declared_functions()
-    for required in ("sage_attn_fwd", "sage_attn_fwd_varlen", "sage_quantize",
-                     "sage_attn_quantized", "sage_quantize_varlen", "sage_sync_status"):
+    for required in ("sage_quant_qk", "sage_attn_fwd", "sage_attn_fwd_varlen", "sage_quantize",
+                     "sage_attn_quantized", "sage_quantize_varlen", "sage_sync_status",
+                     "sage_attn_quantized_dump_s"):
         assert required in names
+    text = open(HEADER).read()
+    sig = re.search(r"sage_status_t sage_attn_fwd\((.*?)\);", text, flags=re.S).group(1)
+    params = [p.split()[-1].strip("*") for p in sig.split(",")]
+    for p in ("q", "k", "v", "out", "B", "H", "N", "D", "causal", "sm_scale", "pv_mode"):
+        assert p in params, p
+    sig = re.search(r"sage_status_t sage_attn_fwd_varlen\((.*?)\);", text, flags=re.S).group(1)
+    assert "cu_seqlens" in sig
+    sig = re.search(r"sage_status_t sage_quant_qk\((.*?)\);", text, flags=re.S).group(1)
+    params = [p.split()[-1].strip("*") for p in sig.split(",")]
+    for p in ("q", "k", "B", "H", "N", "D", "q_codes", "q_scale", "k_codes", "k_scale",
+              "k_mean", "ws"):
+        assert p in params, p
+
+
+def test_quant_qk_and_dump_reject_bad_arguments(lib):
+    """Host-side validation of the two newer entry points (nothing launches)."""
+    qa = dict(q=FAKE, k=FAKE, in_dt=0, B=1, H=2, N=256, D=64, qc=FAKE, qs=FAKE, kc=FAKE, ks=FAKE,
+              km=FAKE, ws=FAKE, wsb=1 << 30, st=None)
+    for bad in (dict(D=96), dict(N=0), dict(in_dt=2), dict(q=None), dict(kc=FAKE + 4),
+                dict(ws=None)):
+        a = dict(qa, **bad)
+        assert lib.sage_quant_qk(*a.values()) == 1, bad
+    a = dict(qa, wsb=16)
+    assert lib.sage_quant_qk(*a.values()) == 3
+    da = dict(qc=FAKE, qs=FAKE, kc=FAKE, ks=FAKE, v=FAKE, vc=FAKE, vs=FAKE, out=FAKE, v_dt=0,
+              out_dt=2, B=1, H=2, N=256, D=64, causal=0, sm=0.0, pv=0, s=FAKE, ws=FAKE,
+              wsb=1 << 30, st=None)
+    for bad in (dict(D=96), dict(s=None), dict(s=FAKE + 4), dict(out_dt=5), dict(pv=3)):
+        a = dict(da, **bad)
+        assert lib.sage_attn_quantized_dump_s(*a.values()) == 1, bad
+    a = dict(da, v_dt=1)  # bf16 V with 16-bit P.V: no diagnostic instance
+    assert lib.sage_attn_quantized_dump_s(*a.values()) == 2
 
 
 def test_library_exports_every_declared_symbol(lib):

@@ -1,10 +1,11 @@
 """GPU parity: the CUDA library against the CPU oracle on the same seeded inputs.
 
   * quantisation outputs (codes, deltas, K mean, FP8 V codes/scales): bit-exact,
-  * int32 QK^T tiles from the tcgen05 INT8 path: bit-exact,
+  * the int32 QK^T scores of the fused attention kernel itself: bit-exact,
   * attention output: within the stated max-abs tolerance of the oracle's
-    emulation of the method (fp32 output, and 16-bit output with half an ulp
-    of slack), and cosine >= 0.999 against the fp64 reference (or, where the
+    emulation of the plain method (fp32 output, and 16-bit output with half an
+    ulp of slack), within 1e-4 of the emulation in the library's evaluation
+    order, and cosine >= 0.999 against the fp64 reference (or, where the
     method's own accuracy is lower, no worse than the emulation's cosine).
 """
 from __future__ import annotations
@@ -80,7 +81,102 @@ def test_constant_k_channels_give_zero_codes():
     assert torch.equal(qz.k_mean.cpu(), k[:, :, 0, :].float())
 
 
+def test_quant_qk_bit_exact_and_equal_to_quantize():
+    """sage_quant_qk (Q and K only) against the oracle, and equal to the Q/K
+    outputs of sage_quantize."""
+    q, k, v = W.make_dense(2, 3, 777, 128, "bf16", bias_sigma=3.0, seed=91)
+    dev = torch.device("cuda")
+    qz = sage.quant_qk(q.to(dev), k.to(dev))
+    torch.cuda.synchronize()
+    sage.sync_status()
+    U.compare_quant_dense(qz, heads.quantize(q, k, v, None, "fp16"), "fp16")
+    full = U.gpu_quantize_dense(q, k, v, "fp16")
+    for a in ("q_codes", "q_scale", "k_codes", "k_scale", "k_mean"):
+        assert torch.equal(getattr(qz, a), getattr(full, a)), a
+
+
 # ----------------------------------------------------------- INT8 QK^T --
+
+def _random_codes(B, H, N, D, seed):
+    """int8 codes in [-127, 127] with padding rows 0, and rows of +-127 for the
+    extreme products (|S| up to 127^2 D)."""
+    rng = np.random.default_rng(seed)
+    NP = (N + 127) // 128 * 128
+    qc = rng.integers(-127, 128, size=(B, H, NP, D)).astype(np.int8)
+    kc = rng.integers(-127, 128, size=(B, H, NP, D)).astype(np.int8)
+    qc[:, :, N:] = 0
+    kc[:, :, N:] = 0
+    qc[:, :, 5] = 127
+    qc[:, :, N - 1] = -127
+    kc[:, :, 9] = -127
+    kc[:, :, 70] = 127      # second 64-key half of the first block
+    kc[:, :, N - 1] = 127
+    return qc, kc
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("pv_mode", ["fp16", "fp8"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [300, 777])
+def test_attention_kernel_s_bit_exact(D, pv_mode, causal, N):
+    """The int32 S = Q^ K^T of the fused attention kernel itself, stored as it
+    reads each 64-key sub-tile from tensor memory, equals the oracle's exact
+    integer product on every (row, key) the kernel visits: first, last,
+    diagonal and ragged-tail blocks, both 64-key halves of each block, the
+    extremes +-127^2 D; nothing outside the visited sub-tiles is written.  The
+    diagnostic build's output equals the product build's bit for bit."""
+    B, H = 1, 2
+    qc, kc = _random_codes(B, H, N, D, seed=N + D)
+    NP = qc.shape[2]
+    rng = np.random.default_rng(7)
+    dev = torch.device("cuda")
+    fp8 = pv_mode == "fp8"
+    qz = sage.alloc_quantized(B, H, N, D, pv_mode, dev)
+    qz.q_codes.copy_(torch.from_numpy(qc))
+    qz.k_codes.copy_(torch.from_numpy(kc))
+    qz.q_scale.copy_(torch.from_numpy(rng.uniform(0.5e-3, 2e-3, qz.q_scale.shape).astype(np.float32)))
+    qz.k_scale.copy_(torch.from_numpy(rng.uniform(0.5e-3, 2e-3, qz.k_scale.shape).astype(np.float32)))
+    v = torch.randn(B, H, N, D, generator=torch.Generator().manual_seed(3)).half().to(dev)
+    if fp8:
+        codes = rng.integers(0, 0x7E, size=qz.v_codes.shape) | (rng.integers(0, 2, size=qz.v_codes.shape) << 7)
+        qz.v_codes.copy_(torch.from_numpy(codes.astype(np.uint8)))
+        qz.v_scale.copy_(torch.from_numpy(rng.uniform(0.001, 0.01, qz.v_scale.shape).astype(np.float32)))
+    out_d, S = sage.attn_quantized_dump_s(qz, v, causal=causal)
+    out = sage.attn_quantized(qz, v, causal=causal, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    sage.sync_status()
+    assert torch.equal(out_d, out)
+    S = S.cpu().numpy().reshape(B * H, NP, NP)
+    ns = (N + 63) // 64
+    rows = np.arange(NP)[:, None]
+    keys = np.arange(NP)[None, :]
+    visited = (rows < N) & (keys < ns * 64)
+    if causal:
+        visited &= keys < (rows // 128 + 1) * 128
+    for bh in range(B * H):
+        want = oracle.qk_int(qc[0, bh], kc[0, bh], 0, NP, 0, NP)
+        U.assert_same(f"S head {bh}", S[bh][visited], want[visited])
+        assert np.all(S[bh][~visited] == -2 ** 31), "the kernel wrote outside its sub-tiles"
+    assert np.abs(S[:, :N, :N]).max() == 127 * 127 * D
+
+
+def test_attention_kernel_s_of_a_quantised_workload():
+    """The same dump on the codes of a quantised causal LLM-shaped input."""
+    q, k, v = W.make_dense(1, 2, 1000, 128, "fp16", 3.0, seed=20260002)
+    dev = torch.device("cuda")
+    qz = sage.quantize(q.to(dev), k.to(dev), v.to(dev), "fp8")
+    _, S = sage.attn_quantized_dump_s(qz, v.to(dev), causal=True)
+    torch.cuda.synchronize()
+    sage.sync_status()
+    qc, kc = qz.q_codes.cpu().numpy(), qz.k_codes.cpu().numpy()
+    S = S.cpu().numpy()
+    NP = qc.shape[2]
+    rows, keys = np.arange(NP)[:, None], np.arange(NP)[None, :]
+    visited = (rows < 1000) & (keys < (rows // 128 + 1) * 128) & (keys < 1024)
+    for bh in range(2):
+        want = qc[0, bh].astype(np.int64) @ kc[0, bh].astype(np.int64).T
+        assert np.array_equal(S[bh][visited].astype(np.int64), want[visited])
+
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_qk_int8_tiles_bit_exact(D):

@@ -1,8 +1,10 @@
 """Q smoothing (SageAttention2's smoothing of Q: "SageAttention v1/v2/v2++/v3
 overview", SageAttention2 bullet 2): the GPU block means, codes and deltas of
-the smoothed Q and the per-key mean term equal the oracle's bit for bit, the
-attention output matches the oracle's smoothed emulation, and on queries with
-a channel offset smoothing is more accurate than plain per-block deltas."""
+the smoothed Q equal the oracle's bit for bit, the per-key mean term lies
+within the fp32 error bound of the plain fp64 term (and equals the fixed-order
+fp32 form bit for bit), the attention output matches the oracle's smoothed
+emulation, and on queries with a channel offset smoothing is more accurate
+than plain per-block deltas."""
 from __future__ import annotations
 
 import numpy as np
@@ -33,26 +35,41 @@ def _inputs(B, H, Hkv, N, D, dtype, seed, q_off=3.0):
 
 
 def _check_bias(qz, ref, k_rep, H, N, causal, sm_scale):
-    """GPU q_bias against the oracle's term, bit for bit: both sum the exact
-    fp64 products in channel order and round once (the FP8 codes of P depend
-    on it).  k_rep: K with the key/value heads repeated to the query heads
-    (ref quantised from it)."""
+    """GPU q_bias against the oracle's term.
+
+    Contract: the plain term fp32(kappa * qmean . k~) (fp64 dot product,
+    rounded once), within the error bound of an fp32 evaluation: D fused
+    multiply-adds and one multiplication by kappa, each rounded once, give
+    |got - want| <= (D + 2) * 2^-24 * kappa * sum_d |qmean_d k~_d| (the standard
+    bound of recursive summation, gamma_D <= (D + 1) u for D u < 2^-10, plus
+    the final rounding of the fp64 side).
+    Evaluation order: the term as fp32 fused multiply-adds in channel order,
+    bit for bit.
+    k_rep: K with the key/value heads repeated to the query heads (ref
+    quantised from it)."""
     got = qz.q_bias.cpu().numpy()
     NB = (N + 127) // 128
     kf = k_rep.float().numpy()
-    B = k_rep.shape[0]
+    B, D = k_rep.shape[0], k_rep.shape[-1]
+    kap = float(oracle.kappa(sm_scale))
     for b in range(B):
         for h in range(H):
             want = oracle.q_smooth_bias(ref.q_mean[b, h], kf[b, h], ref.k_mean[b, h], sm_scale,
                                         ldo=NB * 128)
+            want_fma = oracle.q_smooth_bias(ref.q_mean[b, h], kf[b, h], ref.k_mean[b, h], sm_scale,
+                                            ldo=NB * 128, order="fma")
+            ks = (kf[b, h] - ref.k_mean[b, h][None, :]).astype(np.float32).astype(np.float64)
+            absdot = np.abs(ref.q_mean[b, h].astype(np.float64)) @ np.abs(ks).T  # [NB, N]
+            bound = (D + 2) * 2.0 ** -24 * kap * absdot + 2.0 ** -149
             g = got[b, h][:, :N]
-            w = want[:, :N]
             if causal:  # blocks I < J are not written (the mask hides them)
                 J = np.arange(N) // 128
                 keep = np.arange(NB)[:, None] >= J[None, :]
             else:
                 keep = np.ones_like(g, dtype=bool)
-            U.assert_same(f"mean term b{b} h{h}", g[keep], w[keep])
+            err = np.abs(g.astype(np.float64) - want[:, :N].astype(np.float64))
+            assert np.all(err[keep] <= bound[keep]), (b, h, float((err - bound)[keep].max()))
+            U.assert_same(f"mean term b{b} h{h}", g[keep], want_fma[:, :N][keep])
             if not causal:
                 assert np.all(got[b, h][:, N:] == 0)  # keys past N
 
