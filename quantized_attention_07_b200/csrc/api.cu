@@ -366,7 +366,7 @@ sage_status_t sage_quantize_ex(const void* q, const void* k, const void* v, int 
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes) ||
       !q_scale || !k_scale || !k_mean || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !aligned16(v_scale))) return SAGE_ERR_INVALID_ARG;
   const bool tok = qk_gran == SAGE_QK_PER_TOKEN;
   const Layout L = dense_layout(B, H, N, D, fp8, Hkv, tok);
   if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
@@ -404,7 +404,7 @@ sage_status_t sage_attn_quantized_ex(const int8_t* q_codes, const float* q_scale
   if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !aligned16(k_scale) ||
       !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+  if (fp8 ? (!aligned16(v_codes) || !aligned16(v_scale)) : (!aligned16(v) || !in_dtype_ok(v_dt)))
     return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
   return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
@@ -437,7 +437,7 @@ sage_status_t sage_quantize_sq(const void* q, const void* k, const void* v, int 
       !q_scale || !aligned16(q_mean) || !k_scale || !aligned16(k_mean) || !aligned16(q_bias) ||
       !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !aligned16(v_scale))) return SAGE_ERR_INVALID_ARG;
   const Layout L = dense_layout(B, H, N, D, fp8, Hkv);
   if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
   return quantize_dense_sq(q, k, v, in_dt, B, H, N, D, pv_mode, causal, sm_scale, q_codes,
@@ -458,7 +458,7 @@ sage_status_t sage_attn_quantized_sq(const int8_t* q_codes, const float* q_scale
   if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !k_scale || !aligned16(q_bias) ||
       !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+  if (fp8 ? (!aligned16(v_codes) || !aligned16(v_scale)) : (!aligned16(v) || !in_dtype_ok(v_dt)))
     return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
   return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
@@ -478,7 +478,7 @@ sage_status_t sage_attn_quantized_dump_s(const int8_t* q_codes, const float* q_s
   if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !aligned16(k_scale) ||
       !aligned16(out) || !aligned16(ws) || !aligned16(s_out))
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+  if (fp8 ? (!aligned16(v_codes) || !aligned16(v_scale)) : (!aligned16(v) || !in_dtype_ok(v_dt)))
     return SAGE_ERR_INVALID_ARG;
   if (!fp8 && v_dt != SAGE_F16) return SAGE_ERR_UNSUPPORTED;
   if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
@@ -501,7 +501,7 @@ sage_status_t sage_selftest_attn_timeout(const int8_t* q_codes, const float* q_s
   if (!aligned16(q_codes) || !aligned16(k_codes) || !q_scale || !aligned16(k_scale) ||
       !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 ? (!aligned16(v_codes) || !v_scale) : (!aligned16(v) || !in_dtype_ok(v_dt)))
+  if (fp8 ? (!aligned16(v_codes) || !aligned16(v_scale)) : (!aligned16(v) || !in_dtype_ok(v_dt)))
     return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < kHeader) return SAGE_ERR_WORKSPACE;
   return attn_dense(q_codes, q_scale, k_codes, k_scale, v, v_codes, v_scale, out, v_dt, out_dt, B,
@@ -644,7 +644,7 @@ sage_status_t sage_quantize_varlen(const void* q, const void* k, const void* v, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes) ||
       !q_scale || !k_scale || !k_mean || !aligned16(ws) || !cu_seqlens)
     return SAGE_ERR_INVALID_ARG;
-  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !v_scale)) return SAGE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(v) || !aligned16(v_codes) || !aligned16(v_scale))) return SAGE_ERR_INVALID_ARG;
   const Layout L = varlen_layout(total_tokens, batch, H, D, fp8);
   if (ws_bytes < L.scratch_end) return SAGE_ERR_WORKSPACE;
   if (total_tokens == 0) return SAGE_OK;

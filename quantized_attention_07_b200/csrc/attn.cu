@@ -653,6 +653,10 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
     for (int i = 0; i < D; ++i) o32[i] = 0.0f;
   }
   const int limit = p.causal ? min(w.n, row + 1) : w.n;  // keys >= limit are masked
+  // deltaK of the next 128-key block, loaded one block ahead so that its
+  // global load is not on the path from S to the exponentials
+  float kd_next = 0.0f;
+  if (!TOK && nsub > 0) kd_next = __ldg(p.k_scale + w.ks_idx0);
 
   // sub-tile ii: are all its keys unmasked for every row of the tile?
   auto full_of = [&](int ii) -> bool {
@@ -705,8 +709,8 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
     const int b = I & 1;
     const uint32_t tS = tS0 + SUB * b;
     if (!TOK && (i & 1) == 0) {  // a new 128-key quantisation block: its delta
-      const float kd = __ldg(p.k_scale + w.ks_idx0 + i / 2);
-      c = __fmul_rn(__fmul_rn(qd, kd), p.kappa);
+      c = __fmul_rn(__fmul_rn(qd, kd_next), p.kappa);
+      if (i + 2 < nsub) kd_next = __ldg(p.k_scale + w.ks_idx0 + i / 2 + 1);
     }
     if (!wait_s(i)) return false;
     const int key0 = i * SUB;
@@ -808,23 +812,21 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
       if (lead && i > 0) {
         // two-level accumulation, once per 128-key block: O32 <- alpha_{b-1}
         // O32 + Part_{b-1}, the partial of both halves of the previous block
-        // (its P.V completed before this block's QK^T landed), 64 columns of
-        // the partial per TMEM round trip
+        // (its P.V completed before this block's QK^T landed)
         if (!wait_bar(B, &B->o_full[t], (I - 1) & 1, p.status, true)) return false;
         ptx::tc_fence_after();
         const float2 a2 = make_float2(alpha_prev, alpha_prev);
 #pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb) {
-          uint32_t pv[64];
-          ptx::tmem_ld32(tO + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
-          ptx::tmem_ld32(tO + 64 * cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+        for (int cb = 0; cb < D / 32; ++cb) {  // 32 columns per round trip: o32 is live
+          uint32_t pv[32];
+          ptx::tmem_ld32(tO + 32 * cb, pv);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 64; k += 2) {
-            const float2 x = __ffma2_rn(a2, make_float2(o32[64 * cb + k], o32[64 * cb + k + 1]),
+          for (int k = 0; k < 32; k += 2) {
+            const float2 x = __ffma2_rn(a2, make_float2(o32[32 * cb + k], o32[32 * cb + k + 1]),
                                         make_float2(__uint_as_float(pv[k]), __uint_as_float(pv[k + 1])));
-            o32[64 * cb + k] = x.x;
-            o32[64 * cb + k + 1] = x.y;
+            o32[32 * cb + k] = x.x;
+            o32[32 * cb + k + 1] = x.y;
           }
         }
       }
@@ -845,32 +847,46 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
   const bool store = row < w.n;
   const long long orow = (w.out_row0 + (long long)row * w.out_stride) * D;
   const float inv_l = 1.0f / l;
+  // 16 (FP8 P.V: its fp32 accumulator is live too) or 32 columns at a time
+  constexpr int EC = PV8 ? 16 : 32;
 #pragma unroll
-  for (int cc = 0; cc < D / 32; ++cc) {
-    uint32_t ov[32];
-    ptx::tmem_ld32(tO + 32 * cc, ov);
+  for (int cc = 0; cc < D / EC; ++cc) {
+    uint32_t ov[EC];
+    if constexpr (EC == 16) ptx::tmem_ld16(tO + EC * cc, ov);
+    else ptx::tmem_ld32(tO + EC * cc, ov);
+    float vf[PV8 ? EC : 1];
+    if constexpr (PV8) {  // the chunk's V scales, as vector loads
+      const float4* vs = reinterpret_cast<const float4*>(p.v_scale + w.vs_idx * D + EC * cc);
+#pragma unroll
+      for (int k = 0; k < EC / 4; ++k) {
+        const float4 f = __ldg(vs + k);
+        vf[4 * k] = f.x;
+        vf[4 * k + 1] = f.y;
+        vf[4 * k + 2] = f.z;
+        vf[4 * k + 3] = f.w;
+      }
+    }
     ptx::tmem_wait_ld();
-    float o[32];
+    float o[EC];
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
+    for (int k = 0; k < EC; ++k) {
       if constexpr (PV8) {
-        const float acc = __fmaf_rn(alpha_prev, o32[32 * cc + k], __uint_as_float(ov[k]));
-        const float vf = __ldg(p.v_scale + w.vs_idx * D + 32 * cc + k);
-        o[k] = __fmul_rn(__fmul_rn(acc, vf), inv_l);
+        const float acc = __fmaf_rn(alpha_prev, o32[EC * cc + k], __uint_as_float(ov[k]));
+        o[k] = __fmul_rn(__fmul_rn(acc, vf[k]), inv_l);
       } else {
         o[k] = __fmul_rn(__uint_as_float(ov[k]), inv_l);
       }
     }
     if (!store) continue;
     if (p.out_dt == SAGE_F32) {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + 32 * cc);
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + EC * cc);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) dst[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+      for (int k = 0; k < EC / 4; ++k) dst[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + 32 * cc);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + EC * cc);
       const bool ob = p.out_dt == SAGE_BF16;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < EC / 8; ++k) {
         uint32_t u[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
