@@ -186,17 +186,20 @@ _host_state: dict = {}
 
 def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                   causal: bool = False, sm_scale: Optional[float] = None, pv_mode: str = "fp16",
-                  qk_gran: str = "block", device=None, chunks: int = 8) -> torch.Tensor:
+                  qk_gran: str = "block", device=None, chunks: int = 16,
+                  slots: int = 3) -> torch.Tensor:
     """attn_fwd for dense tensors that live in (pinned) host memory, result
     written to the host tensor `out`.
 
     The problem is cut into about `chunks` pieces along (batch, key/value head
     group) -- independent problems, since every statistic of the method (K
-    mean, deltas, V scales, softmax) is per (sequence, head) -- and each piece
-    is uploaded, computed and downloaded on its own stream, two pieces in
-    flight: piece c+1's upload and piece c-1's download run while piece c
-    computes.  The result equals one attn_fwd over the whole input.  Returns
-    `out`; the work is ordered before anything later on the current stream.
+    mean, deltas, V scales, softmax) is per (sequence, head).  Each piece is
+    uploaded on a copy-in stream, computed on its slot's own stream with its
+    own workspace, and downloaded on a copy-out stream; `slots` pieces are in
+    flight.  So uploads, downloads and compute overlap, and a piece's kernels
+    fill the SMs that the previous piece's last work items leave idle.  The
+    result equals one attn_fwd over the whole input.  Returns `out`; the work
+    is ordered before anything later on the current stream.
     """
     if q.is_cuda or k.is_cuda or v.is_cuda or out.is_cuda:
         raise ValueError("attn_fwd_host takes host tensors")
@@ -204,6 +207,8 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
         raise ValueError("q, out must be [B, H, N, D] and k, v one [B, Hkv, N, D] shape")
     if not all(t.is_contiguous() for t in (q, k, v, out)):
         raise ValueError("tensors must be contiguous")
+    if slots < 2:
+        raise ValueError("slots must be at least 2")
     B, H, N, D = q.shape
     Hkv = k.shape[1]
     if H % Hkv:
@@ -215,45 +220,52 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
     while Hkv % per:
         per -= 1
     pieces = [(b, h0) for b in range(B) for h0 in range(0, Hkv, per)]
-    key = (dev.index, q.dtype, out.dtype, per * g, per, N, D)
+    key = (dev.index, q.dtype, out.dtype, per * g, per, N, D, slots, pv_mode, qk_gran)
     st = _host_state.get(key)
     if st is None:
         e = dict(dtype=q.dtype, device=dev)
+        nbytes = int(_lib.load().sage_workspace_bytes_ex(1, per * g, per, N, D, _pv(pv_mode),
+                                                         _gran(qk_gran)))
         st = _host_state[key] = dict(
-            q=[torch.empty((1, per * g, N, D), **e) for _ in range(2)],
-            k=[torch.empty((1, per, N, D), **e) for _ in range(2)],
-            v=[torch.empty((1, per, N, D), **e) for _ in range(2)],
-            o=[torch.empty((1, per * g, N, D), dtype=out.dtype, device=dev) for _ in range(2)],
+            q=[torch.empty((1, per * g, N, D), **e) for _ in range(slots)],
+            k=[torch.empty((1, per, N, D), **e) for _ in range(slots)],
+            v=[torch.empty((1, per, N, D), **e) for _ in range(slots)],
+            o=[torch.empty((1, per * g, N, D), dtype=out.dtype, device=dev) for _ in range(slots)],
+            ws=[Workspace(nbytes, dev) for _ in range(slots)],
+            comp=[torch.cuda.Stream(dev) for _ in range(slots)],
             s_in=torch.cuda.Stream(dev), s_out=torch.cuda.Stream(dev),
-            ev=[[torch.cuda.Event() for _ in range(3)] for _ in range(2)])
+            ev=[[torch.cuda.Event() for _ in range(3)] for _ in range(slots)])
     cur = torch.cuda.current_stream(dev)
-    s_in, s_out = st["s_in"], st["s_out"]
-    s_in.wait_stream(cur)   # ordered after everything enqueued before the call
-    s_out.wait_stream(cur)
+    s_in, s_out, comp = st["s_in"], st["s_out"], st["comp"]
+    for s_ in (s_in, s_out, *comp):  # ordered after everything enqueued before the call
+        s_.wait_stream(cur)
     for c, (b, h0) in enumerate(pieces):
-        slot = c & 1
+        slot = c % slots
         ev_in, ev_comp, ev_out = st["ev"][slot]
         hq = slice(h0 * g, (h0 + per) * g)
         hk = slice(h0, h0 + per)
         with torch.cuda.stream(s_in):
-            if c >= 2:
+            if c >= slots:
                 s_in.wait_event(ev_comp)          # the slot's inputs were consumed
             st["q"][slot][0].copy_(q[b, hq], non_blocking=True)
             st["k"][slot][0].copy_(k[b, hk], non_blocking=True)
             st["v"][slot][0].copy_(v[b, hk], non_blocking=True)
             ev_in.record(s_in)
-        cur.wait_event(ev_in)
-        if c >= 2:
-            cur.wait_event(ev_out)                # the slot's last result was downloaded
-        attn_fwd(st["q"][slot], st["k"][slot], st["v"][slot], causal=causal, sm_scale=sm_scale,
-                 pv_mode=pv_mode, out=st["o"][slot], qk_gran=qk_gran)
-        ev_comp.record(cur)
+        cs = comp[slot]
+        cs.wait_event(ev_in)
+        if c >= slots:
+            cs.wait_event(ev_out)                 # the slot's last result was downloaded
+        with torch.cuda.stream(cs):
+            attn_fwd(st["q"][slot], st["k"][slot], st["v"][slot], causal=causal,
+                     sm_scale=sm_scale, pv_mode=pv_mode, out=st["o"][slot],
+                     workspace=st["ws"][slot], qk_gran=qk_gran)
+            ev_comp.record(cs)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp)
             out[b, hq].copy_(st["o"][slot][0], non_blocking=True)
             ev_out.record(s_out)
-    cur.wait_stream(s_out)
-    cur.wait_stream(s_in)
+    for s_ in (s_out, s_in, *comp):
+        cur.wait_stream(s_)
     return out
 
 

@@ -1,6 +1,7 @@
-"""attn_fwd_host (pinned host inputs and output, uploads / compute / downloads
-of independent head groups overlapped on three streams) returns exactly what
-one attn_fwd over the device copies returns."""
+"""attn_fwd_host (pinned host inputs and output; uploads, compute and
+downloads of independent head groups overlapped, each slot with its own
+compute stream and workspace) returns exactly what one attn_fwd over the
+device copies returns."""
 from __future__ import annotations
 
 import pytest
@@ -12,20 +13,22 @@ from quantized_attention_07_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,H,Hkv,N,D,dtype,causal,pv_mode,gran,chunks", [
-    (2, 4, 4, 300, 64, "fp16", False, "fp16", "block", 8),
-    (1, 8, 2, 513, 128, "bf16", True, "fp8", "block", 3),
-    (1, 6, 6, 257, 128, "fp16", True, "fp16", "token", 64),
-    (3, 2, 1, 129, 64, "bf16", False, "fp8", "token", 1),
+@pytest.mark.parametrize("B,H,Hkv,N,D,dtype,causal,pv_mode,gran,chunks,slots", [
+    (2, 4, 4, 300, 64, "fp16", False, "fp16", "block", 8, 3),
+    (1, 8, 2, 513, 128, "bf16", True, "fp8", "block", 3, 2),
+    (1, 6, 6, 257, 128, "fp16", True, "fp16", "token", 64, 4),
+    (3, 2, 1, 129, 64, "bf16", False, "fp8", "token", 1, 3),
+    (2, 8, 8, 640, 128, "fp16", False, "fp16", "block_sq", 16, 3),
 ])
-def test_host_pipeline_equals_device_call(B, H, Hkv, N, D, dtype, causal, pv_mode, gran, chunks):
+def test_host_pipeline_equals_device_call(B, H, Hkv, N, D, dtype, causal, pv_mode, gran, chunks,
+                                          slots):
     q, k, v = W.make_dense(B, H, N, D, dtype, bias_sigma=3.0, seed=N + H)
     k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
     hq, hk, hv = (t.pin_memory() for t in (q, k, v))
     hout = torch.empty((B, H, N, D), dtype=torch.float32).pin_memory()
     for _ in range(2):  # the second call reuses the cached buffers and streams
         sage.attn_fwd_host(hq, hk, hv, hout, causal=causal, pv_mode=pv_mode, qk_gran=gran,
-                           chunks=chunks)
+                           chunks=chunks, slots=slots)
         torch.cuda.synchronize()
         dev = torch.device("cuda")
         want = sage.attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=causal, pv_mode=pv_mode,
