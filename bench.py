@@ -316,12 +316,15 @@ def mufu_bound_ms(wl, seqlens, sm_mhz: float) -> float:
     return scores / (16.0 * SM_COUNT * sm_mhz * 1e6) * 1e3
 
 
-def side_config(name: str, dev, local: int, steps: int = 20) -> dict:
+def side_config(name: str, dev, local: int, min_s: float = 0.6) -> dict:
     """One side workload: its step timed like the headline (whole step and the
-    attention stage alone), against the tensor peak and the MUFU floor."""
+    attention stage alone), against the tensor peak and the MUFU floor.  The
+    timed region lasts at least min_s seconds, so the clock sampler sees it."""
     wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl)
     stage1, stage2, _, ws, _, _ = build_step(wl, inp, dev)
+    probe_ms, _, _, _ = time_steps(stage1, stage2, ws, dev, 5, 3, local, 1)
+    steps = int(min(5000, max(20, min_s * 1e3 / max(probe_ms / 5, 1e-3))))
     total_ms, attn_ms, _, clocks = time_steps(stage1, stage2, ws, dev, steps, 3, local, 1)
     ops = W.attention_ops(wl, inp.seqlens)
     pk = peaks()
