@@ -193,7 +193,8 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
 
     The problem is cut into about `chunks` pieces along (batch, key/value head
     group) -- independent problems, since every statistic of the method (K
-    mean, deltas, V scales, softmax) is per (sequence, head).  Each piece is
+    mean, deltas, V scales, softmax) is per (sequence, head) -- each with at
+    least as many work items as the GPU has SMs.  Each piece is
     uploaded on a copy-in stream, computed on its slot's own stream with its
     own workspace, and downloaded on a copy-out stream; `slots` pieces are in
     flight.  So uploads, downloads and compute overlap, and a piece's kernels
@@ -215,10 +216,15 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
         raise ValueError("Hkv must divide H")
     g = H // Hkv
     dev = torch.device(device if device is not None else "cuda")
-    # key/value heads per piece (a divisor of Hkv), about `chunks` pieces in all
-    per = max(1, (B * Hkv) // max(1, chunks))
+    # key/value heads per piece: a divisor of Hkv, about `chunks` pieces in
+    # all, but at least one full wave of the attention kernel's work items
+    # (pairs of 128-row query tiles) per piece
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    items_per_kv_head = g * ((N + 2 * BLOCK - 1) // (2 * BLOCK))
+    per = max(1, (B * Hkv) // max(1, chunks), -(-sms // items_per_kv_head))
+    per = min(per, Hkv)
     while Hkv % per:
-        per -= 1
+        per += 1
     pieces = [(b, h0) for b in range(B) for h0 in range(0, Hkv, per)]
     key = (dev.index, q.dtype, out.dtype, per * g, per, N, D, slots, pv_mode, qk_gran)
     st = _host_state.get(key)
