@@ -381,11 +381,10 @@ def run_ours(args, rank, world, local):
 
         def e2e_step():
             if wl.varlen:
-                dq, dk, dv = (x.to(dev, non_blocking=True) for x in (hq, hk, hv))
-                dcu = hcu.to(dev, non_blocking=True)
-                o = sage.attn_fwd_varlen(dq, dk, dv, dcu, max(inp.seqlens), causal=wl.causal,
-                                         pv_mode=wl.pv_mode, workspace=ws)
-                hout.copy_(o, non_blocking=True)
+                # pieces of consecutive sequences: uploads, compute and
+                # downloads overlapped
+                sage.attn_fwd_varlen_host(hq, hk, hv, hcu, hout, causal=wl.causal,
+                                          pv_mode=wl.pv_mode, qk_gran=wl.qk_gran, device=dev)
             else:
                 # uploads, compute and downloads of independent head groups overlapped
                 sage.attn_fwd_host(hq, hk, hv, hout, causal=wl.causal, pv_mode=wl.pv_mode,

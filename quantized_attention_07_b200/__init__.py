@@ -8,7 +8,7 @@ binding of that library.
 """
 from .api import (  # noqa: F401
     BLOCK, PV_COSINE_THRESHOLD, PV_MODES, Quantized, SageError, Workspace, alloc_quantized,
-    attn_fwd, attn_fwd_host, attn_fwd_varlen, attn_quantized, attn_ref_rows, calibrate_pv_modes,
+    attn_fwd, attn_fwd_host, attn_fwd_varlen, attn_fwd_varlen_host, attn_quantized, attn_ref_rows, calibrate_pv_modes,
     attn_quantized_dump_s, choose_pv_mode, cosine_similarity, pv_mode_similarity, qk_int8_tiles,
     quant_qk, quantize,
     quantize_varlen, sageattn, sageattn_qk_int8_pv_fp16_cuda, sageattn_qk_int8_pv_fp8_cuda,

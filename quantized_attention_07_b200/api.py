@@ -275,6 +275,117 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
     return out
 
 
+def attn_fwd_varlen_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         cu_seqlens: torch.Tensor, out: torch.Tensor, causal: bool = False,
+                         sm_scale: Optional[float] = None, pv_mode: str = "fp16",
+                         qk_gran: str = "block", device=None, chunks: int = 8,
+                         slots: int = 3) -> torch.Tensor:
+    """attn_fwd_varlen for packed tensors that live in (pinned) host memory,
+    result written to the host tensor `out` ([T, H, D]).
+
+    The batch is cut into about `chunks` pieces of consecutive sequences with
+    about equal token counts: each piece is a contiguous range of rows and an
+    independent packed problem (every statistic of the method is per
+    sequence), with its own cu_seqlens.  Pieces are uploaded on a copy-in
+    stream, computed on their slot's stream with the slot's workspace and
+    downloaded on a copy-out stream, `slots` pieces in flight.  The result
+    equals one attn_fwd_varlen over the whole batch.  cu_seqlens: host int32
+    [batch + 1].  Returns `out`; the work is ordered before anything later on
+    the current stream.
+    """
+    if any(t.is_cuda for t in (q, k, v, out, cu_seqlens)):
+        raise ValueError("attn_fwd_varlen_host takes host tensors")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or out.shape != q.shape:
+        raise ValueError("q, out must be [T, H, D] and k, v one [T, Hkv, D] shape")
+    if not all(t.is_contiguous() for t in (q, k, v, out)):
+        raise ValueError("tensors must be contiguous")
+    if cu_seqlens.dtype != torch.int32 or slots < 2:
+        raise ValueError("cu_seqlens must be int32 and slots at least 2")
+    T, H, D = q.shape
+    Hkv = k.shape[1]
+    cu = [int(x) for x in cu_seqlens.tolist()]
+    batch = len(cu) - 1
+    if batch < 1 or cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must rise from 0 to T")
+    dev = torch.device(device if device is not None else "cuda")
+    # consecutive sequences, about T / chunks tokens per piece
+    pieces, s0 = [], 0
+    for c in range(max(1, chunks)):
+        goal = T * (c + 1) / max(1, chunks)
+        s1 = s0
+        while s1 < batch and (s1 == s0 or cu[s1 + 1] <= goal or c == chunks - 1):
+            s1 += 1
+        if s1 > s0:
+            pieces.append((s0, s1))
+        s0 = s1
+        if s0 >= batch:
+            break
+    if s0 < batch:
+        pieces.append((s0, batch))
+    tmax = max(cu[b] - cu[a] for a, b in pieces)
+    bmax = max(b - a for a, b in pieces)
+    key = ("varlen", dev.index, q.dtype, out.dtype, H, Hkv, D, tmax, bmax, slots)
+    st = _host_state.get(key)
+    if st is None:
+        e = dict(dtype=q.dtype, device=dev)
+        st = _host_state[key] = dict(
+            q=[torch.empty((tmax, H, D), **e) for _ in range(slots)],
+            k=[torch.empty((tmax, Hkv, D), **e) for _ in range(slots)],
+            v=[torch.empty((tmax, Hkv, D), **e) for _ in range(slots)],
+            o=[torch.empty((tmax, H, D), dtype=out.dtype, device=dev) for _ in range(slots)],
+            ws=[Workspace(256, dev) for _ in range(slots)],
+            comp=[torch.cuda.Stream(dev) for _ in range(slots)],
+            s_in=torch.cuda.Stream(dev), s_out=torch.cuda.Stream(dev),
+            ev=[[torch.cuda.Event() for _ in range(3)] for _ in range(slots)])
+    cur = torch.cuda.current_stream(dev)
+    s_in, s_out, comp = st["s_in"], st["s_out"], st["comp"]
+    for s_ in (s_in, s_out, *comp):  # ordered after everything enqueued before the call
+        s_.wait_stream(cur)
+    # every piece's own cu_seqlens (rebased to its first token), one upload
+    offs, local = [], []
+    for a, b in pieces:
+        offs.append(len(local))
+        local += [x - cu[a] for x in cu[a:b + 1]]
+    with torch.cuda.stream(s_in):
+        cu_d = torch.tensor(local, dtype=torch.int32).pin_memory().to(dev, non_blocking=True)
+    for c, (a, b) in enumerate(pieces):
+        slot = c % slots
+        ev_in, ev_comp, ev_out = st["ev"][slot]
+        t0, t1 = cu[a], cu[b]
+        n = t1 - t0
+        lens = [cu[i + 1] - cu[i] for i in range(a, b)]
+        with torch.cuda.stream(s_in):
+            if c >= slots:
+                s_in.wait_event(ev_comp)          # the slot's inputs were consumed
+            if n:
+                st["q"][slot][:n].copy_(q[t0:t1], non_blocking=True)
+                st["k"][slot][:n].copy_(k[t0:t1], non_blocking=True)
+                st["v"][slot][:n].copy_(v[t0:t1], non_blocking=True)
+            ev_in.record(s_in)
+        cs = comp[slot]
+        cs.wait_event(ev_in)
+        if c >= slots:
+            cs.wait_event(ev_out)                 # the slot's last result was downloaded
+        with torch.cuda.stream(cs):
+            if n:
+                attn_fwd_varlen(st["q"][slot][:n], st["k"][slot][:n], st["v"][slot][:n],
+                                cu_d[offs[c]:offs[c] + b - a + 1], max(lens), causal=causal,
+                                sm_scale=sm_scale, pv_mode=pv_mode, out=st["o"][slot][:n],
+                                workspace=st["ws"][slot], qk_gran=qk_gran)
+            ev_comp.record(cs)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp)
+            if n:
+                out[t0:t1].copy_(st["o"][slot][:n], non_blocking=True)
+            ev_out.record(s_out)
+    for s_ in (s_out, s_in, *comp):
+        cur.wait_stream(s_)
+    cu_d.record_stream(cur)
+    for cs in comp:
+        cu_d.record_stream(cs)
+    return out
+
+
 def attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                     max_seqlen: int, causal: bool = False, sm_scale: Optional[float] = None,
                     pv_mode: str = "fp16", out_dtype: Optional[torch.dtype] = None,
