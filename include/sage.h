@@ -159,11 +159,24 @@ sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* o
  * b_Ij = fp32(kappa * qmean_I . fp32(k_j - kmean)), the dot product as fp32
  * fused multiply-adds in channel order (within (D + 2) 2^-24 kappa
  * sum_d |qmean_d k~_jd| of the exact value), then arg = y - m.
- * Its workspace also holds qmean and b (B*H*NB*(D + NB*128) floats).
- *   ws : at least sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, qk_gran).
+ * Its workspace also holds qmean (B*H*NB*D floats) and b for R query blocks
+ * at a time (B*H*R*NB*128 floats): the call computes b of query blocks
+ * [0, R), attends those query tiles, then the next R, so that the workspace
+ * grows with N*R rather than N^2/128.  sage_workspace_bytes_ex gives R = as
+ * many blocks as fit 256 MiB (at least 2, at most NB).  A call takes R = the
+ * most blocks its ws_bytes holds, an even count unless it is all NB, and
+ * fails with SAGE_ERR_WORKSPACE below R = 2.  The output does not depend on
+ * R: every term and every query tile is computed as in one pass.
+ *   ws : at least sage_workspace_bytes_ex(B, H, Hkv, N, D, pv_mode, qk_gran),
+ *        or, with Q smoothing, sage_workspace_bytes_sq(..., R) for a chosen R.
  * sage_attn_fwd(...) = sage_attn_fwd_ex(..., Hkv = H, ..., SAGE_QK_PER_BLOCK).
  */
 size_t sage_workspace_bytes_ex(int B, int H, int Hkv, int N, int D, int pv_mode, int qk_gran);
+/* Workspace of sage_attn_fwd_ex with SAGE_QK_PER_BLOCK_SMOOTH_Q whose mean term
+ * holds q_blocks_per_chunk query blocks (R above; clamped to NB; an even
+ * count when below NB).  Returns 0 for invalid arguments. */
+size_t sage_workspace_bytes_sq(int B, int H, int Hkv, int N, int D, int pv_mode,
+                               int q_blocks_per_chunk);
 sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
                                int in_dt, int out_dt, int B, int H, int Hkv, int N, int D,
                                int causal, float sm_scale, int pv_mode, int qk_gran, void* ws,

@@ -26,6 +26,7 @@ SIGNATURES = {
     "sage_workspace_bytes_gqa": ([_I, _I, _I, _I, _I, _I], _SZ),
     "sage_workspace_bytes_varlen_gqa": ([_I, _I, _I, _I, _I, _I], _SZ),
     "sage_workspace_bytes_varlen_sq": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
+    "sage_workspace_bytes_sq": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sage_workspace_bytes_varlen_ex": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sage_attn_fwd_varlen_ex": ([_P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                  _I, _P, _SZ, _P], _I),

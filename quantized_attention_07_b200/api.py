@@ -132,13 +132,17 @@ def workspace_bytes_varlen(total_tokens: int, batch: int, H: int, D: int,
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
              sm_scale: Optional[float] = None, pv_mode: str = "fp16",
              out_dtype: Optional[torch.dtype] = None, out: Optional[torch.Tensor] = None,
-             workspace: Optional[Workspace] = None, qk_gran: str = "block") -> torch.Tensor:
+             workspace: Optional[Workspace] = None, qk_gran: str = "block",
+             sq_chunk_blocks: Optional[int] = None) -> torch.Tensor:
     """SageAttention forward over dense [B, H, N, D] fp16/bf16 tensors.
 
     k and v may have fewer heads than q ([B, Hkv, N, D], H a multiple of Hkv):
     grouped-query attention, query head h reading key/value head h // (H // Hkv).
     qk_gran: "block" (one Q/K delta per 128 tokens), "token" (one per token) or
     "block_sq" (per block, with each Q block smoothed by its channel mean).
+    sq_chunk_blocks ("block_sq"): query blocks whose mean term the workspace
+    holds at a time (even, or at least all of them); by default as many as fit
+    256 MiB.  The output does not depend on it.
     """
     _need_cuda_contig(q, k, v)
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
@@ -158,12 +162,20 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     lib = _lib.load()
     gran = _gran(qk_gran)
     if gran:
-        ws = _workspace(q.device, int(lib.sage_workspace_bytes_ex(B, H, Hkv, N, D, mode, gran)),
-                        workspace)
+        if gran == 2 and sq_chunk_blocks is not None:
+            nbytes = int(lib.sage_workspace_bytes_sq(B, H, Hkv, N, D, mode, int(sq_chunk_blocks)))
+            if nbytes == 0:
+                raise ValueError("sq_chunk_blocks must be even or at least ceil(N/128)")
+        else:
+            nbytes = int(lib.sage_workspace_bytes_ex(B, H, Hkv, N, D, mode, gran))
+        ws = _workspace(q.device, nbytes, workspace)
+        # with a chosen chunk, exactly the bytes that size it (a cached
+        # workspace may be larger, and the call would hold more blocks)
         _check(lib.sage_attn_fwd_ex(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q.dtype),
             _dtype_code(out.dtype, True), B, H, Hkv, N, D, int(bool(causal)), scale, mode, gran,
-            ws.ptr, ws.nbytes, _stream(q.device)), "sage_attn_fwd_ex")
+            ws.ptr, nbytes if sq_chunk_blocks is not None else ws.nbytes, _stream(q.device)),
+            "sage_attn_fwd_ex")
     elif Hkv == H:
         ws = _workspace(q.device, workspace_bytes(B, H, N, D, pv_mode), workspace)
         _check(lib.sage_attn_fwd(

@@ -1,6 +1,7 @@
 // C ABI of libsageb200.so: argument validation, workspace layout, launches,
 // and the device status word.  Nothing here allocates device memory; every
 // buffer is the caller's.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -24,7 +25,7 @@ cudaError_t launch_quant_q_smooth(const SeqLayout& L, dim3 grid, int D, bool bf1
 cudaError_t launch_q_smooth_bias(const SeqLayout& L, dim3 grid, int H, int Hkv, int D, bool bf16,
                                  int causal, float kappa, const void* k, const float* k_mean,
                                  const float* q_mean, float* bias, long long head_stride,
-                                 const long long* sq_off, cudaStream_t st);
+                                 const long long* sq_off, int qb0, int qrows, cudaStream_t st);
 cudaError_t launch_qk_tiles(const int8_t* qc, const int8_t* kc, int BH, int NP, int D,
                             const int32_t* tiles, int n, int32_t* out, uint32_t* status,
                             cudaStream_t st);
@@ -66,6 +67,7 @@ struct Layout {
   size_t q_codes, k_codes, q_scale, k_scale, k_mean;   // quantised operands
   size_t v_codes, v_scale;
   size_t q_mean, q_bias, sq_off;                      // Q smoothing
+  int sq_rows;                                        // dense Q smoothing: query blocks per head in q_bias
   long long bias_head_stride;                         // varlen Q smoothing: floats per head
   size_t scratch_end, total;
 };
@@ -75,8 +77,17 @@ struct Layout {
 // key/value head for the launch that quantises K (and Q when Hkv = H);
 // sync_q: the work counter of the separate Q launch when Hkv < H.
 // gran: a sage_qk_gran_t (per-token deltas; Q smoothing adds the block means
-// and the per-key mean term).
-Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, int gran = SAGE_QK_PER_BLOCK) {
+// and the per-key mean term of sq_rows query blocks per head, by default as
+// many as fit kSqTermCap bytes, at least 2 and at most all of them).
+constexpr size_t kSqTermCap = size_t(256) << 20;
+
+int sq_rows_default(size_t BH, size_t NB) {
+  const size_t row = BH * NB * BLK * 4, fit = (kSqTermCap / row) & ~size_t(1);
+  return (int)std::min(NB, std::max<size_t>(2, fit));
+}
+
+Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, int gran = SAGE_QK_PER_BLOCK,
+                    int sq_rows = 0) {
   const bool per_token = gran == SAGE_QK_PER_TOKEN;
   const size_t BH = (size_t)B * H, BK = (size_t)B * Hkv, NB = ((size_t)N + BLK - 1) / BLK,
                NP = NB * BLK, NS = per_token ? NP : NB;  // deltas per head
@@ -97,8 +108,9 @@ Layout dense_layout(int B, int H, int N, int D, bool fp8, int Hkv, int gran = SA
     L.v_scale = o; o += al(BK * D * 4);
   }
   if (gran == SAGE_QK_PER_BLOCK_SMOOTH_Q) {
+    L.sq_rows = sq_rows > 0 ? (int)std::min<size_t>(sq_rows, NB) : sq_rows_default(BH, NB);
     L.q_mean = o; o += al(BH * NB * D * 4);
-    L.q_bias = o; o += al(BH * NB * NP * 4);
+    L.q_bias = o; o += al(BH * (size_t)L.sq_rows * NP * 4);
   }
   L.total = o;
   return L;
@@ -224,7 +236,7 @@ sage_status_t quantize_dense_sq(const void* q, const void* k, const void* v, int
                                 int8_t* q_codes, float* q_scale, float* q_mean, int8_t* k_codes,
                                 float* k_scale, float* k_mean, uint8_t* v_codes, float* v_scale,
                                 float* q_bias, void* ws, const Layout& L, cudaStream_t st,
-                                int Hkv) {
+                                int Hkv, bool with_bias = true) {
   const bool fp8 = pv_mode == SAGE_PV_FP8, bf16 = in_dt == SAGE_BF16;
   sage_status_t r = clear_scratch(ws, L, fp8, st);
   if (r != SAGE_OK) return r;
@@ -241,9 +253,10 @@ sage_status_t quantize_dense_sq(const void* q, const void* k, const void* v, int
   if (e == cudaSuccess)
     e = launch_quant_q_smooth(S, dim3(NB, (unsigned)(B * H)), D, bf16, q, q_codes, q_scale,
                               q_mean, at<uint32_t>(ws, 0), st);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && with_bias)  // the term of every query block
     e = launch_q_smooth_bias(S, dim3(NB, (unsigned)(B * H)), H, Hkv, D, bf16, causal ? 1 : 0,
-                             kappa_of(sm_scale, D), k, k_mean, q_mean, q_bias, 0, nullptr, st);
+                             kappa_of(sm_scale, D), k, k_mean, q_mean, q_bias, 0, nullptr, 0,
+                             (int)NB, st);
   if (e == cudaErrorNotSupported) return SAGE_ERR_UNSUPPORTED;
   return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
 }
@@ -254,7 +267,8 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
                          int N, int D, int causal, float sm_scale, int pv_mode, void* ws,
                          cudaStream_t st, int Hkv, int per_token = 0,
                          const float* q_bias = nullptr, int32_t* s_dump = nullptr,
-                         long long wait_limit = 0, int fault_skip_k = 0) {
+                         long long wait_limit = 0, int fault_skip_k = 0, int pair0 = 0,
+                         int npairs = -1, int bias_nb = -1) {
   const bool fp8 = pv_mode == SAGE_PV_FP8;
   AttnLaunch A{};
   A.p.H = H;
@@ -264,7 +278,11 @@ sage_status_t attn_dense(const int8_t* q_codes, const float* q_scale, const int8
   A.p.N = N;
   A.p.BH = B * H;
   A.p.NB = (N + BLK - 1) / BLK;
-  A.p.NPAIR = (N + 2 * BLK - 1) / (2 * BLK);
+  // query tile pairs [pair0, pair0 + npairs) (all by default); q_bias holds
+  // bias_nb query blocks per head from block 2*pair0
+  A.p.NPAIR = npairs < 0 ? (N + 2 * BLK - 1) / (2 * BLK) : npairs;
+  A.p.pair0 = pair0;
+  A.p.bias_nb = bias_nb < 0 ? A.p.NB : bias_nb;
   A.p.causal = causal ? 1 : 0;
   A.p.kappa = kappa_of(sm_scale, D);
   A.p.q_scale = q_scale;
@@ -514,6 +532,16 @@ size_t sage_workspace_bytes_ex(int B, int H, int Hkv, int N, int D, int pv_mode,
   return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv, qk_gran).total;
 }
 
+size_t sage_workspace_bytes_sq(int B, int H, int Hkv, int N, int D, int pv_mode,
+                               int q_blocks_per_chunk) {
+  if (!dense_args_ok(B, H, N, D, pv_mode) || !gqa_heads_ok(H, Hkv)) return 0;
+  const int NB = (N + BLK - 1) / BLK;
+  if (q_blocks_per_chunk < 1 || (q_blocks_per_chunk < NB && (q_blocks_per_chunk & 1))) return 0;
+  return dense_layout(B, H, N, D, pv_mode == SAGE_PV_FP8, Hkv, SAGE_QK_PER_BLOCK_SMOOTH_Q,
+                      q_blocks_per_chunk)
+      .total;
+}
+
 sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int in_dt,
                                int out_dt, int B, int H, int Hkv, int N, int D, int causal,
                                float sm_scale, int pv_mode, int qk_gran, void* ws,
@@ -524,23 +552,47 @@ sage_status_t sage_attn_fwd_ex(const void* q, const void* k, const void* v, void
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
     return SAGE_ERR_INVALID_ARG;
   const bool fp8 = pv_mode == SAGE_PV_FP8, tok = qk_gran == SAGE_QK_PER_TOKEN;
-  const Layout L = dense_layout(B, H, N, D, fp8, Hkv, qk_gran);
-  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  Layout L = dense_layout(B, H, N, D, fp8, Hkv, qk_gran);
   cudaStream_t st = as_stream(stream);
   if (qk_gran == SAGE_QK_PER_BLOCK_SMOOTH_Q) {
+    // The mean term of as many query blocks as the workspace holds at a time
+    // (an even count unless all fit): each chunk's term, then attention on
+    // that chunk's query tiles.  Every value is the one of a single pass.
+    const int NB = (N + BLK - 1) / BLK;
+    const size_t row = (size_t)B * H * NB * BLK * 4;
+    int rows = ws_bytes > L.q_bias ? (int)std::min<size_t>((ws_bytes - L.q_bias) / row, NB) : 0;
+    if (rows < NB) rows &= ~1;
+    if (rows < 1) return SAGE_ERR_WORKSPACE;
+    L = dense_layout(B, H, N, D, fp8, Hkv, qk_gran, rows);
+    if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
     sage_status_t r = quantize_dense_sq(
         q, k, v, in_dt, B, H, N, D, pv_mode, causal, sm_scale, at<int8_t>(ws, L.q_codes),
         at<float>(ws, L.q_scale), at<float>(ws, L.q_mean), at<int8_t>(ws, L.k_codes),
         at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
         fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr, fp8 ? at<float>(ws, L.v_scale) : nullptr,
-        at<float>(ws, L.q_bias), ws, L, st, Hkv);
-    if (r != SAGE_OK) return r;
-    return attn_dense(at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
-                      at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), v,
-                      fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
-                      fp8 ? at<float>(ws, L.v_scale) : nullptr, out, in_dt, out_dt, B, H, N, D,
-                      causal, sm_scale, pv_mode, ws, st, Hkv, 2, at<float>(ws, L.q_bias));
+        at<float>(ws, L.q_bias), ws, L, st, Hkv, false);
+    SeqLayout S{};
+    S.varlen = 0;
+    S.N = N;
+    S.H = H;
+    for (int qb0 = 0; r == SAGE_OK && qb0 < NB; qb0 += rows) {
+      const int qr = std::min(rows, NB - qb0);
+      // with a causal mask, key tiles past the chunk's last query block add nothing
+      const cudaError_t e = launch_q_smooth_bias(
+          S, dim3((unsigned)(causal ? qb0 + qr : NB), (unsigned)(B * H)), H, Hkv, D,
+          in_dt == SAGE_BF16, causal ? 1 : 0, kappa_of(sm_scale, D), k, at<float>(ws, L.k_mean),
+          at<float>(ws, L.q_mean), at<float>(ws, L.q_bias), 0, nullptr, qb0, rows, st);
+      if (e != cudaSuccess) return cuda_fail(e, "quantisation launch");
+      r = attn_dense(at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
+                     at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), v,
+                     fp8 ? at<uint8_t>(ws, L.v_codes) : nullptr,
+                     fp8 ? at<float>(ws, L.v_scale) : nullptr, out, in_dt, out_dt, B, H, N, D,
+                     causal, sm_scale, pv_mode, ws, st, Hkv, 2, at<float>(ws, L.q_bias), nullptr,
+                     0, 0, qb0 / 2, (qr + 1) / 2, rows);
+    }
+    return r;
   }
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   sage_status_t r = quantize_dense(
       q, k, v, in_dt, B, H, N, D, pv_mode, at<int8_t>(ws, L.q_codes), at<float>(ws, L.q_scale),
       at<int8_t>(ws, L.k_codes), at<float>(ws, L.k_scale), at<float>(ws, L.k_mean),
@@ -611,7 +663,7 @@ static sage_status_t varlen_stage1(const void* q, const void* k, const void* v, 
       e = launch_q_smooth_bias(S, dim3((unsigned)TB, H), H, Hkv, D, bf16, causal ? 1 : 0,
                                kappa_of(sm_scale, D), k, k_mean, at<float>(ws, L.q_mean),
                                at<float>(ws, L.q_bias), L.bias_head_stride,
-                               at<long long>(ws, L.sq_off), st);
+                               at<long long>(ws, L.sq_off), 0, 0, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e, "quantisation launch");
   }
   // grouped-query: K (, V) over the Hkv key/value heads, then Q over the H

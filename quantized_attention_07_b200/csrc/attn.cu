@@ -175,11 +175,11 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p, int idx) {
   if (!p.varlen) {
     int bh;
     if (p.causal) {  // heaviest pairs first
-      pair = p.NPAIR - 1 - idx / p.BH;
+      pair = p.pair0 + p.NPAIR - 1 - idx / p.BH;
       bh = idx % p.BH;
     } else {         // head-major: a head's K^/V stay hot in L2
       bh = idx / p.NPAIR;
-      pair = idx % p.NPAIR;
+      pair = p.pair0 + idx % p.NPAIR;
     }
     n = p.N;
     // grouped-query attention: query head h of batch b reads key/value head
@@ -199,7 +199,7 @@ __device__ __forceinline__ Work decode_work(const AttnParams& p, int idx) {
     w.out_stride = 1;
     w.vs_idx = bkv;
     w.bias_ld = (long long)p.NB * BLK;
-    w.bias_row0 = ((long long)bh * p.NB + 2 * pair) * w.bias_ld;
+    w.bias_row0 = ((long long)bh * p.bias_nb + 2 * (pair - p.pair0)) * w.bias_ld;
   } else {
     const int h = idx / p.PM;
     const int item = idx - h * p.PM;

@@ -9,11 +9,13 @@ struct AttnParams {
   int H, N, BH;          // dense: N, BH = B*H (query heads)
   int Hkv;               // dense: key/value heads (H is a multiple; query head h reads h / (H/Hkv))
   int NB;                // dense: key blocks per head = ceil(N/128)
-  int NPAIR;             // dense: query tile pairs per head = ceil(N/256)
+  int NPAIR;             // dense: query tile pairs per head in this launch (all: ceil(N/256))
+  int pair0;             // dense: first query tile pair of the launch
+  int bias_nb;           // dense per_token 2: query blocks per head in q_bias, from block 2*pair0
   int causal;
   int per_token;         // 1: one delta per token ([BH][NP] / [B*Hkv][NP]), not per block;
                          // 2: per block, Q smoothed (q_bias holds the mean term)
-  const float* q_bias;   // per_token 2: dense [BH][NB][NB*128] fp32, kappa applied;
+  const float* q_bias;   // per_token 2: dense [BH][bias_nb][NB*128] fp32, kappa applied;
                          // varlen: sequence s, head h at h*bias_head_stride + sq_off[s]*128
   const long long* sq_off;        // varlen per_token 2: [batch+1] prefix of ceil(n_s/128)^2
   long long bias_head_stride;     // varlen per_token 2: floats per query head

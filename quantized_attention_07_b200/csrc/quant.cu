@@ -520,31 +520,37 @@ __global__ void __launch_bounds__(THREADS) quant_q_smooth_kernel(
 struct BiasPos {
   int n;                 // sequence length
   int nb;                // its query / key blocks
+  int qb0, qend;          // query blocks [qb0, qend) written (varlen: all)
   int J;                 // key tile within the sequence
   const uint16_t* k0;    // key token 0 of the sequence, this key/value head
   long long k_stride;    // elements between consecutive tokens of k
   const float* kmean;    // [D] of the key/value head
   const float* qm;       // [nb][D] block means of the query head
-  float* out;            // [nb][nb*128] term of the (sequence, query head)
+  float* out;            // rows of the (sequence, query head), row I - qb0 for block I, nb*128 floats each
 };
 
-// Dense: grid (NB, B*H); varlen: grid (TBmax, H) over the global key blocks.
+// Dense: grid (key tiles, B*H), the term of query blocks [qb0, qb0 + qrows)
+// into [B*H][qrows][NB*128]; varlen: grid (TBmax, H) over the global key
+// blocks, every query block.
 __device__ __forceinline__ bool bias_pos(const SeqLayout& L, int Hq, int Hkv, int D,
                                          const void* k, const float* k_mean, const float* q_mean,
                                          float* bias, long long head_stride,
-                                         const long long* sq_off, BiasPos& P) {
+                                         const long long* sq_off, int qb0, int qrows,
+                                         BiasPos& P) {
   if (!L.varlen) {
     const int NB = (L.N + BLK - 1) / BLK;
     const int bh = blockIdx.y, b = bh / Hq, h = bh - b * Hq;
     const int bkv = b * Hkv + h / (Hq / Hkv);
     P.n = L.N;
     P.nb = NB;
+    P.qb0 = qb0;
+    P.qend = min(NB, qb0 + qrows);
     P.J = blockIdx.x;
     P.k0 = static_cast<const uint16_t*>(k) + (long long)bkv * L.N * D;
     P.k_stride = D;
     P.kmean = k_mean + (long long)bkv * D;
     P.qm = q_mean + (long long)bh * NB * D;
-    P.out = bias + (long long)bh * NB * NB * BLK;
+    P.out = bias + (long long)bh * qrows * NB * BLK;
     return true;
   }
   const int gb = blockIdx.x, h = blockIdx.y;
@@ -556,6 +562,8 @@ __device__ __forceinline__ bool bias_pos(const SeqLayout& L, int Hq, int Hkv, in
   const int hk = h / (Hq / Hkv);
   P.n = __ldg(L.cu + s + 1) - t0;
   P.nb = (P.n + BLK - 1) / BLK;
+  P.qb0 = 0;
+  P.qend = P.nb;
   P.J = gb - b0;
   P.k0 = static_cast<const uint16_t*>(k) + ((long long)t0 * Hkv + hk) * D;
   P.k_stride = (long long)Hkv * D;
@@ -580,11 +588,13 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
     SeqLayout L, int H, int Hkv, int causal, float kappa, const void* __restrict__ k,
     const float* __restrict__ k_mean, const float* __restrict__ q_mean,
-    float* __restrict__ bias, long long head_stride, const long long* __restrict__ sq_off) {
+    float* __restrict__ bias, long long head_stride, const long long* __restrict__ sq_off,
+    int qb0, int qrows) {
   constexpr int G = 8;                 // query blocks per pass
   __shared__ __align__(16) float s_qm[D][G];  // means of G blocks, channel-major
   BiasPos P;
-  if (!bias_pos(L, H, Hkv, D, k, k_mean, q_mean, bias, head_stride, sq_off, P)) return;
+  if (!bias_pos(L, H, Hkv, D, k, k_mean, q_mean, bias, head_stride, sq_off, qb0, qrows, P))
+    return;
   const int jl = P.J * BLK + threadIdx.x;  // key within the sequence
   float kt[D];
   if (jl < P.n) {
@@ -608,11 +618,11 @@ __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
   }
   const long long NP = (long long)P.nb * BLK;
   float* out = P.out + jl;
-  for (int I0 = causal ? P.J : 0; I0 < P.nb; I0 += G) {
+  for (int I0 = max(causal ? P.J : 0, P.qb0); I0 < P.qend; I0 += G) {
     __syncthreads();  // the previous group's means are no longer read
     for (int x = threadIdx.x; x < G * D; x += 128) {
       const int g = x / D, d = x - g * D;
-      s_qm[d][g] = I0 + g < P.nb ? __ldg(P.qm + (long long)(I0 + g) * D + d) : 0.0f;
+      s_qm[d][g] = I0 + g < P.qend ? __ldg(P.qm + (long long)(I0 + g) * D + d) : 0.0f;
     }
     __syncthreads();
     float2 acc[G / 2];
@@ -631,9 +641,9 @@ __global__ void __launch_bounds__(128) q_smooth_bias_kernel(
     }
 #pragma unroll
     for (int g2 = 0; g2 < G / 2; ++g2) {
-      if (I0 + 2 * g2 < P.nb) out[(long long)(I0 + 2 * g2) * NP] = __fmul_rn(acc[g2].x, kappa);
-      if (I0 + 2 * g2 + 1 < P.nb)
-        out[(long long)(I0 + 2 * g2 + 1) * NP] = __fmul_rn(acc[g2].y, kappa);
+      const int I = I0 + 2 * g2 - P.qb0;  // row in the output
+      if (I0 + 2 * g2 < P.qend) out[(long long)I * NP] = __fmul_rn(acc[g2].x, kappa);
+      if (I0 + 2 * g2 + 1 < P.qend) out[(long long)(I + 1) * NP] = __fmul_rn(acc[g2].y, kappa);
     }
   }
 }
@@ -1329,18 +1339,20 @@ cudaError_t launch_quant_q_smooth(const SeqLayout& L, dim3 grid, int D, bool bf1
   return cudaGetLastError();
 }
 
-// The per-key term of Q smoothing (fp32, kappa applied).  Dense: grid (NB,
-// B*H), k [B*Hkv, N, D], k_mean [B*Hkv, D], q_mean [B*H, NB, D], bias
-// [B*H][NB][NB*128].  Varlen: grid (TBmax, H), k [T, Hkv, D], k_mean
-// [batch, Hkv, D], q_mean [H, TBmax, D], bias of sequence s and head h at
-// h*head_stride + sq_off[s]*128, [nb_s][nb_s*128].
+// The per-key term of Q smoothing (fp32, kappa applied).  Dense: grid (key
+// tiles, B*H), k [B*Hkv, N, D], k_mean [B*Hkv, D], q_mean [B*H, NB, D], the
+// term of query blocks [qb0, qb0 + qrows) into bias [B*H][qrows][NB*128].
+// Varlen: grid (TBmax, H), k [T, Hkv, D], k_mean [batch, Hkv, D], q_mean
+// [H, TBmax, D], bias of sequence s and head h at h*head_stride +
+// sq_off[s]*128, [nb_s][nb_s*128] (qb0, qrows unused).
 cudaError_t launch_q_smooth_bias(const SeqLayout& L, dim3 grid, int H, int Hkv, int D, bool bf16,
                                  int causal, float kappa, const void* k, const float* k_mean,
                                  const float* q_mean, float* bias, long long head_stride,
-                                 const long long* sq_off, cudaStream_t st) {
+                                 const long long* sq_off, int qb0, int qrows, cudaStream_t st) {
 #define SAGE_B(DD, BB)                                                                        \
   q_smooth_bias_kernel<DD, BB><<<grid, 128, 0, st>>>(L, H, Hkv, causal, kappa, k, k_mean,    \
-                                                     q_mean, bias, head_stride, sq_off)
+                                                     q_mean, bias, head_stride, sq_off, qb0, \
+                                                     qrows)
   if (D == 64) {
     if (bf16) SAGE_B(64, true); else SAGE_B(64, false);
   } else {

@@ -183,6 +183,22 @@ def test_q_smoothing_sizes_and_validation(lib):
     sq = lib.sage_workspace_bytes_ex(B, H, H, N, D, 1, 2)
     assert sq == plain + al(B * H * NB * D * 4) + al(B * H * NB * NB * 128 * 4)
     assert lib.sage_workspace_bytes_ex(B, H, H, N, D, 1, 3) == 0        # unknown granularity
+    # the mean term of R query blocks at a time: R even below NB, clamped to NB
+    sqr = lambda r: lib.sage_workspace_bytes_sq(B, H, H, N, D, 1, r)
+    assert sqr(NB) == sqr(NB + 5) == sq
+    assert sqr(2) == plain + al(B * H * NB * D * 4) + al(B * H * 2 * NB * 128 * 4)
+    assert sqr(4) - sqr(2) == B * H * 2 * NB * 128 * 4
+    assert sqr(3) == sqr(0) == sqr(-2) == 0
+    assert lib.sage_workspace_bytes_sq(B, H, H, N, 96, 1, 2) == 0      # D
+    # by default the term holds as many query blocks as fit 256 MiB (at least 2)
+    Bl, Hl, Nl, Dl = 1, 32, 32768, 128
+    NBl = Nl // 128
+    row = Bl * Hl * NBl * 128 * 4                                      # 4 MiB per query block
+    base = lib.sage_workspace_bytes_ex(Bl, Hl, Hl, Nl, Dl, 0, 0)
+    assert lib.sage_workspace_bytes_ex(Bl, Hl, Hl, Nl, Dl, 0, 2) == (
+        base + al(Bl * Hl * NBl * Dl * 4) + (256 << 20) // row * row)
+    huge = lib.sage_workspace_bytes_ex(1, 1024, 1024, 1 << 20, 64, 0, 2)
+    assert huge == lib.sage_workspace_bytes_sq(1, 1024, 1024, 1 << 20, 64, 0, 2)
     # packed: 0 through the _ex query (no max_seqlen), sized by the _sq query
     assert lib.sage_workspace_bytes_varlen_ex(5000, 4, 8, 8, 128, 1, 2) == 0
     short = lib.sage_workspace_bytes_varlen_sq(5000, 4, 1000, 8, 8, 128, 1)

@@ -143,6 +143,30 @@ def test_split_stages_equal_fused_call():
             sage.attn_quantized(qz, v, causal=not causal)
 
 
+@pytest.mark.parametrize("B,H,Hkv,N,D,dtype,pv_mode,chunks", [
+    (1, 4, 2, 1000, 128, "bf16", "fp16", (2, 4, 6)),      # NB 8
+    (2, 3, 3, 700, 64, "fp16", "fp8", (2, 4)),            # NB 6, ragged tail
+    (1, 2, 1, 1290, 64, "bf16", "fp8", (2, 8, 10)),       # NB 11: odd, last chunk one block
+    (1, 2, 2, 129, 128, "fp16", "fp16", (2,)),            # NB 2: one chunk of both
+])
+def test_chunked_mean_term_equals_one_pass(B, H, Hkv, N, D, dtype, pv_mode, chunks):
+    """With a workspace that holds the mean term of R query blocks at a time,
+    the fused call runs R blocks' term and attention per chunk; every value
+    is that of the single pass, so the outputs are equal bit for bit."""
+    q, k, v = (t.cuda() for t in _inputs(B, H, Hkv, N, D, dtype, seed=N + H))
+    for causal in (False, True):
+        one = sage.attn_fwd(q, k, v, causal=causal, pv_mode=pv_mode, out_dtype=torch.float32,
+                            qk_gran="block_sq")
+        for r in chunks:
+            got = sage.attn_fwd(q, k, v, causal=causal, pv_mode=pv_mode,
+                                out_dtype=torch.float32, qk_gran="block_sq", sq_chunk_blocks=r)
+            torch.cuda.synchronize()
+            sage.sync_status()
+            assert torch.equal(got, one), (causal, r)
+    with pytest.raises(ValueError):
+        sage.attn_fwd(q, k, v, qk_gran="block_sq", sq_chunk_blocks=3 if N > 500 else -1)
+
+
 def test_smoothing_helps_with_a_query_offset():
     """A channel offset in Q (sigma 3, as K's) eats most of the int8 range of the
     unsmoothed codes; with smoothing the result is closer to fp64 attention."""
