@@ -1008,9 +1008,6 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
       int pass, u, b;
       item_of(x, NB, U, lag, parts, pass, u, b);
       const int nt = tensors_of(pass, parts, FP8);
-      for (int t = 1; t < nt; ++t) ok = ptx::mbar_wait(&full[(cidx + t) % NS], ((cidx + t) / NS) & 1) && ok;
-      ok = ptx::named_all<256>(ok);
-      if (!ok) break;
       BlockPos P;
       dense_block_pos(L, u, b, P);
       const long long chan0 = (long long)P.seq * D;
@@ -1022,7 +1019,17 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
 
       const bool full_blk = P.rows == BLK;
       uint4 rg[T::NIT];
-      auto take = [&](int t) {  // slab t of this item -> registers; free the slot
+      // slab t of this item -> registers; free the slot.  Slabs after the
+      // first are awaited only here, so their copies overlap the work on the
+      // earlier ones; a wait that runs out marks the abort, which the next
+      // loop's uniform check sees (this item's values are then garbage).
+      auto await_slab = [&](int t) {
+        if (t > 0 && !ptx::mbar_wait(&full[(cidx + t) % NS], ((cidx + t) / NS) & 1)) {
+          set_status(status, ST_TIMEOUT);
+          s_abort = 1;
+        }
+      };
+      auto take = [&](int t) {  // (after await_slab(t))
         if (full_blk) slab_to_regs<D, true>(slab(t), P.rows, rg);
         else slab_to_regs<D, false>(slab(t), P.rows, rg);
         release_slot(empty_of(t));
@@ -1053,6 +1060,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
         }
         // K: exact fixed-point channel sums
         if (has_kv) {
+          await_slab(tk);
           take(tk);
           float2 hi[4], fr[4];
           uint32_t absbits;
@@ -1094,6 +1102,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
         }
         // V: per-channel max|v| (FP8 P.V only)
         if (FP8 && has_kv) {
+          await_slab(tk + 1);
           take(tk + 1);
           uint32_t m2[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
@@ -1158,6 +1167,7 @@ __global__ void __launch_bounds__(Stream<D>::THREADS, Stream<D>::CTAS_PER_SM) qu
         }
         // V: FP8 E4M3 codes with a per-channel scale
         if constexpr (FP8) {
+          await_slab(1);  // its V scale factors come with the slot
           const float* side = s_side[(cidx + 1) % NS];  // V scale factors
           float2 sv[4];
 #pragma unroll
