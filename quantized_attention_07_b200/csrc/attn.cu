@@ -27,8 +27,12 @@
 // over both.  With fp16 P it is taken per 64-key sub-tile and moves only when
 // a row's sub-tile maximum exceeds it by more than 8, so O rescales are rare.
 //
-// TMEM columns (512): S_0[0] [0,64) S_0[1] [64,128) S_1[0] [128,192)
-// S_1[1] [192,256) O_0 [256,256+D) O_1 [256+D,256+2D).
+// TMEM columns (512): NBUF S buffers of 64 columns per tile, S_t[b] at
+// [64(NBUF t + b), +64), then O_0 at 128 NBUF and O_1 D columns later.  D = 128
+// keeps two buffers (O takes 256 columns); D = 64 has room for three, so
+// QK^T runs three sub-tiles ahead of the softmax instead of two (with FP8
+// P.V the first half of a 128-key block then finds the second half's S
+// computed before P.V of the previous block's second half completes).
 //
 // Method steps (SageAttention pages): INT8 QK^T with the per-block deltas
 // ("SageAttention -- brand new attention", quantisation intro step 3 and
@@ -78,6 +82,17 @@ struct Cfg {
   static constexpr bool block_max(bool bf16v) { return PV8 || bf16v; }
   static constexpr float tau(bool bf16v) { return block_max(bf16v) ? 0.0f : 8.0f; }
 
+  // S buffers per tile: 2 x NBUF x 64 columns of S and 2 x D of O fit 512.
+  // Three at D = 64 (measured +1.0 % on the FP8 video shape, +1.5 % with
+  // per-token deltas); with Q smoothing the longer-lived buffer indices cost
+  // registers and it measured 0.3 % slower, so two.
+  static constexpr int NBUF = (D == 64 && GR != 2) ? 3 : 2;
+  static constexpr uint32_t TO = 2 * NBUF * SUB;        // first O column
+  static_assert(TO + 2 * D <= 512, "TMEM columns");
+  // S buffer of a tile's I-th sub-tile, and the parity of its barrier phase
+  // (I >= 0; unsigned, so NBUF = 2 is a mask and a shift)
+  static __device__ __forceinline__ int sbuf(int I) { return (int)((unsigned)I % NBUF); }
+  static __device__ __forceinline__ uint32_t sphase(int I) { return ((unsigned)I / NBUF) & 1u; }
   static constexpr int QT = BLK * D;                    // bytes of one int8 Q^/K^ tile
   static constexpr int VT = BLK * D * (PV8 ? 1 : 2);    // bytes of one V tile
   // per stage, on the K barrier: the 128 per-token K deltas (GR 1), or the
@@ -104,12 +119,15 @@ struct Cfg {
   static constexpr int PV_STEPS = SUB / PV_KSTEP;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(NS >= 2, "need at least two stages");
+  // QK^T of sub-tile i + NBUF reads stage (i + NBUF)/2 before stage i/2 is
+  // released: NBUF/2 + 2 stages resident at once
+  static_assert(NS >= NBUF / 2 + 2, "stages for the S lookahead");
 };
 
 struct Bars {
   uint64_t q_full, done[2];
-  uint64_t s_full[2][2];   // [tile][S buffer]: QK^T of a sub-tile landed
-  uint64_t p_full[2][2];   // P of a sub-tile written, O rescaled (128 softmax threads)
+  uint64_t s_full[2][3];   // [tile][S buffer]: QK^T of a sub-tile landed
+  uint64_t p_full[2][3];   // P of a sub-tile written, O rescaled (128 softmax threads)
   uint64_t o_full[2];      // P.V of a sub-tile completed
   uint64_t o_done[2];      // the last P.V of a query tile of an item completed
   uint64_t q_empty;        // both MMA warps' last QK^T of the item completed (2 commits)
@@ -377,8 +395,8 @@ __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const
 
 // One warp per query tile issues that tile's MMAs (the whole warp runs the
 // loop; one elected lane issues).  Per 64-key sub-tile i:
-//   wait P_t(i) -> O_t (+)= P_t(i) V_i  ->  S_t(i+2) = Q^_t K^_{i+2}^T
-// Issue order per thread is execution order, so S_t(i+2) never overwrites
+//   wait P_t(i) -> O_t (+)= P_t(i) V_i  ->  S_t(i+NBUF) = Q^_t K^_{i+NBUF}^T
+// Issue order per thread is execution order, so S_t(i+NBUF) never overwrites
 // P_t(i) before P.V has read it.  A 128-key stage is released to the producer
 // when both tiles' warps have committed it (kv_empty counts two arrivals).
 template <int D, bool PV8, bool BF16V, int GR>
@@ -392,7 +410,7 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
           : ptx::instr_desc(1, BF16V ? 1 : 0, BF16V ? 1 : 0, 0, 1, 128, D);
   uint32_t* status = p.status;
   const uint32_t qa = ptx::smem_u32(sQ + t * C::QT);
-  const uint32_t tO = tmem + 256 + D * t;
+  const uint32_t tO = tmem + C::TO + D * t;
   // Counts over the CTA's work items: sub-tiles of this tile (I0: S buffer
   // and barrier phases), stages of the ring (G0), items (n: q_full phase).
   int I0 = 0, G0 = 0, n = 0;
@@ -414,14 +432,14 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
   auto issue_qk = [&](int i) {  // i: sub-tile of the item
     const int I = I0 + i, g = G0 + i / 2;
     const uint32_t kb = ptx::smem_u32(sK + (g % C::NS) * C::QT + (i & 1) * C::K_SUB_BYTES);
-    const uint32_t dst = tmem + 128 * t + SUB * (I & 1);
+    const uint32_t dst = tmem + C::NBUF * SUB * t + SUB * C::sbuf(I);
     if (ptx::elect_one()) {
       const uint64_t a0 = ptx::smem_desc(qa, 16, C::QK_SBO, C::QK_SWZ);
       const uint64_t b0 = ptx::smem_desc(kb, 16, C::QK_SBO, C::QK_SWZ);
 #pragma unroll
       for (int kk = 0; kk < D / 32; ++kk)  // +32 bytes along K per step: +2 in the address field
         ptx::mma_i8_ss(dst, a0 + 2 * kk, b0 + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
-      ptx::mma_commit(&B->s_full[t][I & 1]);
+      ptx::mma_commit(&B->s_full[t][C::sbuf(I)]);
       // after the item's last QK^T the Q^ tiles may be reloaded
       if (i == nt - 1) ptx::mma_commit(&B->q_empty);
     }
@@ -430,7 +448,7 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
   auto issue_pv = [&](int i) {
     const int I = I0 + i, g = G0 + i / 2;
     const uint32_t vb = ptx::smem_u32(sV + (g % C::NS) * C::VT + (i & 1) * C::V_SUB_BYTES);
-    const uint32_t tP = tmem + 128 * t + SUB * (I & 1);
+    const uint32_t tP = tmem + C::NBUF * SUB * t + SUB * C::sbuf(I);
     // an item's first P.V starts O; FP8: each block's first half starts a
     // fresh partial, its second half accumulates into it
     const uint32_t acc0 = PV8 ? ((i & 1) ? 1u : 0u) : (i > 0 ? 1u : 0u);
@@ -478,7 +496,7 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
       if (ptx::elect_one()) ptx::mma_commit(&B->q_empty);
       __syncwarp();
     }
-    for (int i = 0; ok && i < 2 && i < nt; ++i) {
+    for (int i = 0; ok && i < C::NBUF && i < nt; ++i) {
       ok = need_k(G0 + i / 2);
       if (!ok) break;
       ptx::tc_fence_after();
@@ -486,15 +504,15 @@ __device__ void mma_issuer(const AttnParams& p, Bars* B, uint32_t tmem, const ui
     }
     for (int i = 0; ok && i < nt; ++i) {
       ok = need_v(G0 + i / 2) &&
-           wait_bar(B, &B->p_full[t][(I0 + i) & 1], ((I0 + i) / 2) & 1, status, true);
+           wait_bar(B, &B->p_full[t][C::sbuf(I0 + i)], C::sphase(I0 + i), status, true);
       if (!ok) break;
       ptx::tc_fence_after();
       issue_pv(i);
-      if (i + 2 < nt) {
-        ok = need_k(G0 + (i + 2) / 2);
+      if (i + C::NBUF < nt) {
+        ok = need_k(G0 + (i + C::NBUF) / 2);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_qk(i + 2);
+        issue_qk(i + C::NBUF);
       }
       if ((i & 1) || i == nt - 1) ok = release(true);
     }
@@ -642,8 +660,8 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
   const int qt = 2 * w.pair + t;
   const int row = qt * BLK + r;                   // query index in the sequence
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-  const uint32_t tS0 = tmem + 128 * t + lane_off;
-  const uint32_t tO = tmem + 256 + D * t + lane_off;
+  const uint32_t tS0 = tmem + C::NBUF * SUB * t + lane_off;
+  const uint32_t tO = tmem + C::TO + D * t + lane_off;
   const int nsub = t == 0 ? w.nsub0 : w.nsub1;
 
   // deltaQ of this tile's block, or (per token) of this row
@@ -669,12 +687,12 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
   // wait for QK^T of sub-tile ii and load its 64 columns of S
   auto wait_s = [&](int ii) -> bool {
     const int Ii = I0 + ii;
-    if (!wait_bar(B, &B->s_full[t][Ii & 1], (Ii / 2) & 1, p.status, true)) return false;
+    if (!wait_bar(B, &B->s_full[t][C::sbuf(Ii)], C::sphase(Ii), p.status, true)) return false;
     ptx::tc_fence_after();
     return true;
   };
   auto load_s = [&](int ii, uint32_t (&sv)[SUB]) {
-    const uint32_t tS = tS0 + SUB * ((I0 + ii) & 1);
+    const uint32_t tS = tS0 + SUB * C::sbuf(I0 + ii);
 #pragma unroll
     for (int cc = 0; cc < SUB / 32; ++cc)
       ptx::tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
@@ -709,7 +727,7 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
 
   for (int i = 0; i < nsub; ++i) {
     const int I = I0 + i;                        // sub-tile count of this tile over the items
-    const int b = I & 1;
+    const int b = C::sbuf(I);                    // S buffer
     const uint32_t tS = tS0 + SUB * b;
     if (!TOK && (i & 1) == 0) {  // a new 128-key quantisation block: its delta
       c = __fmul_rn(__fmul_rn(qd, kd_next), p.kappa);
@@ -964,7 +982,7 @@ __global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(&B->o_full[t], 1);
       ptx::mbar_init(&B->o_done[t], 1);
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < 3; ++b) {
         ptx::mbar_init(&B->s_full[t][b], 1);
         ptx::mbar_init(&B->p_full[t][b], 128);
       }
