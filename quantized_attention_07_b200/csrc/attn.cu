@@ -19,9 +19,10 @@
 //                in use moves; FP8: fold the previous 128-key block's partial
 //                into an fp32 register accumulator (two-level accumulation).
 //
-// Each query tile owns two 64-column S buffers, so QK^T of sub-tile i+1 runs
-// on the tensor core while the softmax works on sub-tile i, and the two query
-// tiles keep both softmax warpgroups busy.  With FP8 P.V or bf16 P the maximum
+// Each query tile owns two (D = 128) or three (D = 64) 64-column S buffers,
+// so QK^T of the next sub-tiles runs on the tensor core while the softmax
+// works on sub-tile i, and the two query tiles keep both softmax warpgroups
+// busy.  With FP8 P.V or bf16 P the maximum
 // used for p is the plain running maximum over whole 128-key blocks: the first
 // half of a block waits for the second half's S as well and takes the maximum
 // over both.  With fp16 P it is taken per 64-key sub-tile and moves only when
