@@ -237,7 +237,17 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
     per = min(per, Hkv)
     while Hkv % per:
         per += 1
-    pieces = [(b, h0) for b in range(B) for h0 in range(0, Hkv, per)]
+    # (batch, first key/value head, heads).  The job's first and last pieces
+    # are cut down to one head: the first upload is what the pipeline waits
+    # for before any work, the last piece's work and download are what it
+    # waits for after the last upload.
+    pieces = [(b, h0, min(per, Hkv - h0)) for b in range(B) for h0 in range(0, Hkv, per)]
+    if pieces[0][2] > 1:
+        b, h0, nh = pieces[0]
+        pieces[0:1] = [(b, h0, 1), (b, h0 + 1, nh - 1)]
+    if pieces[-1][2] > 1:
+        b, h0, nh = pieces[-1]
+        pieces[-1:] = [(b, h0, nh - 1), (b, h0 + nh - 1, 1)]
     key = (dev.index, q.dtype, out.dtype, per * g, per, N, D, slots, pv_mode, qk_gran)
     st = _host_state.get(key)
     if st is None:
@@ -257,30 +267,32 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
     s_in, s_out, comp = st["s_in"], st["s_out"], st["comp"]
     for s_ in (s_in, s_out, *comp):  # ordered after everything enqueued before the call
         s_.wait_stream(cur)
-    for c, (b, h0) in enumerate(pieces):
+    for c, (b, h0, nh) in enumerate(pieces):
         slot = c % slots
         ev_in, ev_comp, ev_out = st["ev"][slot]
-        hq = slice(h0 * g, (h0 + per) * g)
-        hk = slice(h0, h0 + per)
+        hq = slice(h0 * g, (h0 + nh) * g)
+        hk = slice(h0, h0 + nh)
+        # the slot's buffers hold `per` heads; a piece uses the leading nh
+        sq, sk, sv, so = (st[n][slot][:, :w] for n, w in
+                          (("q", nh * g), ("k", nh), ("v", nh), ("o", nh * g)))
         with torch.cuda.stream(s_in):
             if c >= slots:
                 s_in.wait_event(ev_comp)          # the slot's inputs were consumed
-            st["q"][slot][0].copy_(q[b, hq], non_blocking=True)
-            st["k"][slot][0].copy_(k[b, hk], non_blocking=True)
-            st["v"][slot][0].copy_(v[b, hk], non_blocking=True)
+            sq[0].copy_(q[b, hq], non_blocking=True)
+            sk[0].copy_(k[b, hk], non_blocking=True)
+            sv[0].copy_(v[b, hk], non_blocking=True)
             ev_in.record(s_in)
         cs = comp[slot]
         cs.wait_event(ev_in)
         if c >= slots:
             cs.wait_event(ev_out)                 # the slot's last result was downloaded
         with torch.cuda.stream(cs):
-            attn_fwd(st["q"][slot], st["k"][slot], st["v"][slot], causal=causal,
-                     sm_scale=sm_scale, pv_mode=pv_mode, out=st["o"][slot],
+            attn_fwd(sq, sk, sv, causal=causal, sm_scale=sm_scale, pv_mode=pv_mode, out=so,
                      workspace=st["ws"][slot], qk_gran=qk_gran)
             ev_comp.record(cs)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp)
-            out[b, hq].copy_(st["o"][slot][0], non_blocking=True)
+            out[b, hq].copy_(so[0], non_blocking=True)
             ev_out.record(s_out)
     for s_ in (s_out, s_in, *comp):
         cur.wait_stream(s_)
