@@ -196,6 +196,35 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
 _host_state: dict = {}
 
 
+def dense_host_pieces(B: int, Hkv: int, per: int) -> list:
+    """Pieces (batch, first key/value head, heads) of attn_fwd_host: `per`
+    heads each, except that the job's first and last pieces are cut down to
+    one head -- the first upload is what the pipeline waits for before any
+    work, the last piece's work and download are what it waits for after the
+    last upload."""
+    pieces = [(b, h0, min(per, Hkv - h0)) for b in range(B) for h0 in range(0, Hkv, per)]
+    if pieces[0][2] > 1:
+        b, h0, nh = pieces[0]
+        pieces[0:1] = [(b, h0, 1), (b, h0 + 1, nh - 1)]
+    if pieces[-1][2] > 1:
+        b, h0, nh = pieces[-1]
+        pieces[-1:] = [(b, h0, nh - 1), (b, h0 + nh - 1, 1)]
+    return pieces
+
+
+def varlen_host_order(pieces: list, cu: list) -> list:
+    """Order of attn_fwd_varlen_host's pieces (sequence ranges [a, b)): the one
+    with the fewest tokens first and the next fewest last, for the same reason
+    as dense_host_pieces.  Pieces are independent problems, each writing its
+    own token range of the output, so any order gives the same result."""
+    if len(pieces) <= 2:
+        return list(pieces)
+    order = sorted(range(len(pieces)), key=lambda i: cu[pieces[i][1]] - cu[pieces[i][0]])
+    ends = {order[0], order[1]}
+    return ([pieces[order[0]]] + [x for i, x in enumerate(pieces) if i not in ends]
+            + [pieces[order[1]]])
+
+
 def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                   causal: bool = False, sm_scale: Optional[float] = None, pv_mode: str = "fp16",
                   qk_gran: str = "block", device=None, chunks: int = 16,
@@ -237,17 +266,7 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.
     per = min(per, Hkv)
     while Hkv % per:
         per += 1
-    # (batch, first key/value head, heads).  The job's first and last pieces
-    # are cut down to one head: the first upload is what the pipeline waits
-    # for before any work, the last piece's work and download are what it
-    # waits for after the last upload.
-    pieces = [(b, h0, min(per, Hkv - h0)) for b in range(B) for h0 in range(0, Hkv, per)]
-    if pieces[0][2] > 1:
-        b, h0, nh = pieces[0]
-        pieces[0:1] = [(b, h0, 1), (b, h0 + 1, nh - 1)]
-    if pieces[-1][2] > 1:
-        b, h0, nh = pieces[-1]
-        pieces[-1:] = [(b, h0, nh - 1), (b, h0 + nh - 1, 1)]
+    pieces = dense_host_pieces(B, Hkv, per)
     key = (dev.index, q.dtype, out.dtype, per * g, per, N, D, slots, pv_mode, qk_gran)
     st = _host_state.get(key)
     if st is None:
@@ -346,6 +365,7 @@ def attn_fwd_varlen_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             break
     if s0 < batch:
         pieces.append((s0, batch))
+    pieces = varlen_host_order(pieces, cu)
     tmax = max(cu[b] - cu[a] for a, b in pieces)
     bmax = max(b - a for a, b in pieces)
     key = ("varlen", dev.index, q.dtype, out.dtype, H, Hkv, D, tmax, bmax, slots)
