@@ -99,7 +99,8 @@ struct Cfg {
   // per stage, on the K barrier: the 128 per-token K deltas (GR 1), or the
   // Q-smoothing term of both query tiles for the stage's keys (GR 2)
   static constexpr int KS = GR == 1 ? BLK * 4 : GR == 2 ? 2 * BLK * 4 : 0;
-  static constexpr int AUX = 1024;                      // barriers
+  // barriers (1 KiB), then with FP8 P.V each tile's V scales ([2][D] fp32)
+  static constexpr int AUX = 1024 + (PV8 ? 2 * D * 4 : 0);
   static constexpr int SMEM_BUDGET = 227 * 1024 - 1024 - AUX;
   static constexpr int NS_RAW = (SMEM_BUDGET - 2 * QT) / (QT + VT + KS);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;    // pipeline stages (128 keys each)
@@ -130,6 +131,7 @@ struct Bars {
   uint64_t s_full[2][3];   // [tile][S buffer]: QK^T of a sub-tile landed
   uint64_t p_full[2][3];   // P of a sub-tile written, O rescaled (128 softmax threads)
   uint64_t o_full[2];      // P.V of a sub-tile completed
+  uint64_t vs_full[2];     // FP8: a tile's V scales staged for its epilogue (4 softmax warps)
   uint64_t o_done[2];      // the last P.V of a query tile of an item completed
   uint64_t q_empty;        // both MMA warps' last QK^T of the item completed (2 commits)
   uint64_t item_full[2];   // work-item ring: index published by the producer
@@ -862,10 +864,28 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
   }
 
   // ------------------------------------------------------------ epilogue --
+  // FP8: the tile's V scales, one global load per thread issued before the
+  // wait below, staged in shared memory once per item (rather than 8
+  // dependent global loads per row)
+  [[maybe_unused]] float vsc = 0.0f;
+  if constexpr (PV8) {
+    if (r < D) vsc = __ldg(p.v_scale + w.vs_idx * D + r);
+  }
   // (o_full may lag by two phases here in 16-bit mode; o_done is unambiguous:
   // one phase per item in which this tile has keys)
   if (!wait_bar(B, &B->o_done[t], loop[1] & 1, p.status, true)) return false;
   ptx::tc_fence_after();
+  [[maybe_unused]] const float* svs = reinterpret_cast<const float*>(
+      reinterpret_cast<const uint8_t*>(B) + 1024) + t * D;
+  if constexpr (PV8) {
+    // Every warp of the tile is past the previous item's reads of the buffer:
+    // this item's last P.V, just waited for, needed all four warps' P, which
+    // each stored after its previous epilogue.
+    if (r < D) const_cast<float*>(svs)[r] = vsc;
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&B->vs_full[t]);  // release: the lanes' stores
+    if (!wait_bar(B, &B->vs_full[t], loop[1] & 1, p.status, true)) return false;
+  }
   const bool store = row < w.n;
   const long long orow = (w.out_row0 + (long long)row * w.out_stride) * D;
   const float inv_l = 1.0f / l;
@@ -877,11 +897,11 @@ __device__ __forceinline__ bool softmax_item(const AttnParams& p, const Work& w,
     if constexpr (EC == 16) ptx::tmem_ld16(tO + EC * cc, ov);
     else ptx::tmem_ld32(tO + EC * cc, ov);
     float vf[PV8 ? EC : 1];
-    if constexpr (PV8) {  // the chunk's V scales, as vector loads
-      const float4* vs = reinterpret_cast<const float4*>(p.v_scale + w.vs_idx * D + EC * cc);
+    if constexpr (PV8) {  // the chunk's V scales, from the staged copy
+      const float4* vs = reinterpret_cast<const float4*>(svs + EC * cc);
 #pragma unroll
       for (int k = 0; k < EC / 4; ++k) {
-        const float4 f = __ldg(vs + k);
+        const float4 f = vs[k];
         vf[4 * k] = f.x;
         vf[4 * k + 1] = f.y;
         vf[4 * k + 2] = f.z;
@@ -965,7 +985,7 @@ __global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
   uint8_t* sV = sK + C::NS * C::QT;
   float* sKs = reinterpret_cast<float*>(sV + C::NS * C::VT);  // GR 1: [NS][128] K deltas; GR 2: [NS][2][128] mean terms
   Bars* B = reinterpret_cast<Bars*>(sV + C::NS * (C::VT + C::KS));
-  static_assert(sizeof(Bars) <= C::AUX, "aux layout");
+  static_assert(sizeof(Bars) <= 1024, "aux layout");
 
   const int warp = threadIdx.x / 32;
   const int wg = warp / 4;
@@ -982,6 +1002,7 @@ __global__ void __launch_bounds__(Cfg<D, PV8, GR>::THREADS, 1)
     ptx::mbar_init(&B->done[1], 1);
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(&B->o_full[t], 1);
+      ptx::mbar_init(&B->vs_full[t], 4);
       ptx::mbar_init(&B->o_done[t], 1);
       for (int b = 0; b < 3; ++b) {
         ptx::mbar_init(&B->s_full[t][b], 1);
